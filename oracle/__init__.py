@@ -1,0 +1,15 @@
+"""Oracle for the batch-1 decode path -- TEST INFRASTRUCTURE.
+
+A plain, slow CPU implementation (numpy, float32 or float64) of what the
+decode monokernel computes, written from the definitions and sharing no code
+with the CUDA path.  Only `tests/`, `__graft_entry__.smoke()` and the CPU
+baseline leg of `bench.py` may import it; the library itself never does.
+
+Every function carries its definition in its docstring; `tests/test_oracle_pins.py`
+pins each of them to closed forms, invariants and brute force.  Parity status
+of each function: all pinned (none is "parity unpinned").
+"""
+from .model import (  # noqa: F401
+    DecodeState, OracleModel, apply_rope, argmax_lowest, attention_one_query,
+    causal_attention, rms_norm, rope_cos_sin, rope_inv_freq, silu, top2_margin,
+)
