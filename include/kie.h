@@ -1,0 +1,210 @@
+/*
+ * kie.h -- C ABI of the batch-1 decode monokernel library (libkie.so).
+ *
+ * The library runs batch-1 greedy autoregressive decode of a dense
+ * decoder-only transformer as ONE persistent CUDA kernel per call: every
+ * layer and every token step (RMSNorm, QKV GEMV, RoPE, KV-cache append,
+ * attention over the cache, O projection, SwiGLU FFN GEMVs, LM-head GEMV,
+ * argmax, EOS check) runs inside the resident kernel with no per-op launch
+ * and no host round-trip.  This is the "monokernel" of revietech.ru, "Kog
+ * выжимает максимум из GPU: 3000 токенов/с", section "Что такое monokernel":
+ * one resident program for prefill, decode, LM-head token selection and the
+ * EOS check, without returning to the CPU and without a launch per token.
+ * The projections are matrix-vector products on the vector ALUs, not tensor
+ * cores (same page, section "Архитектура и особенности", "GEMV вместо GEMM").
+ * Token selection is greedy (argmax, lowest index on ties).
+ *
+ * Model (pre-norm decoder; the pages never print the block, this is the
+ * reading the library implements):
+ *   h = E[tok];  per layer:  a = RMSNorm(h; g_attn);  q,k,v = Wq a, Wk a, Wv a;
+ *   RoPE on q and k (pairs (i, i+hd/2), angle pos*base^(-2i/hd), 0-based pos);
+ *   K,V appended to the cache;  o_h = softmax(q_h K_j^T / sqrt(hd)) V_j over
+ *   positions 0..pos with j = h / (n_heads / n_kv_heads);  h += Wo o;
+ *   b = RMSNorm(h; g_ffn);  h += Wd (silu(Wg b) * (Wu b));
+ *   logits = Wlm RMSNorm(h; g_final);  next = argmax(logits).
+ *   RMSNorm(x; g) = g * x / sqrt(mean(x^2) + eps).  No biases, untied head.
+ *
+ * Data layout and ownership
+ *   - All weights are fp16, row-major [out][in] (row r of W holds the
+ *     weights of output r); norm gains are fp16 [d_model].  Wq rows
+ *     h*hd .. h*hd+hd-1 belong to query head h, Wk/Wv rows likewise to KV
+ *     head j, Wo columns follow the same head order.  Shapes:
+ *       tok_emb, lm_head [vocab][d_model]; wq [n_heads*hd][d_model];
+ *       wk, wv [n_kv_heads*hd][d_model]; wo [d_model][n_heads*hd];
+ *       w_gate, w_up [ffn_dim][d_model]; w_down [d_model][ffn_dim].
+ *     Every pointer must be device memory, 16-byte aligned.
+ *   - The KV cache is one device buffer of kie_kv_cache_bytes() bytes,
+ *     16-byte aligned, laid out fp16 [n_layers][2][n_kv_heads][max_seq][hd]
+ *     (index 0 = K after RoPE, 1 = V).
+ *   - The CALLER owns the weights and the KV cache; both must stay valid and
+ *     unmodified (except by this library) until kie_destroy.  The library
+ *     owns its scratch (activation words, attention partials, the RoPE
+ *     table, id buffers), allocated in kie_create and freed in kie_destroy.
+ *
+ * Errors
+ *   Every call returns a kie_status; nothing is thrown across the ABI.
+ *   Calls are synchronous: they return after the device work they enqueue
+ *   on the context's stream has finished.  Device-side waits are bounded:
+ *   a wait that exceeds the timeout (KIE_OPT_TIMEOUT_NS) makes the kernel
+ *   exit and the call return KIE_ERR_TIMEOUT.  After KIE_ERR_TIMEOUT,
+ *   KIE_ERR_PROTOCOL or KIE_ERR_CUDA from a launch the context is failed:
+ *   every later call except kie_destroy, kie_get_stats and kie_last_error
+ *   returns KIE_ERR_STATE.  A context is not thread-safe; use one per host
+ *   thread.
+ */
+#ifndef KIE_H
+#define KIE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define KIE_API __attribute__((visibility("default")))
+#else
+#define KIE_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  KIE_OK = 0,
+  KIE_ERR_INVALID_ARG = 1,  /* NULL pointer, bad size, misaligned pointer */
+  KIE_ERR_UNSUPPORTED = 2,  /* shape the kernel does not handle (see kie_check_desc) */
+  KIE_ERR_CUDA = 3,         /* a CUDA runtime call failed (kie_last_error has the text) */
+  KIE_ERR_CAPACITY = 4,     /* the call would write past max_seq positions */
+  KIE_ERR_STATE = 5,        /* decode before prefill, or the context is failed */
+  KIE_ERR_TIMEOUT = 6,      /* a device-side wait gave up (bounded spin) */
+  KIE_ERR_PROTOCOL = 7      /* a device-side consistency check failed */
+} kie_status;
+
+/* Model shape.  Supported: head_dim 64 or 128; n_heads a multiple of
+ * n_kv_heads with n_heads/n_kv_heads <= 8; d_model, ffn_dim and
+ * n_heads*head_dim multiples of 256; max_seq >= 1; eos_id in [-1, vocab). */
+typedef struct {
+  int32_t n_layers;
+  int32_t d_model;
+  int32_t n_heads;
+  int32_t n_kv_heads;
+  int32_t head_dim;
+  int32_t ffn_dim;
+  int32_t vocab;
+  float rope_base;
+  float rms_eps;
+  int32_t max_seq;   /* capacity of the KV cache in positions */
+  int32_t eos_id;    /* -1: no end-of-sequence id */
+} kie_model_desc;
+
+typedef struct {
+  const void *attn_norm, *wq, *wk, *wv, *wo, *ffn_norm, *w_gate, *w_up, *w_down;
+} kie_layer_weights;
+
+typedef struct {
+  const void *tok_emb;
+  const void *final_norm;
+  const void *lm_head;
+  const kie_layer_weights *layers;  /* HOST array [n_layers] of device pointers;
+                                       copied by kie_create */
+} kie_weights;
+
+typedef struct kie_ctx kie_ctx;
+
+typedef struct {
+  int32_t pos;              /* positions held in the KV cache */
+  int32_t grid;             /* persistent CTAs (one per SM) */
+  int32_t ring_slots;       /* weight-stream ring depth per CTA */
+  int32_t slot_bytes;       /* bytes per ring slot */
+  int32_t smem_bytes;       /* dynamic shared memory per CTA */
+  int32_t last_steps;       /* forward passes run by the last launch */
+  float last_device_ms;     /* device time of the last launch (CUDA events) */
+  uint64_t launches;        /* kernel launches made by this context */
+  /* Per-CTA cycle counters of the last launch, averaged over CTAs:
+   * consumer-side cycles in the persistent loop, cycles spent polling for
+   * other CTAs' outputs (the intra-kernel sync), and cycles spent waiting
+   * for the weight stream to land in shared memory. */
+  double loop_cycles;
+  double sync_wait_cycles;
+  double stream_wait_cycles;
+  double sync_wait_max_frac; /* max over CTAs of sync_wait/loop */
+} kie_stats;
+
+typedef enum {
+  KIE_OPT_TIMEOUT_NS = 1,     /* bound of every device-side wait (default 2e9) */
+  KIE_OPT_SLOT_BYTES = 2,     /* ring slot size in bytes, multiple of 4096; re-plans the ring */
+  KIE_OPT_MIN_SPLIT_LEN = 3,  /* minimum positions per attention split (default 64) */
+  KIE_OPT_FAULT_CTA = 4,      /* test hook: CTA that withholds one publication (-1 off) */
+  KIE_OPT_FAULT_STEP = 5,     /* test hook: step of the withheld publication */
+  KIE_OPT_FAULT_LAYER = 6,    /* test hook: layer of the withheld publication */
+  KIE_OPT_FAULT_STAGE = 7     /* test hook: 0 QKV, 1 O, 2 gate/up, 3 down, 4 LM */
+} kie_option;
+
+/* Bytes of the caller-provided KV cache: 2*n_layers*n_kv_heads*max_seq*head_dim*2.
+ * Returns 0 for a NULL or invalid desc.  Host only. */
+KIE_API size_t kie_kv_cache_bytes(const kie_model_desc *desc);
+
+/* Checks a shape against the limits above.  Host only, no CUDA call. */
+KIE_API kie_status kie_check_desc(const kie_model_desc *desc);
+
+/* Creates a context on the current CUDA device.  `kv_cache` is the
+ * caller's device buffer (kie_kv_cache_bytes bytes); `cuda_stream` is a
+ * cudaStream_t (NULL = legacy default stream).  On success *out receives
+ * the context; on failure *out is set to NULL. */
+KIE_API kie_status kie_create(const kie_model_desc *desc, const kie_weights *weights,
+                      void *kv_cache, void *cuda_stream, kie_ctx **out);
+
+/* Runs the prompt through the model in one launch, writing K/V for
+ * positions 0..n-1 (the session restarts at position 0), and returns in
+ * *first_id the greedy id picked from the last position's logits.
+ * prompt_ids: HOST array [n] with ids in [0, vocab).  first_id may be NULL. */
+KIE_API kie_status kie_prefill(kie_ctx *ctx, const int32_t *prompt_ids, int32_t n,
+                       int32_t *first_id);
+
+/* Runs n_steps greedy decode steps in ONE launch.  Step i feeds the
+ * previous id (the id from kie_prefill or the last id of the previous
+ * decode call for i = 0) at the next position and writes the picked id to
+ * out_ids[i] (HOST array [n_steps]).  Stops after emitting eos_id; *n_out
+ * (nullable) receives the number of ids written.  n_steps = 0 is a no-op. */
+KIE_API kie_status kie_decode(kie_ctx *ctx, int32_t n_steps, int32_t *out_ids,
+                      int32_t *n_out);
+
+/* Teacher-forced decode, one launch: step i feeds ids[i] (HOST [n]) at the
+ * next position instead of the previous pick, and still writes the greedy
+ * pick to out_ids[i] (HOST [n], nullable).  Afterwards the session
+ * continues from the last pick.  Used to compare logits against a
+ * reference on a fixed token stream. */
+KIE_API kie_status kie_decode_forced(kie_ctx *ctx, const int32_t *ids, int32_t n,
+                             int32_t *out_ids);
+
+/* Moves the session back to `pos` positions (1 <= pos <= current): the
+ * next decode step runs at position `pos` and feeds the id that was fed
+ * (or picked) for that position.  K/V of positions >= pos are rewritten by
+ * later steps.  Host-side only. */
+KIE_API kie_status kie_rewind(kie_ctx *ctx, int32_t pos);
+
+/* Logit capture (measurement / parity): while set, every launch writes the
+ * fp32 logits of each step that picks an id to dev_logits[row][vocab],
+ * row = index among those steps, for rows < capacity_rows.  dev_logits is a
+ * device buffer owned by the caller; NULL turns capture off. */
+KIE_API kie_status kie_set_logits_capture(kie_ctx *ctx, float *dev_logits,
+                                  int32_t capacity_rows);
+
+KIE_API kie_status kie_set_option(kie_ctx *ctx, kie_option opt, int64_t value);
+KIE_API kie_status kie_get_stats(const kie_ctx *ctx, kie_stats *out);
+KIE_API const char *kie_status_str(kie_status s);
+/* Text of the last error on this context ("" if none); valid until the next call. */
+KIE_API const char *kie_last_error(const kie_ctx *ctx);
+KIE_API kie_status kie_destroy(kie_ctx *ctx);
+
+/* Host-only planning query (no CUDA call): the unit range [begin, end) that
+ * CTA `cta` of a `grid`-CTA launch owns in GEMV stage `stage` (0 QKV, 1 O,
+ * 2 gate/up, 3 down, 4 LM head).  Units are rows, except RoPE pairs of q/k
+ * rows and gate/up row pairs, which count as one unit of two rows. */
+KIE_API kie_status kie_plan_units(const kie_model_desc *desc, int32_t grid, int32_t stage,
+                          int32_t cta, int32_t *begin, int32_t *end);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KIE_H */

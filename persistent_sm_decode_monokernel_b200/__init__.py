@@ -1,0 +1,99 @@
+"""Batch-1 decode monokernel for B200 (sm_100a).
+
+The compute path is libkie.so (CUDA, C ABI in include/kie.h).  This package
+holds its ctypes binding (`_kie`, same names as the C calls) and `Session`,
+a convenience owner of the device buffers: PyTorch allocates device memory
+and provides the stream, nothing more.
+"""
+from __future__ import annotations
+
+from typing import Mapping, Optional, Sequence
+
+import numpy as np
+
+from . import _kie
+from ._kie import (KieError, kie_check_desc, kie_create, kie_decode, kie_decode_forced,  # noqa: F401
+                   kie_destroy, kie_get_stats, kie_kv_cache_bytes, kie_last_error,
+                   kie_plan_units, kie_prefill, kie_rewind, kie_set_logits_capture,
+                   kie_set_option, load_library, make_desc)
+
+__all__ = ["Session", "KieError", "load_library", "make_desc", "upload_weights"]
+
+
+def upload_weights(host: Mapping[str, np.ndarray], device="cuda"):
+    """Copies host fp16 arrays to device tensors (same names)."""
+    import torch
+    out = {}
+    for k, v in host.items():
+        out[k] = torch.from_numpy(np.ascontiguousarray(v)).to(device)
+    return out
+
+
+class Session:
+    """One decode session on the current CUDA device.
+
+    shape: any object with n_layers, d_model, n_heads, n_kv_heads, head_dim,
+    ffn_dim, vocab, rope_base, rms_eps.  weights: device fp16 tensors named
+    tok_emb, final_norm, lm_head and "{l}.{attn_norm,wq,wk,wv,wo,ffn_norm,
+    w_gate,w_up,w_down}".  The KV cache is allocated here with torch.
+    """
+
+    def __init__(self, shape, weights: Mapping[str, object], max_seq: int, eos_id: int = -1,
+                 stream=None):
+        import torch
+        load_library()
+        self.shape = shape
+        self.desc = make_desc(shape.n_layers, shape.d_model, shape.n_heads, shape.n_kv_heads,
+                              shape.head_dim, shape.ffn_dim, shape.vocab, shape.rope_base,
+                              shape.rms_eps, max_seq, eos_id)
+        st = kie_check_desc(self.desc)
+        if st != _kie.KIE_OK:
+            raise KieError(st, "kie_check_desc")
+        nbytes = kie_kv_cache_bytes(self.desc)
+        self.kv = torch.empty(nbytes // 2, dtype=torch.float16, device="cuda")
+        self.weights = weights
+        if stream is None:
+            stream = torch.cuda.current_stream()
+        self.stream = stream
+        self.ctx = kie_create(self.desc, weights, self.kv, stream.cuda_stream)
+        self._capture = None
+
+    def prefill(self, ids: Sequence[int]) -> int:
+        return kie_prefill(self.ctx, ids)
+
+    def decode(self, n_steps: int, out: Optional[np.ndarray] = None) -> np.ndarray:
+        return kie_decode(self.ctx, n_steps, out)
+
+    def decode_forced(self, ids: Sequence[int]) -> np.ndarray:
+        return kie_decode_forced(self.ctx, ids)
+
+    def rewind(self, pos: int) -> None:
+        kie_rewind(self.ctx, pos)
+
+    def capture_logits(self, rows: int):
+        """Turns logit capture on into a fresh [rows, vocab] fp32 device tensor."""
+        import torch
+        self._capture = torch.empty((rows, self.shape.vocab), dtype=torch.float32, device="cuda")
+        kie_set_logits_capture(self.ctx, self._capture, rows)
+        return self._capture
+
+    def capture_off(self) -> None:
+        kie_set_logits_capture(self.ctx, None, 0)
+        self._capture = None
+
+    def set_option(self, opt: int, value: int) -> None:
+        kie_set_option(self.ctx, opt, value)
+
+    def stats(self):
+        return kie_get_stats(self.ctx)
+
+    def close(self) -> None:
+        if getattr(self, "ctx", None):
+            kie_destroy(self.ctx)
+            self.ctx = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass

@@ -1,0 +1,554 @@
+// Host side of the C ABI declared in include/kie.h: validation, planning,
+// scratch ownership, launches of the persistent decode kernel and session
+// state (position, fed ids).
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <string>
+#include <vector>
+
+#include "kie.h"
+#include "kie_kernel.h"
+#include "kie_params.h"
+#include "kie_plan.h"
+
+using kie::DevStatus;
+using kie::LayerW;
+using kie::MonoParams;
+
+struct kie_ctx {
+  kie_model_desc desc{};
+  kie::Shape shape{};
+  int device = 0;
+  cudaStream_t stream = nullptr;
+
+  // caller-owned device memory
+  std::vector<LayerW> hlayers;
+  const __half *tok_emb = nullptr, *final_norm = nullptr, *lm_head = nullptr;
+  __half* kv = nullptr;
+
+  // library-owned device memory
+  LayerW* dlayers = nullptr;
+  float2* rope = nullptr;
+  int2* ranges = nullptr;
+  unsigned long long* tagged = nullptr;
+  size_t tagged_words = 0;
+  unsigned long long *x_attn = nullptr, *x_ffn = nullptr, *hbuf = nullptr, *qbuf = nullptr,
+                     *kvnew = nullptr, *obuf = nullptr, *slots = nullptr;
+  float* partials = nullptr;
+  unsigned int* att_ctr = nullptr;
+  int* d_ids = nullptr;               // fed ids of a launch [max_seq]
+  unsigned char* d_io = nullptr;      // DevStatus + out ids [max_seq]
+  unsigned long long* cta_stats = nullptr;
+  unsigned char* h_io = nullptr;      // pinned mirror of d_io
+  cudaEvent_t ev0 = nullptr, ev1 = nullptr;
+
+  // plan
+  std::vector<std::vector<int2>> hranges;
+  int grid = 0, slots_n = 0, slot_bytes = 20480, smem = 0, max_split = 1, min_split_len = 64;
+  kie::SmemLayout sm{};
+
+  // session
+  int pos = 0;
+  bool primed = false;             // a prefill ran; next_tok is valid
+  std::vector<int32_t> fed;        // fed[t] = id fed at position t
+  int32_t next_tok = 0;            // id to feed at position pos
+  unsigned int epoch = 0;
+  bool failed = false;
+
+  // options and capture
+  long long timeout_ns = 2000000000LL;
+  int fault_cta = -1, fault_step = -1, fault_layer = -1, fault_stage = -1;
+  float* capture = nullptr;
+  int capture_rows = 0;
+
+  kie_stats stats{};
+  std::string err;
+};
+
+namespace {
+
+constexpr size_t kStatusBytes = sizeof(DevStatus);
+
+kie_status set_err(kie_ctx* c, kie_status s, const std::string& msg) {
+  if (c) c->err = msg;
+  return s;
+}
+
+kie_status cuda_fail(kie_ctx* c, cudaError_t e, const char* what) {
+  std::string m = std::string(what) + ": " + cudaGetErrorString(e);
+  if (c) c->failed = true;
+  return set_err(c, KIE_ERR_CUDA, m);
+}
+
+#define KIE_CUDA(c, call)                                   \
+  do {                                                      \
+    cudaError_t e_ = (call);                                \
+    if (e_ != cudaSuccess) return cuda_fail((c), e_, #call); \
+  } while (0)
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+kie::Shape shape_of(const kie_model_desc& d) {
+  return kie::Shape{d.n_layers, d.d_model, d.n_heads, d.n_kv_heads, d.head_dim, d.ffn_dim,
+                    d.vocab};
+}
+
+void free_all(kie_ctx* c) {
+  cudaFree(c->dlayers);
+  cudaFree(c->rope);
+  cudaFree(c->ranges);
+  cudaFree(c->tagged);
+  cudaFree(c->partials);
+  cudaFree(c->att_ctr);
+  cudaFree(c->d_ids);
+  cudaFree(c->d_io);
+  cudaFree(c->cta_stats);
+  if (c->h_io) cudaFreeHost(c->h_io);
+  if (c->ev0) cudaEventDestroy(c->ev0);
+  if (c->ev1) cudaEventDestroy(c->ev1);
+}
+
+// One launch of the persistent kernel over n_steps forward passes starting
+// at position pos0.  Step i feeds ids[i] when `forced`, else first_tok for
+// i = 0 and the previous pick afterwards; steps i >= lm_from pick an id.
+kie_status launch(kie_ctx* c, int n_steps, int pos0, const int32_t* host_ids, bool forced,
+                  int first_tok, int lm_from, int* n_done_out) {
+  const kie_model_desc& d = c->desc;
+  const unsigned need = (unsigned)n_steps * (unsigned)(d.n_layers + 1) + 2u;
+  if ((unsigned long long)c->epoch + need >= 0xFFFFFF00ull) {
+    KIE_CUDA(c, cudaMemsetAsync(c->tagged, 0, c->tagged_words * 8, c->stream));
+    c->epoch = 0;
+  }
+  if (forced) {
+    KIE_CUDA(c, cudaMemcpyAsync(c->d_ids, host_ids, sizeof(int32_t) * n_steps,
+                                cudaMemcpyHostToDevice, c->stream));
+  }
+  KIE_CUDA(c, cudaMemsetAsync(c->d_io, 0, kStatusBytes, c->stream));
+
+  MonoParams p{};
+  p.L = d.n_layers;
+  p.d = d.d_model;
+  p.H = d.n_heads;
+  p.KV = d.n_kv_heads;
+  p.hd = d.head_dim;
+  p.F = d.ffn_dim;
+  p.V = d.vocab;
+  p.G = d.n_heads / d.n_kv_heads;
+  p.eps = d.rms_eps;
+  p.max_seq = d.max_seq;
+  p.eos = d.eos_id;
+  p.layers = c->dlayers;
+  p.tok_emb = c->tok_emb;
+  p.final_norm = c->final_norm;
+  p.lm_head = c->lm_head;
+  p.kv = c->kv;
+  p.rope = c->rope;
+  p.ranges = c->ranges;
+  p.grid = c->grid;
+  p.ring_slots = c->slots_n;
+  p.slot_bytes = c->slot_bytes;
+  p.max_split = c->max_split;
+  p.min_split_len = c->min_split_len;
+  p.sm = c->sm;
+  p.x_attn = c->x_attn;
+  p.x_ffn = c->x_ffn;
+  p.hbuf = c->hbuf;
+  p.qbuf = c->qbuf;
+  p.kvnew = c->kvnew;
+  p.obuf = c->obuf;
+  p.slots = c->slots;
+  p.partials = c->partials;
+  p.att_ctr = c->att_ctr;
+  p.n_steps = n_steps;
+  p.pos0 = pos0;
+  p.first_tok = first_tok;
+  p.forced = forced ? c->d_ids : nullptr;
+  p.lm_from = lm_from;
+  p.e0 = c->epoch;
+  p.capture = c->capture;
+  p.capture_rows = c->capture_rows;
+  p.out_ids = reinterpret_cast<int*>(c->d_io + kStatusBytes);
+  p.status = reinterpret_cast<DevStatus*>(c->d_io);
+  p.cta_stats = c->cta_stats;
+  p.timeout_ns = c->timeout_ns;
+  p.fault_cta = c->fault_cta;
+  p.fault_step = c->fault_step;
+  p.fault_layer = c->fault_layer;
+  p.fault_stage = c->fault_stage;
+
+  KIE_CUDA(c, cudaEventRecord(c->ev0, c->stream));
+  KIE_CUDA(c, kie::mono_launch(p, d.head_dim, c->grid, c->smem, c->stream));
+  KIE_CUDA(c, cudaEventRecord(c->ev1, c->stream));
+  KIE_CUDA(c, cudaMemcpyAsync(c->h_io, c->d_io, kStatusBytes + sizeof(int32_t) * n_steps,
+                              cudaMemcpyDeviceToHost, c->stream));
+  KIE_CUDA(c, cudaStreamSynchronize(c->stream));
+  c->epoch += need;
+  c->stats.launches += 1;
+  float ms = 0.f;
+  cudaEventElapsedTime(&ms, c->ev0, c->ev1);
+  c->stats.last_device_ms = ms;
+
+  const DevStatus* st = reinterpret_cast<const DevStatus*>(c->h_io);
+  c->stats.last_steps = st->n_done;
+  *n_done_out = st->n_done;
+  if (st->code != kie::DEV_OK) {
+    c->failed = true;
+    char buf[256];
+    std::snprintf(buf, sizeof buf,
+                  "device %s in CTA %d (step %d, layer %d, stage %d, site %d)",
+                  st->code == kie::DEV_TIMEOUT ? "wait timeout" : "protocol violation", st->cta,
+                  st->step, st->layer, st->stage, st->where);
+    return set_err(c, st->code == kie::DEV_TIMEOUT ? KIE_ERR_TIMEOUT : KIE_ERR_PROTOCOL, buf);
+  }
+  return KIE_OK;
+}
+
+kie_status usable(kie_ctx* c) {
+  if (!c) return KIE_ERR_INVALID_ARG;
+  if (c->failed) return set_err(c, KIE_ERR_STATE, "context failed earlier; destroy it");
+  c->err.clear();
+  return KIE_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t kie_kv_cache_bytes(const kie_model_desc* d) {
+  if (!d || kie_check_desc(d) != KIE_OK) return 0;
+  return (size_t)2 * d->n_layers * d->n_kv_heads * (size_t)d->max_seq * d->head_dim * 2;
+}
+
+kie_status kie_check_desc(const kie_model_desc* d) {
+  if (!d) return KIE_ERR_INVALID_ARG;
+  if (d->n_layers < 1 || d->d_model < 1 || d->n_heads < 1 || d->n_kv_heads < 1 ||
+      d->head_dim < 1 || d->ffn_dim < 1 || d->vocab < 1 || d->max_seq < 1)
+    return KIE_ERR_INVALID_ARG;
+  if (!(d->rms_eps >= 0.f) || !(d->rope_base > 0.f) || !std::isfinite(d->rope_base))
+    return KIE_ERR_INVALID_ARG;
+  if (d->eos_id < -1 || d->eos_id >= d->vocab) return KIE_ERR_INVALID_ARG;
+  if (d->head_dim != 64 && d->head_dim != 128) return KIE_ERR_UNSUPPORTED;
+  if (d->n_heads % d->n_kv_heads != 0) return KIE_ERR_UNSUPPORTED;
+  if (d->n_heads / d->n_kv_heads > kie::kMaxGroup) return KIE_ERR_UNSUPPORTED;
+  if (d->d_model % 256 || d->ffn_dim % 256 || (d->n_heads * d->head_dim) % 256)
+    return KIE_ERR_UNSUPPORTED;
+  return KIE_OK;
+}
+
+kie_status kie_plan_units(const kie_model_desc* d, int32_t grid, int32_t stage, int32_t cta,
+                          int32_t* begin, int32_t* end) {
+  if (!d || !begin || !end) return KIE_ERR_INVALID_ARG;
+  kie_status s = kie_check_desc(d);
+  if (s != KIE_OK) return s;
+  if (grid < 1 || stage < 0 || stage >= kie::N_STAGES || cta < 0 || cta >= grid)
+    return KIE_ERR_INVALID_ARG;
+  const auto r = kie::partition(shape_of(*d), grid, stage);
+  *begin = r[cta].x;
+  *end = r[cta].y;
+  return KIE_OK;
+}
+
+kie_status kie_create(const kie_model_desc* d, const kie_weights* w, void* kv_cache,
+                      void* cuda_stream, kie_ctx** out) {
+  if (!out) return KIE_ERR_INVALID_ARG;
+  *out = nullptr;
+  if (!d || !w || !kv_cache || !w->layers || !w->tok_emb || !w->final_norm || !w->lm_head)
+    return KIE_ERR_INVALID_ARG;
+  kie_status s = kie_check_desc(d);
+  if (s != KIE_OK) return s;
+  if (!aligned16(kv_cache) || !aligned16(w->tok_emb) || !aligned16(w->final_norm) ||
+      !aligned16(w->lm_head))
+    return KIE_ERR_INVALID_ARG;
+  for (int l = 0; l < d->n_layers; ++l) {
+    const kie_layer_weights& lw = w->layers[l];
+    const void* ps[] = {lw.attn_norm, lw.wq, lw.wk, lw.wv, lw.wo, lw.ffn_norm, lw.w_gate, lw.w_up,
+                        lw.w_down};
+    for (const void* q : ps)
+      if (!q || !aligned16(q)) return KIE_ERR_INVALID_ARG;
+  }
+
+  kie_ctx* c = new kie_ctx();
+  c->desc = *d;
+  c->shape = shape_of(*d);
+  c->stream = static_cast<cudaStream_t>(cuda_stream);
+  c->tok_emb = static_cast<const __half*>(w->tok_emb);
+  c->final_norm = static_cast<const __half*>(w->final_norm);
+  c->lm_head = static_cast<const __half*>(w->lm_head);
+  c->kv = static_cast<__half*>(kv_cache);
+  for (int l = 0; l < d->n_layers; ++l) {
+    const kie_layer_weights& lw = w->layers[l];
+    c->hlayers.push_back(LayerW{static_cast<const __half*>(lw.attn_norm),
+                                static_cast<const __half*>(lw.wq), static_cast<const __half*>(lw.wk),
+                                static_cast<const __half*>(lw.wv), static_cast<const __half*>(lw.wo),
+                                static_cast<const __half*>(lw.ffn_norm),
+                                static_cast<const __half*>(lw.w_gate),
+                                static_cast<const __half*>(lw.w_up),
+                                static_cast<const __half*>(lw.w_down)});
+  }
+  auto fail = [&](kie_status st) {
+    free_all(c);
+    delete c;
+    return st;
+  };
+  auto cuda_bad = [&](cudaError_t e) { return e != cudaSuccess; };
+
+  if (cuda_bad(cudaGetDevice(&c->device))) return fail(KIE_ERR_CUDA);
+  int n_sm = 0, smem_optin = 0;
+  if (cuda_bad(cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, c->device)) ||
+      cuda_bad(cudaDeviceGetAttribute(&smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin,
+                                      c->device)))
+    return fail(KIE_ERR_CUDA);
+
+  // grid: one CTA per SM, but never more CTAs than units of the smallest stage
+  int grid = n_sm;
+  for (int st = 0; st < kie::N_STAGES; ++st)
+    grid = std::min(grid, kie::stage_units(c->shape, st));
+  c->grid = grid;
+  c->hranges.resize(kie::N_STAGES);
+  for (int st = 0; st < kie::N_STAGES; ++st) c->hranges[st] = kie::partition(c->shape, grid, st);
+  if (!kie::plan_smem(c->shape, grid, c->slot_bytes, smem_optin, c->hranges, &c->sm, &c->slots_n))
+    return fail(KIE_ERR_UNSUPPORTED);
+  c->smem = c->sm.total;
+  int per_sm = 0;
+  if (cuda_bad(kie::mono_configure(d->head_dim, c->smem, &per_sm))) return fail(KIE_ERR_CUDA);
+  if (per_sm < 1) return fail(KIE_ERR_UNSUPPORTED);
+  c->max_split = std::max(1, grid / d->n_kv_heads);
+
+  const int G = d->n_heads / d->n_kv_heads;
+  const size_t qd = (size_t)d->n_heads * d->head_dim, kvd = (size_t)d->n_kv_heads * d->head_dim;
+  c->tagged_words = 2 * (size_t)d->d_model + d->ffn_dim + qd + 2 * kvd + qd + 2 * (size_t)grid;
+  std::vector<int2> flat;
+  for (auto& v : c->hranges) flat.insert(flat.end(), v.begin(), v.end());
+  const size_t half = d->head_dim / 2;
+  std::vector<float2> rope((size_t)d->max_seq * half);
+  for (int t = 0; t < d->max_seq; ++t)
+    for (size_t i = 0; i < half; ++i) {
+      const double th = std::pow((double)d->rope_base, -2.0 * (double)i / d->head_dim);
+      const double a = (double)t * th;
+      rope[(size_t)t * half + i] = make_float2((float)std::cos(a), (float)std::sin(a));
+    }
+
+  if (cuda_bad(cudaMalloc(&c->dlayers, sizeof(LayerW) * d->n_layers)) ||
+      cuda_bad(cudaMalloc(&c->rope, sizeof(float2) * rope.size())) ||
+      cuda_bad(cudaMalloc(&c->ranges, sizeof(int2) * flat.size())) ||
+      cuda_bad(cudaMalloc(&c->tagged, 8 * c->tagged_words)) ||
+      cuda_bad(cudaMalloc(&c->partials, sizeof(float) * (size_t)grid * G * (d->head_dim + 2))) ||
+      cuda_bad(cudaMalloc(&c->att_ctr, sizeof(unsigned) * d->n_layers * d->n_kv_heads)) ||
+      cuda_bad(cudaMalloc(&c->d_ids, sizeof(int32_t) * d->max_seq)) ||
+      cuda_bad(cudaMalloc(&c->d_io, kStatusBytes + sizeof(int32_t) * d->max_seq)) ||
+      cuda_bad(cudaMalloc(&c->cta_stats, sizeof(unsigned long long) * 4 * grid)) ||
+      cuda_bad(cudaMallocHost(&c->h_io, kStatusBytes + sizeof(int32_t) * d->max_seq)) ||
+      cuda_bad(cudaEventCreate(&c->ev0)) || cuda_bad(cudaEventCreate(&c->ev1)))
+    return fail(KIE_ERR_CUDA);
+  unsigned long long* t = c->tagged;
+  c->x_attn = t;  t += d->d_model;
+  c->x_ffn = t;   t += d->d_model;
+  c->hbuf = t;    t += d->ffn_dim;
+  c->qbuf = t;    t += qd;
+  c->kvnew = t;   t += 2 * kvd;
+  c->obuf = t;    t += qd;
+  c->slots = t;
+  if (cuda_bad(cudaMemcpyAsync(c->dlayers, c->hlayers.data(), sizeof(LayerW) * d->n_layers,
+                               cudaMemcpyHostToDevice, c->stream)) ||
+      cuda_bad(cudaMemcpyAsync(c->rope, rope.data(), sizeof(float2) * rope.size(),
+                               cudaMemcpyHostToDevice, c->stream)) ||
+      cuda_bad(cudaMemcpyAsync(c->ranges, flat.data(), sizeof(int2) * flat.size(),
+                               cudaMemcpyHostToDevice, c->stream)) ||
+      cuda_bad(cudaMemsetAsync(c->tagged, 0, 8 * c->tagged_words, c->stream)) ||
+      cuda_bad(cudaMemsetAsync(c->att_ctr, 0, sizeof(unsigned) * d->n_layers * d->n_kv_heads,
+                               c->stream)) ||
+      cuda_bad(cudaMemsetAsync(c->cta_stats, 0, sizeof(unsigned long long) * 4 * grid,
+                               c->stream)) ||
+      cuda_bad(cudaStreamSynchronize(c->stream)))
+    return fail(KIE_ERR_CUDA);
+
+  c->stats.grid = grid;
+  c->stats.ring_slots = c->slots_n;
+  c->stats.slot_bytes = c->slot_bytes;
+  c->stats.smem_bytes = c->smem;
+  *out = c;
+  return KIE_OK;
+}
+
+kie_status kie_prefill(kie_ctx* c, const int32_t* ids, int32_t n, int32_t* first_id) {
+  kie_status s = usable(c);
+  if (s != KIE_OK) return s;
+  if (!ids || n < 1) return set_err(c, KIE_ERR_INVALID_ARG, "prefill needs n >= 1 ids");
+  if (n > c->desc.max_seq) return set_err(c, KIE_ERR_CAPACITY, "prompt longer than max_seq");
+  for (int i = 0; i < n; ++i)
+    if (ids[i] < 0 || ids[i] >= c->desc.vocab)
+      return set_err(c, KIE_ERR_INVALID_ARG, "prompt id out of range");
+  c->primed = false;
+  int done = 0;
+  s = launch(c, n, 0, ids, true, 0, n - 1, &done);
+  if (s != KIE_OK) return s;
+  const int32_t g0 = reinterpret_cast<const int32_t*>(c->h_io + kStatusBytes)[n - 1];
+  c->fed.assign(ids, ids + n);
+  c->pos = n;
+  c->next_tok = g0;
+  c->primed = true;
+  if (first_id) *first_id = g0;
+  c->stats.pos = c->pos;
+  return KIE_OK;
+}
+
+static kie_status decode_impl(kie_ctx* c, int32_t n, const int32_t* forced_ids,
+                              int32_t* out_ids, int32_t* n_out) {
+  kie_status s = usable(c);
+  if (s != KIE_OK) return s;
+  if (n_out) *n_out = 0;
+  if (n < 0) return set_err(c, KIE_ERR_INVALID_ARG, "n_steps < 0");
+  if (!c->primed) return set_err(c, KIE_ERR_STATE, "decode before prefill");
+  if (n == 0) return KIE_OK;
+  if (!out_ids && !forced_ids) return set_err(c, KIE_ERR_INVALID_ARG, "out_ids is NULL");
+  if ((long long)c->pos + n > c->desc.max_seq)
+    return set_err(c, KIE_ERR_CAPACITY, "decode would pass max_seq positions");
+  if (forced_ids)
+    for (int i = 0; i < n; ++i)
+      if (forced_ids[i] < 0 || forced_ids[i] >= c->desc.vocab)
+        return set_err(c, KIE_ERR_INVALID_ARG, "forced id out of range");
+  int done = 0;
+  s = launch(c, n, c->pos, forced_ids, forced_ids != nullptr, c->next_tok, 0, &done);
+  if (s != KIE_OK) return s;
+  const int32_t* picks = reinterpret_cast<const int32_t*>(c->h_io + kStatusBytes);
+  if (out_ids) std::memcpy(out_ids, picks, sizeof(int32_t) * done);
+  for (int i = 0; i < done; ++i) {
+    c->fed.push_back(forced_ids ? forced_ids[i] : (i == 0 ? c->next_tok : picks[i - 1]));
+  }
+  c->pos += done;
+  if (done > 0) c->next_tok = picks[done - 1];
+  if (n_out) *n_out = done;
+  c->stats.pos = c->pos;
+  return KIE_OK;
+}
+
+kie_status kie_decode(kie_ctx* c, int32_t n, int32_t* out_ids, int32_t* n_out) {
+  return decode_impl(c, n, nullptr, out_ids, n_out);
+}
+
+kie_status kie_decode_forced(kie_ctx* c, const int32_t* ids, int32_t n, int32_t* out_ids) {
+  if (c && n > 0 && !ids) return set_err(c, KIE_ERR_INVALID_ARG, "ids is NULL");
+  std::vector<int32_t> tmp;
+  if (!out_ids && n > 0) {
+    tmp.resize(n);
+    out_ids = tmp.data();
+  }
+  return decode_impl(c, n, ids, out_ids, nullptr);
+}
+
+kie_status kie_rewind(kie_ctx* c, int32_t pos) {
+  kie_status s = usable(c);
+  if (s != KIE_OK) return s;
+  if (!c->primed) return set_err(c, KIE_ERR_STATE, "rewind before prefill");
+  if (pos < 1 || pos > c->pos) return set_err(c, KIE_ERR_INVALID_ARG, "rewind out of range");
+  if (pos < c->pos) {
+    c->next_tok = c->fed[pos];
+    c->fed.resize(pos);
+    c->pos = pos;
+  }
+  c->stats.pos = c->pos;
+  return KIE_OK;
+}
+
+kie_status kie_set_logits_capture(kie_ctx* c, float* dev_logits, int32_t rows) {
+  if (!c) return KIE_ERR_INVALID_ARG;
+  if (dev_logits && rows < 1) return set_err(c, KIE_ERR_INVALID_ARG, "capacity_rows < 1");
+  c->capture = dev_logits;
+  c->capture_rows = dev_logits ? rows : 0;
+  return KIE_OK;
+}
+
+kie_status kie_set_option(kie_ctx* c, kie_option opt, int64_t v) {
+  if (!c) return KIE_ERR_INVALID_ARG;
+  switch (opt) {
+    case KIE_OPT_TIMEOUT_NS:
+      if (v < 1000) return KIE_ERR_INVALID_ARG;
+      c->timeout_ns = v;
+      return KIE_OK;
+    case KIE_OPT_SLOT_BYTES: {
+      if (v < 4096 || v % 4096 || v > (1 << 20)) return KIE_ERR_INVALID_ARG;
+      int smem_optin = 0;
+      if (cudaDeviceGetAttribute(&smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin,
+                                 c->device) != cudaSuccess)
+        return set_err(c, KIE_ERR_CUDA, "device attribute query failed");
+      kie::SmemLayout sm{};
+      int slots = 0;
+      if (!kie::plan_smem(c->shape, c->grid, (int)v, smem_optin, c->hranges, &sm, &slots))
+        return set_err(c, KIE_ERR_UNSUPPORTED, "slot size does not fit shared memory");
+      int per_sm = 0;
+      if (kie::mono_configure(c->desc.head_dim, sm.total, &per_sm) != cudaSuccess || per_sm < 1)
+        return set_err(c, KIE_ERR_UNSUPPORTED, "kernel does not fit with this slot size");
+      c->slot_bytes = (int)v;
+      c->sm = sm;
+      c->slots_n = slots;
+      c->smem = sm.total;
+      c->stats.ring_slots = slots;
+      c->stats.slot_bytes = (int)v;
+      c->stats.smem_bytes = sm.total;
+      return KIE_OK;
+    }
+    case KIE_OPT_MIN_SPLIT_LEN:
+      if (v < 1 || v > (1 << 20)) return KIE_ERR_INVALID_ARG;
+      c->min_split_len = (int)v;
+      return KIE_OK;
+    case KIE_OPT_FAULT_CTA: c->fault_cta = (int)v; return KIE_OK;
+    case KIE_OPT_FAULT_STEP: c->fault_step = (int)v; return KIE_OK;
+    case KIE_OPT_FAULT_LAYER: c->fault_layer = (int)v; return KIE_OK;
+    case KIE_OPT_FAULT_STAGE: c->fault_stage = (int)v; return KIE_OK;
+  }
+  return KIE_ERR_INVALID_ARG;
+}
+
+kie_status kie_get_stats(const kie_ctx* cc, kie_stats* out) {
+  if (!cc || !out) return KIE_ERR_INVALID_ARG;
+  kie_ctx* c = const_cast<kie_ctx*>(cc);
+  *out = c->stats;
+  if (c->stats.launches > 0 && c->cta_stats) {
+    std::vector<unsigned long long> st((size_t)4 * c->grid);
+    if (cudaMemcpy(st.data(), c->cta_stats, sizeof(unsigned long long) * st.size(),
+                   cudaMemcpyDeviceToHost) == cudaSuccess) {
+      double loop = 0, sync = 0, stream = 0, mx = 0;
+      for (int i = 0; i < c->grid; ++i) {
+        loop += (double)st[4 * i];
+        sync += (double)st[4 * i + 1];
+        stream += (double)st[4 * i + 2];
+        if (st[4 * i] > 0) mx = std::max(mx, (double)st[4 * i + 1] / (double)st[4 * i]);
+      }
+      out->loop_cycles = loop / c->grid;
+      out->sync_wait_cycles = sync / c->grid;
+      out->stream_wait_cycles = stream / c->grid;
+      out->sync_wait_max_frac = mx;
+    }
+  }
+  return KIE_OK;
+}
+
+const char* kie_status_str(kie_status s) {
+  switch (s) {
+    case KIE_OK: return "ok";
+    case KIE_ERR_INVALID_ARG: return "invalid argument";
+    case KIE_ERR_UNSUPPORTED: return "unsupported shape";
+    case KIE_ERR_CUDA: return "CUDA error";
+    case KIE_ERR_CAPACITY: return "KV cache capacity exceeded";
+    case KIE_ERR_STATE: return "invalid state";
+    case KIE_ERR_TIMEOUT: return "device wait timed out";
+    case KIE_ERR_PROTOCOL: return "device protocol violation";
+  }
+  return "unknown status";
+}
+
+const char* kie_last_error(const kie_ctx* c) { return c ? c->err.c_str() : ""; }
+
+kie_status kie_destroy(kie_ctx* c) {
+  if (!c) return KIE_ERR_INVALID_ARG;
+  if (c->stream) cudaStreamSynchronize(c->stream);
+  free_all(c);
+  delete c;
+  return KIE_OK;
+}
+
+}  // extern "C"

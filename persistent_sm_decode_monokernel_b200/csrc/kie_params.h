@@ -1,0 +1,78 @@
+// Parameters shared by the host side (kie_host.cu) and the persistent
+// decode kernel (kie_kernel.cu).  Plain data only.
+#pragma once
+
+#include <cstdint>
+#include <cuda_fp16.h>
+
+namespace kie {
+
+// GEMV stages of one decoder layer plus the LM head.  The attention stage
+// has no weight stream and is not listed here.
+enum Stage : int { ST_QKV = 0, ST_O = 1, ST_GU = 2, ST_DOWN = 3, ST_LM = 4, N_STAGES = 5 };
+
+constexpr int kConsumerWarps = 8;            // warps that compute
+constexpr int kThreads = (kConsumerWarps + 1) * 32;  // + one producer warp
+constexpr int kConsumerThreads = kConsumerWarps * 32;
+constexpr int kPieceElems = 256;             // one warp pass: 32 lanes x 8 fp16
+constexpr int kPieceBytes = kPieceElems * 2;
+constexpr int kMaxSlots = 16;
+constexpr int kMaxGroup = 8;                 // heads per KV head handled by one CTA
+constexpr int kAttnBlock = 256;              // positions per attention block
+
+// Device status word block (library scratch, zeroed before each launch).
+struct DevStatus {
+  unsigned int code;   // 0 ok, 1 timeout, 2 protocol
+  int cta, step, layer, stage, where;
+  int n_done;          // forward passes finished (written by CTA 0)
+  int pad;
+};
+enum : unsigned int { DEV_OK = 0, DEV_TIMEOUT = 1, DEV_PROTOCOL = 2 };
+
+struct LayerW {
+  const __half *attn_norm, *wq, *wk, *wv, *wo, *ffn_norm, *wg, *wu, *wd;
+};
+
+// Shared-memory carve-up of one CTA (byte offsets from the dynamic base).
+struct SmemLayout {
+  int ring_off, bar_off, xs_off, rowacc_off, misc_off, total;
+  int xs_bytes, rowacc_rows;
+};
+
+struct MonoParams {
+  // model
+  int L, d, H, KV, hd, F, V, G;
+  float eps;
+  int max_seq, eos;
+  // weights (device)
+  const LayerW* layers;
+  const __half* tok_emb;
+  const __half* final_norm;
+  const __half* lm_head;
+  __half* kv;              // [L][2][KV][max_seq][hd]
+  const float2* rope;      // [max_seq][hd/2] (cos, sin)
+  // plan
+  const int2* ranges;      // [N_STAGES][grid] unit range per CTA
+  int grid;
+  int ring_slots, slot_bytes;
+  int max_split, min_split_len;
+  SmemLayout sm;
+  // scratch (tagged 64-bit words: high 32 bits = epoch tag, low = fp32 bits)
+  unsigned long long *x_attn, *x_ffn, *hbuf, *qbuf, *kvnew, *obuf, *slots;
+  float* partials;         // [grid][G][hd + 2]
+  unsigned int* att_ctr;   // [L][KV] last-arriver counters
+  // run
+  int n_steps, pos0, first_tok;
+  const int* forced;       // [n_steps] or null
+  int lm_from;
+  unsigned int e0;
+  float* capture;
+  int capture_rows;
+  int* out_ids;
+  DevStatus* status;
+  unsigned long long* cta_stats;  // [grid][4]: loop, sync wait, stream wait, spare
+  long long timeout_ns;
+  int fault_cta, fault_step, fault_layer, fault_stage;
+};
+
+}  // namespace kie

@@ -1,0 +1,124 @@
+#include "kie_plan.h"
+
+#include <algorithm>
+
+namespace kie {
+
+int stage_units(const Shape& s, int stage) {
+  switch (stage) {
+    case ST_QKV: return s.H * s.hd / 2 + s.KV * s.hd / 2 + s.KV * s.hd;
+    case ST_O: return s.d;
+    case ST_GU: return s.F;
+    case ST_DOWN: return s.d;
+    case ST_LM: return s.V;
+  }
+  return 0;
+}
+
+int stage_rows(const Shape& s, int stage) {
+  switch (stage) {
+    case ST_QKV: return (s.H + 2 * s.KV) * s.hd;
+    case ST_GU: return 2 * s.F;
+    default: return stage_units(s, stage);
+  }
+}
+
+int stage_k(const Shape& s, int stage) {
+  switch (stage) {
+    case ST_QKV: return s.d;
+    case ST_O: return s.H * s.hd;
+    case ST_GU: return s.d;
+    case ST_DOWN: return s.F;
+    case ST_LM: return s.d;
+  }
+  return 0;
+}
+
+// rows held by units [0, u)
+static long long cum_rows(const Shape& s, int stage, long long u) {
+  if (stage == ST_QKV) {
+    const long long np = (long long)(s.H + s.KV) * s.hd / 2;
+    return u <= np ? 2 * u : 2 * np + (u - np);
+  }
+  if (stage == ST_GU) return 2 * u;
+  return u;
+}
+
+// unit boundary whose cumulative row count is nearest to `rows`
+// (ties to the lower boundary)
+static int unit_at_rows(const Shape& s, int stage, long long rows) {
+  if (stage == ST_QKV) {
+    const long long np = (long long)(s.H + s.KV) * s.hd / 2;
+    if (rows <= 2 * np) return (int)(rows / 2);
+    return (int)(np + (rows - 2 * np));
+  }
+  if (stage == ST_GU) return (int)(rows / 2);
+  return (int)rows;
+}
+
+int rows_in_range(const Shape& s, int stage, int ub, int ue) {
+  return (int)(cum_rows(s, stage, ue) - cum_rows(s, stage, ub));
+}
+
+std::vector<int2> partition(const Shape& s, int grid, int stage) {
+  const long long R = stage_rows(s, stage);
+  std::vector<int> bound(grid + 1);
+  for (int v = 0; v <= grid; ++v) {
+    long long target = (R * v + grid / 2) / grid;
+    bound[v] = unit_at_rows(s, stage, target);
+  }
+  bound[grid] = stage_units(s, stage);
+  const int rot = (stage * 41) % grid;
+  std::vector<int2> r(grid);
+  for (int c = 0; c < grid; ++c) {
+    const int v = (c + rot) % grid;
+    r[c] = make_int2(bound[v], bound[v + 1]);
+  }
+  return r;
+}
+
+int attn_smem_bytes(int G, int hd) {
+  const int ngrp = kConsumerThreads / (hd / 2);
+  int b = 0;
+  b += G * hd * 4;              // q (scaled)
+  b += G * kAttnBlock * 4;      // scores / probabilities of one block
+  b += 2 * hd * 4;              // current position's k and v
+  b += ngrp * G * hd * 4;       // V-phase partial sums per position group
+  b += G * hd * 4;              // running output
+  b += 4 * kMaxGroup * 4;       // running max, sum, rescale, spare
+  return b;
+}
+
+static int align_up(int x, int a) { return (x + a - 1) / a * a; }
+
+bool plan_smem(const Shape& s, int grid, int slot_bytes, int smem_limit,
+               const std::vector<std::vector<int2>>& ranges, SmemLayout* out,
+               int* ring_slots) {
+  const int G = s.H / s.KV;
+  const int kmax = std::max(std::max(s.d, s.H * s.hd), s.F);
+  SmemLayout L{};
+  L.xs_bytes = align_up(std::max(kmax * 4, attn_smem_bytes(G, s.hd)), 128);
+  int maxrows = 0;
+  for (int st = 0; st < N_STAGES; ++st)
+    for (int c = 0; c < grid; ++c)
+      maxrows = std::max(maxrows, rows_in_range(s, st, ranges[st][c].x, ranges[st][c].y));
+  L.rowacc_rows = maxrows;
+  const int bars = 2 * kMaxSlots * 8;
+  const int misc = 1024;
+  const int fixed = align_up(bars, 128) + L.xs_bytes + align_up(maxrows * 4, 128) + misc;
+  const int avail = smem_limit - fixed;
+  int slots = avail / slot_bytes;
+  if (slots > kMaxSlots) slots = kMaxSlots;
+  if (slots < 2) return false;
+  L.ring_off = 0;
+  L.bar_off = slots * slot_bytes;
+  L.xs_off = L.bar_off + align_up(bars, 128);
+  L.rowacc_off = L.xs_off + L.xs_bytes;
+  L.misc_off = L.rowacc_off + align_up(maxrows * 4, 128);
+  L.total = L.misc_off + misc;
+  *out = L;
+  *ring_slots = slots;
+  return L.total <= smem_limit;
+}
+
+}  // namespace kie

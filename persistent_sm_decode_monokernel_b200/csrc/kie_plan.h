@@ -1,0 +1,40 @@
+// Host-side planning of the persistent decode kernel: which rows of each
+// weight matrix every CTA streams, and how its shared memory is carved.
+#pragma once
+
+#include <cstdint>
+#include <vector>
+
+#include "kie_params.h"
+
+namespace kie {
+
+struct Shape {
+  int L, d, H, KV, hd, F, V;
+};
+
+// Units of a GEMV stage.  A unit is the smallest piece of work a CTA owns:
+//   QKV:  H*hd/2 q RoPE pairs, then KV*hd/2 k RoPE pairs (2 rows each),
+//         then KV*hd v rows (1 row each);
+//   O:    d rows of Wo;      GU: F (gate row, up row) pairs;
+//   DOWN: d rows of Wd;      LM: V rows of the LM head.
+int stage_units(const Shape& s, int stage);
+int stage_rows(const Shape& s, int stage);
+int stage_k(const Shape& s, int stage);
+// Rows held by units [ub, ue) of a stage.
+int rows_in_range(const Shape& s, int stage, int ub, int ue);
+
+// Contiguous unit ranges for `grid` CTAs, balanced by rows (at most one
+// unit apart); the assignment is rotated by a stage-dependent offset so
+// that the CTAs holding an extra unit differ from stage to stage.
+std::vector<int2> partition(const Shape& s, int grid, int stage);
+
+// Attention shared-memory bytes for group size G and head_dim hd.
+int attn_smem_bytes(int G, int hd);
+
+// Shared memory carve-up; returns false if it does not fit `smem_limit`.
+bool plan_smem(const Shape& s, int grid, int slot_bytes, int smem_limit,
+               const std::vector<std::vector<int2>>& ranges, SmemLayout* out,
+               int* ring_slots);
+
+}  // namespace kie
