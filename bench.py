@@ -1,0 +1,373 @@
+#!/usr/bin/env python
+"""Batch-1 decode benchmark of the persistent decode kernel on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+                    [--impl reference] [--no-cpu-baseline]
+
+A step is one request's decode: the session is rewound to the end of the
+prompt (P positions of KV already in HBM) and kie_decode runs S greedy steps
+in ONE launch of the persistent kernel.  W untimed steps, then K timed
+steps bracketed by a barrier and a device synchronize, timed with CUDA
+events on the launching stream.  `value` is decode tokens/s per request:
+N * K * S / (max over ranks of the timed region).  With N > 1 every rank
+runs an independent replica (the path does not shard; there is no
+collective on the data path).
+
+`--impl reference` times the CPU oracle instead (rank 0 only), on a bounded
+sample of the same workload, and prints the same JSON line with
+"impl": "reference".
+
+Prints one JSON line on rank 0.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+DEFAULT_WORKLOAD = "l28-d2560"
+NOMINAL_HBM_GBS = 8000.0
+FALLBACK_HBM_GBS = 6650.0
+METRIC = "batch-1 decode tokens/s per request"
+
+
+def _peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def decode_bytes(w: synth.Workload, pos0: int, n_steps: int) -> float:
+    """Algorithmic HBM bytes of n_steps decode steps starting at position
+    pos0: every weight matrix, the norm gains and one embedding row per
+    step, plus K/V reads of positions 0..pos and the K/V write at pos."""
+    s = w.shape
+    per_pos = s.kv_bytes_per_position()
+    total = 0.0
+    for i in range(n_steps):
+        pos = pos0 + i
+        total += s.matrix_bytes_per_token() + per_pos * (pos + 1) + per_pos
+    return total
+
+
+# ------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    """nvidia-smi clock/throttle samples while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.idx = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(prefix="clocks_", suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        for line in open(self.path):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append(parts)
+            except ValueError:
+                pass
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return None
+        sm = [num(r[1]) for r in rows if num(r[1]) is not None]
+        mx = [num(r[2]) for r in rows if num(r[2]) is not None]
+        power = [num(r[3]) for r in rows if num(r[3]) is not None]
+        # samples under load: the upper half by power draw
+        loaded = sm
+        if power and len(power) == len(sm):
+            thr = statistics.median(power)
+            loaded = [s for s, p in zip(sm, power) if p >= thr] or sm
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[k] for r in rows for k in range(4)
+                          if r[5 + k].lower() == "active"})
+        return {"sm_mhz": statistics.median(loaded) if loaded else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(rows), "power_w_max": max(power) if power else None}
+
+
+# ------------------------------------------------------------ distribution
+
+def init_dist():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if world <= 1:
+        return None, 0, 1
+    import torch.distributed as dist
+    from datetime import timedelta
+    backend = os.environ.get("KIE_BENCH_BACKEND", "nccl")
+    dist.init_process_group(backend=backend, timeout=timedelta(seconds=300))
+    return dist, dist.get_rank(), dist.get_world_size()
+
+
+def reduce_max_sum(dist, elapsed_s: float, tokens: float, device=None):
+    """(max over ranks of elapsed, sum over ranks of tokens)."""
+    if dist is None:
+        return elapsed_s, tokens
+    import torch
+    t = torch.tensor([elapsed_s], dtype=torch.float64, device=device)
+    n = torch.tensor([tokens], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    dist.all_reduce(n, op=dist.ReduceOp.SUM)
+    return float(t.item()), float(n.item())
+
+
+# ------------------------------------------------------------- CPU oracle
+
+def cpu_oracle_rate(w: synth.Workload, model, budget_s: float = 12.0, max_steps: int = 64,
+                    warmup: int = 1):
+    """Times the oracle's incremental decode (fp32, numpy/BLAS on the host
+    cores) after a batched prefill of the prompt.  Returns (tok/s, info)."""
+    from oracle import OracleModel, argmax_lowest
+    from threadpoolctl import threadpool_info
+    om = OracleModel(model, dtype=np.float32)
+    prompt = synth.make_prompt(w.shape.vocab, w.prompt_len, seed=w.seed)
+    t0 = time.perf_counter()
+    st, lg = om.prefill_batched(prompt)
+    t_prefill = time.perf_counter() - t0
+    tok = argmax_lowest(lg)
+    for _ in range(warmup):
+        tok = argmax_lowest(om.decode_step(st, tok))
+    n = 0
+    t0 = time.perf_counter()
+    while n < max_steps and (time.perf_counter() - t0) < budget_s:
+        tok = argmax_lowest(om.decode_step(st, tok))
+        n += 1
+    el = time.perf_counter() - t0
+    threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    return n / el, {"steps": n, "seconds": el, "prefill_s": t_prefill, "threads": threads,
+                    "first_pos": w.prompt_len + warmup}
+
+
+# ------------------------------------------------------------------ arms
+
+def run_reference(args, w, rank, world):
+    if rank != 0:
+        return 0
+    model = synth.make_model(w.shape, seed=w.seed)
+    from oracle import OracleModel, argmax_lowest
+    from threadpoolctl import threadpool_info
+    om = OracleModel(model, dtype=np.float32)
+    prompt = synth.make_prompt(w.shape.vocab, w.prompt_len, seed=w.seed)
+    st, lg = om.prefill_batched(prompt)
+    tok = argmax_lowest(lg)
+    per_step = args.ref_tokens_per_step
+    for _ in range(args.warmup):
+        for _ in range(per_step):
+            tok = argmax_lowest(om.decode_step(st, tok))
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        for _ in range(per_step):
+            tok = argmax_lowest(om.decode_step(st, tok))
+    el = time.perf_counter() - t0
+    value = args.steps * per_step / el
+    threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    sample = (f"{per_step} oracle decode steps per bench step (fp32 numpy, cached fp32 weights) "
+              f"at positions {w.prompt_len}+ after a batched prefill of the {w.prompt_len}-id "
+              f"prompt; {args.steps} timed bench steps")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tok/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1000.0 * el / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": workload_config(w),
+        "cpu_baseline": {"value": value, "unit": "tok/s", "cores": threads, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "tok/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def workload_config(w: synth.Workload):
+    s = w.shape
+    return {"workload": w.name, "layers": s.n_layers, "d_model": s.d_model,
+            "heads": s.n_heads, "kv_heads": s.n_kv_heads, "head_dim": s.head_dim,
+            "ffn": s.ffn_dim, "vocab": s.vocab, "params": s.n_params(),
+            "prompt_len": w.prompt_len, "decode_steps_per_launch": w.decode_steps,
+            "batch": 1, "weights": "fp16 N(0,0.02), seed 0", "kv_cache": "fp16",
+            "parallelism": "replicas",
+            "l2": "inputs larger than L2 (weights streamed per token exceed the 126 MB L2)"}
+
+
+def run_gpu(args, w, dist, rank, world):
+    import torch
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    from persistent_sm_decode_monokernel_b200 import Session, build, upload_weights
+    if rank == 0 or not os.path.exists(os.path.join(ROOT, "persistent_sm_decode_monokernel_b200",
+                                                      "libkie.so")):
+        build.build()
+    if dist is not None:
+        dist.barrier()
+    model = synth.make_model(w.shape, seed=w.seed)
+    dev = upload_weights(model.tensors)
+    prompt = synth.make_prompt(w.shape.vocab, w.prompt_len, seed=w.seed)
+    stream = torch.cuda.current_stream()
+    sess = Session(w.shape, dev, max_seq=w.max_seq, stream=stream)
+    sess.prefill(prompt)
+    P, S = w.prompt_len, w.decode_steps
+    out = np.empty(S, dtype=np.int32)
+
+    def one_step():
+        sess.rewind(P)
+        ids = sess.decode(S, out)
+        assert len(ids) == S
+        return sess.stats()["last_device_ms"]
+
+    for _ in range(args.warmup):
+        one_step()
+    ref_ids = out.copy()
+
+    clocks = ClockSampler(local)
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    ev0 = torch.cuda.Event(enable_timing=True)
+    ev1 = torch.cuda.Event(enable_timing=True)
+    launch_ms = []
+    ev0.record(stream)
+    for _ in range(args.steps):
+        launch_ms.append(one_step())
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    if dist is not None:
+        dist.barrier()
+    elapsed = ev0.elapsed_time(ev1) / 1000.0
+    deterministic = bool(np.array_equal(out, ref_ids))
+    t_max, tokens = reduce_max_sum(dist, elapsed, float(args.steps * S),
+                                   device=torch.device("cuda", local))
+    value = tokens / t_max
+
+    # end to end through the public call with host buffers, host clock
+    e2e_times = []
+    for _ in range(max(1, min(args.steps, 3))):
+        sess.rewind(P)
+        t0 = time.perf_counter()
+        sess.decode(S, out)
+        e2e_times.append(time.perf_counter() - t0)
+    e2e_local = sum(e2e_times)
+    e2e_max, e2e_tok = reduce_max_sum(dist, e2e_local, float(len(e2e_times) * S),
+                                      device=torch.device("cuda", local))
+
+    st = sess.stats()
+    loop = st["loop_cycles"] or 1.0
+    sync_frac = st["sync_wait_cycles"] / loop
+    stream_frac = st["stream_wait_cycles"] / loop
+    sess.close()
+
+    if rank != 0:
+        return 0
+    peak, peak_kind = _peaks()
+    avg_launch_s = (sum(launch_ms) / len(launch_ms)) / 1000.0
+    bytes_launch = decode_bytes(w, P, S)
+    achieved = bytes_launch / avg_launch_s / 1e9
+    line = {
+        "metric": METRIC, "value": value, "unit": "tok/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1000.0 * t_max / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f16 weights+KV, f32 accumulate",
+        "data": "synthetic", "config": workload_config(w),
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "peak_source": peak_kind,
+                     "frac_vs_nominal_8tbs": achieved / NOMINAL_HBM_GBS,
+                     "traffic": args.traffic,
+                     "algorithmic_bytes_per_launch": bytes_launch,
+                     "avg_launch_ms": avg_launch_s * 1000.0},
+        "e2e": {"value": e2e_tok / e2e_max, "unit": "tok/s",
+                "h2d_bytes_per_step": 4, "d2h_bytes_per_step": 4 * S + 32,
+                "how": "host clock around kie_decode (host id buffer): launch, device run, "
+                       "D2H of ids and status"},
+        "gpu_launches": args.steps,
+        "clocks": clk,
+        "sync_wait_frac": sync_frac, "stream_wait_frac": stream_frac,
+        "per_token_us": 1e6 * avg_launch_s / S,
+        "deterministic_ids": deterministic,
+    }
+    if not args.no_cpu_baseline:
+        rate, info = cpu_oracle_rate(w, model)
+        line["cpu_baseline"] = {
+            "value": rate, "unit": "tok/s", "cores": info["threads"], "kind": "oracle",
+            "sample": f"{info['steps']} fp32 oracle decode steps at positions "
+                      f"{info['first_pos']}+ after a batched prefill of the prompt "
+                      f"({info['seconds']:.1f} s timed)"}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--impl", default="kie", choices=["kie", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--ref-tokens-per-step", type=int, default=4)
+    ap.add_argument("--traffic", type=float, default=None,
+                    help="DRAM bytes per launch from an ncu capture of the same kernel")
+    args = ap.parse_args(argv)
+    w = synth.WORKLOADS[args.workload]
+    if args.impl == "reference":
+        rank = int(os.environ.get("RANK", "0"))
+        world = int(os.environ.get("WORLD_SIZE", str(args.gpus)))
+        return run_reference(args, w, rank, world)
+    dist, rank, world = init_dist()
+    try:
+        return run_gpu(args, w, dist, rank, world)
+    finally:
+        if dist is not None:
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -36,10 +36,16 @@
  *   - The KV cache is one device buffer of kie_kv_cache_bytes() bytes,
  *     16-byte aligned, laid out fp16 [n_layers][2][n_kv_heads][max_seq][hd]
  *     (index 0 = K after RoPE, 1 = V).
- *   - The CALLER owns the weights and the KV cache; both must stay valid and
- *     unmodified (except by this library) until kie_destroy.  The library
- *     owns its scratch (activation words, attention partials, the RoPE
- *     table, id buffers), allocated in kie_create and freed in kie_destroy.
+ *   - The CALLER owns the weights and the KV cache.  kie_create copies the
+ *     weight matrices (wq..w_down, lm_head) into a library-owned buffer laid
+ *     out in the order each CTA streams them, so that every streamed chunk
+ *     is one contiguous bulk copy; after kie_create the library reads only
+ *     tok_emb and the norm gains from the caller (these must stay valid and
+ *     unmodified until kie_destroy), and the caller's matrices are read
+ *     again only by KIE_OPT_CHUNK_BYTES.  The KV cache must stay valid until
+ *     kie_destroy.  The library owns the packed copy and its scratch
+ *     (activation words, attention partials, the RoPE table, id buffers),
+ *     allocated in kie_create and freed in kie_destroy.
  *
  * Errors
  *   Every call returns a kie_status; nothing is thrown across the ABI.
@@ -113,8 +119,8 @@ typedef struct kie_ctx kie_ctx;
 typedef struct {
   int32_t pos;              /* positions held in the KV cache */
   int32_t grid;             /* persistent CTAs (one per SM) */
-  int32_t ring_slots;       /* weight-stream ring depth per CTA */
-  int32_t slot_bytes;       /* bytes per ring slot */
+  int32_t ring_bytes;       /* shared-memory weight ring per CTA */
+  int32_t chunk_bytes;      /* largest weight chunk (one bulk copy) */
   int32_t smem_bytes;       /* dynamic shared memory per CTA */
   int32_t last_steps;       /* forward passes run by the last launch */
   float last_device_ms;     /* device time of the last launch (CUDA events) */
@@ -126,17 +132,22 @@ typedef struct {
   double loop_cycles;
   double sync_wait_cycles;
   double stream_wait_cycles;
-  double sync_wait_max_frac; /* max over CTAs of sync_wait/loop */
+  double producer_wait_cycles; /* producer cycles waiting for a free ring slot */
+  double sync_wait_max_frac;   /* max over CTAs of sync_wait/loop */
 } kie_stats;
 
 typedef enum {
   KIE_OPT_TIMEOUT_NS = 1,     /* bound of every device-side wait (default 2e9) */
-  KIE_OPT_SLOT_BYTES = 2,     /* ring slot size in bytes, multiple of 4096; re-plans the ring */
+  KIE_OPT_CHUNK_BYTES = 2,    /* largest weight chunk in bytes (>= 8192, multiple of 512;
+                                 default 32768); re-plans the ring and rebuilds the packed
+                                 weight copy, so the caller's matrices must still be valid */
   KIE_OPT_MIN_SPLIT_LEN = 3,  /* minimum positions per attention split (default 64) */
   KIE_OPT_FAULT_CTA = 4,      /* test hook: CTA that withholds one publication (-1 off) */
   KIE_OPT_FAULT_STEP = 5,     /* test hook: step of the withheld publication */
   KIE_OPT_FAULT_LAYER = 6,    /* test hook: layer of the withheld publication */
-  KIE_OPT_FAULT_STAGE = 7     /* test hook: 0 QKV, 1 O, 2 gate/up, 3 down, 4 LM */
+  KIE_OPT_FAULT_STAGE = 7,    /* test hook: 0 QKV, 1 O, 2 gate/up, 3 down, 4 LM */
+  KIE_OPT_POLL_BACKOFF_NS = 8, /* sleep between re-polls of another CTA's data (default 128) */
+  KIE_OPT_TRACE_CLOCK = 9      /* stage trace in SM cycles (1) instead of ns (0, default) */
 } kie_option;
 
 /* Bytes of the caller-provided KV cache: 2*n_layers*n_kv_heads*max_seq*head_dim*2.
@@ -189,12 +200,39 @@ KIE_API kie_status kie_rewind(kie_ctx *ctx, int32_t pos);
 KIE_API kie_status kie_set_logits_capture(kie_ctx *ctx, float *dev_logits,
                                   int32_t capacity_rows);
 
+/* Stage trace (measurement): while set, CTA `cta` of every launch writes
+ * %globaltimer stamps (ns) to dev_buf, a device buffer of `capacity` u64
+ * owned by the caller.  Per step it writes n_layers*16 + 4 slots: for each
+ * layer QKV begin, QKV input ready, QKV done, attention done, O input
+ * ready, O done, gate/up input ready, gate/up done, down input ready, down
+ * done, and (CTAs with attention work) q ready, attention math done,
+ * partial published, combine done (slots 10-13; 14-15 unused); then
+ * LM-head begin, input ready, GEMV done, pick known.  Steps beyond the
+ * capacity are not traced.  NULL turns tracing off. */
+KIE_API kie_status kie_set_trace(kie_ctx *ctx, uint64_t *dev_buf, int32_t capacity, int32_t cta);
+
 KIE_API kie_status kie_set_option(kie_ctx *ctx, kie_option opt, int64_t value);
 KIE_API kie_status kie_get_stats(const kie_ctx *ctx, kie_stats *out);
 KIE_API const char *kie_status_str(kie_status s);
 /* Text of the last error on this context ("" if none); valid until the next call. */
 KIE_API const char *kie_last_error(const kie_ctx *ctx);
 KIE_API kie_status kie_destroy(kie_ctx *ctx);
+
+/* The decode kernel's weight-stream GEMV engine run alone, for unit tests
+ * and bandwidth measurement: y[N] = W[N][K] x[K] with W fp16 row-major and
+ * x, y fp32 (all device pointers, 16-byte aligned; K a multiple of 256),
+ * computed `iters` times in one launch of one CTA per SM (the rows split as
+ * the LM-head stage splits the vocabulary).  mode 1 computes y; mode 0
+ * only streams W through the shared-memory ring (y untouched).
+ * chunk_bytes: largest streamed chunk (>= 8192, multiple of 512).  *ms_out
+ * (nullable): device time of the GEMV launch.  stats_out (nullable, 4
+ * doubles): mean per-CTA cycles the consumers waited for the stream, mean
+ * producer cycles waiting for ring space, CTAs, ring bytes.  Allocates and
+ * frees its own scratch, including a stream-ordered copy of W; synchronous
+ * on `cuda_stream`. */
+KIE_API kie_status kie_gemv_f16(const void *W, const float *x, float *y, int32_t N, int32_t K,
+                                int32_t iters, int32_t mode, int32_t chunk_bytes,
+                                void *cuda_stream, float *ms_out, double *stats_out);
 
 /* Host-only planning query (no CUDA call): the unit range [begin, end) that
  * CTA `cta` of a `grid`-CTA launch owns in GEMV stage `stage` (0 QKV, 1 O,

@@ -15,7 +15,7 @@ from . import _kie
 from ._kie import (KieError, kie_check_desc, kie_create, kie_decode, kie_decode_forced,  # noqa: F401
                    kie_destroy, kie_get_stats, kie_kv_cache_bytes, kie_last_error,
                    kie_plan_units, kie_prefill, kie_rewind, kie_set_logits_capture,
-                   kie_set_option, load_library, make_desc)
+                   kie_set_option, kie_set_trace, load_library, make_desc)
 
 __all__ = ["Session", "KieError", "load_library", "make_desc", "upload_weights"]
 
@@ -80,6 +80,19 @@ class Session:
     def capture_off(self) -> None:
         kie_set_logits_capture(self.ctx, None, 0)
         self._capture = None
+
+    def trace(self, steps: int, cta: int = 0):
+        """Turns the stage trace on for `steps` steps of CTA `cta`; returns the
+        [steps, n_layers*16 + 4] int64 device buffer it fills."""
+        import torch
+        per = self.shape.n_layers * 16 + 4
+        self._trace = torch.zeros((steps, per), dtype=torch.int64, device="cuda")
+        kie_set_trace(self.ctx, self._trace, steps * per, cta)
+        return self._trace
+
+    def trace_off(self) -> None:
+        kie_set_trace(self.ctx, None, 0, 0)
+        self._trace = None
 
     def set_option(self, opt: int, value: int) -> None:
         kie_set_option(self.ctx, opt, value)

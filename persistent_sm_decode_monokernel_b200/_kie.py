@@ -27,12 +27,14 @@ KIE_ERR_TIMEOUT = 6
 KIE_ERR_PROTOCOL = 7
 
 KIE_OPT_TIMEOUT_NS = 1
-KIE_OPT_SLOT_BYTES = 2
+KIE_OPT_CHUNK_BYTES = 2
 KIE_OPT_MIN_SPLIT_LEN = 3
 KIE_OPT_FAULT_CTA = 4
 KIE_OPT_FAULT_STEP = 5
 KIE_OPT_FAULT_LAYER = 6
 KIE_OPT_FAULT_STAGE = 7
+KIE_OPT_POLL_BACKOFF_NS = 8
+KIE_OPT_TRACE_CLOCK = 9
 
 STAGE_QKV, STAGE_O, STAGE_GU, STAGE_DOWN, STAGE_LM = range(5)
 
@@ -58,11 +60,12 @@ class KieWeights(ctypes.Structure):
 
 class KieStats(ctypes.Structure):
     _fields_ = [("pos", ctypes.c_int32), ("grid", ctypes.c_int32),
-                ("ring_slots", ctypes.c_int32), ("slot_bytes", ctypes.c_int32),
+                ("ring_bytes", ctypes.c_int32), ("chunk_bytes", ctypes.c_int32),
                 ("smem_bytes", ctypes.c_int32), ("last_steps", ctypes.c_int32),
                 ("last_device_ms", ctypes.c_float), ("launches", ctypes.c_uint64),
                 ("loop_cycles", ctypes.c_double), ("sync_wait_cycles", ctypes.c_double),
-                ("stream_wait_cycles", ctypes.c_double), ("sync_wait_max_frac", ctypes.c_double)]
+                ("stream_wait_cycles", ctypes.c_double), ("producer_wait_cycles", ctypes.c_double),
+                ("sync_wait_max_frac", ctypes.c_double)]
 
 
 _P = ctypes.c_void_p
@@ -82,11 +85,15 @@ SIGNATURES = {
     "kie_rewind": (ctypes.c_int, [_P, _I32]),
     "kie_set_logits_capture": (ctypes.c_int, [_P, _P, _I32]),
     "kie_set_option": (ctypes.c_int, [_P, ctypes.c_int, ctypes.c_int64]),
+    "kie_set_trace": (ctypes.c_int, [_P, _P, _I32, _I32]),
     "kie_get_stats": (ctypes.c_int, [_P, ctypes.POINTER(KieStats)]),
     "kie_status_str": (ctypes.c_char_p, [ctypes.c_int]),
     "kie_last_error": (ctypes.c_char_p, [_P]),
     "kie_destroy": (ctypes.c_int, [_P]),
     "kie_plan_units": (ctypes.c_int, [_PDESC, _I32, _I32, _I32, _PI32, _PI32]),
+    "kie_gemv_f16": (ctypes.c_int, [_P, _P, _P, _I32, _I32, _I32, _I32, _I32, _P,
+                                    ctypes.POINTER(ctypes.c_float),
+                                    ctypes.POINTER(ctypes.c_double)]),
 }
 
 _lib: Optional[ctypes.CDLL] = None
@@ -215,6 +222,12 @@ def kie_set_logits_capture(ctx, logits=None, rows: int = 0) -> None:
            "kie_set_logits_capture", ctx)
 
 
+def kie_set_trace(ctx, buf=None, capacity: int = 0, cta: int = 0) -> None:
+    ptr = _ptr(buf) if buf is not None else None
+    _check(load_library().kie_set_trace(ctx, ptr, capacity if buf is not None else 0, cta),
+           "kie_set_trace", ctx)
+
+
 def kie_set_option(ctx, opt: int, value: int) -> None:
     _check(load_library().kie_set_option(ctx, opt, int(value)), "kie_set_option", ctx)
 
@@ -227,6 +240,19 @@ def kie_get_stats(ctx) -> Dict[str, float]:
 
 def kie_last_error(ctx) -> str:
     return (load_library().kie_last_error(ctx) or b"").decode()
+
+
+def kie_gemv_f16(W, x, y, iters: int = 1, mode: int = 1, chunk_bytes: int = 32768, stream=None):
+    """y = W x with the decode kernel's GEMV engine; returns (ms, stats dict)."""
+    N, K = W.shape
+    ms = ctypes.c_float()
+    st = (ctypes.c_double * 4)()
+    _check(load_library().kie_gemv_f16(_ptr(W), _ptr(x), _ptr(y) if y is not None else None,
+                                       N, K, iters, mode, chunk_bytes,
+                                       ctypes.c_void_p(stream or 0), ctypes.byref(ms), st),
+           "kie_gemv_f16")
+    return ms.value, {"stream_wait_cycles": st[0], "producer_wait_cycles": st[1],
+                      "grid": int(st[2]), "ring_bytes": int(st[3])}
 
 
 def kie_destroy(ctx) -> None:

@@ -48,7 +48,10 @@ struct kie_ctx {
 
   // plan
   std::vector<std::vector<int2>> hranges;
-  int grid = 0, slots_n = 0, slot_bytes = 20480, smem = 0, max_split = 1, min_split_len = 64;
+  int grid = 0, ring_bytes = 0, chunk_bytes = 32768, smem = 0, max_split = 1, min_split_len = 64;
+  unsigned char* packed = nullptr;            // weight matrices in per-CTA stream order
+  unsigned long long* packed_off = nullptr;   // [grid]
+  size_t packed_bytes = 0;
   kie::SmemLayout sm{};
 
   // session
@@ -61,9 +64,12 @@ struct kie_ctx {
 
   // options and capture
   long long timeout_ns = 2000000000LL;
+  unsigned poll_ns = 128;
   int fault_cta = -1, fault_step = -1, fault_layer = -1, fault_stage = -1;
   float* capture = nullptr;
   int capture_rows = 0;
+  unsigned long long* trace = nullptr;
+  int trace_cta = 0, trace_steps = 0, trace_clock = 0;
 
   kie_stats stats{};
   std::string err;
@@ -107,6 +113,8 @@ void free_all(kie_ctx* c) {
   cudaFree(c->d_ids);
   cudaFree(c->d_io);
   cudaFree(c->cta_stats);
+  cudaFree(c->packed);
+  cudaFree(c->packed_off);
   if (c->h_io) cudaFreeHost(c->h_io);
   if (c->ev0) cudaEventDestroy(c->ev0);
   if (c->ev1) cudaEventDestroy(c->ev1);
@@ -149,8 +157,10 @@ kie_status launch(kie_ctx* c, int n_steps, int pos0, const int32_t* host_ids, bo
   p.rope = c->rope;
   p.ranges = c->ranges;
   p.grid = c->grid;
-  p.ring_slots = c->slots_n;
-  p.slot_bytes = c->slot_bytes;
+  p.ring_bytes = c->ring_bytes;
+  p.chunk_bytes = c->chunk_bytes;
+  p.packed = c->packed;
+  p.packed_off = c->packed_off;
   p.max_split = c->max_split;
   p.min_split_len = c->min_split_len;
   p.sm = c->sm;
@@ -175,6 +185,11 @@ kie_status launch(kie_ctx* c, int n_steps, int pos0, const int32_t* host_ids, bo
   p.status = reinterpret_cast<DevStatus*>(c->d_io);
   p.cta_stats = c->cta_stats;
   p.timeout_ns = c->timeout_ns;
+  p.poll_ns = c->poll_ns;
+  p.trace = c->trace;
+  p.trace_cta = c->trace_cta;
+  p.trace_steps = c->trace_steps;
+  p.trace_clock = c->trace_clock;
   p.fault_cta = c->fault_cta;
   p.fault_step = c->fault_step;
   p.fault_layer = c->fault_layer;
@@ -204,6 +219,41 @@ kie_status launch(kie_ctx* c, int n_steps, int pos0, const int32_t* host_ids, bo
                   st->step, st->layer, st->stage, st->where);
     return set_err(c, st->code == kie::DEV_TIMEOUT ? KIE_ERR_TIMEOUT : KIE_ERR_PROTOCOL, buf);
   }
+  return KIE_OK;
+}
+
+// (Re)builds the library's stream-ordered copy of the weight matrices for
+// the current partition and chunk size.  Reads the caller's matrices.
+kie_status repack(kie_ctx* c) {
+  std::vector<unsigned long long> off(c->grid);
+  size_t total = 0;
+  for (int i = 0; i < c->grid; ++i) {
+    off[i] = total;
+    total += (kie::stream_bytes(c->shape, c->hranges, i) + 511) / 512 * 512;
+  }
+  cudaFree(c->packed);
+  c->packed = nullptr;
+  if (!c->packed_off) KIE_CUDA(c, cudaMalloc(&c->packed_off, sizeof(unsigned long long) * c->grid));
+  KIE_CUDA(c, cudaMalloc(&c->packed, total));
+  c->packed_bytes = total;
+  KIE_CUDA(c, cudaMemcpyAsync(c->packed_off, off.data(), sizeof(unsigned long long) * c->grid,
+                              cudaMemcpyHostToDevice, c->stream));
+  MonoParams p{};
+  p.L = c->desc.n_layers;
+  p.d = c->desc.d_model;
+  p.H = c->desc.n_heads;
+  p.KV = c->desc.n_kv_heads;
+  p.hd = c->desc.head_dim;
+  p.F = c->desc.ffn_dim;
+  p.V = c->desc.vocab;
+  p.layers = c->dlayers;
+  p.lm_head = c->lm_head;
+  p.ranges = c->ranges;
+  p.grid = c->grid;
+  p.chunk_bytes = c->chunk_bytes;
+  p.packed_off = c->packed_off;
+  KIE_CUDA(c, kie::repack_launch(p, c->packed, c->stream));
+  KIE_CUDA(c, cudaStreamSynchronize(c->stream));
   return KIE_OK;
 }
 
@@ -310,13 +360,14 @@ kie_status kie_create(const kie_model_desc* d, const kie_weights* w, void* kv_ca
   c->grid = grid;
   c->hranges.resize(kie::N_STAGES);
   for (int st = 0; st < kie::N_STAGES; ++st) c->hranges[st] = kie::partition(c->shape, grid, st);
-  if (!kie::plan_smem(c->shape, grid, c->slot_bytes, smem_optin, c->hranges, &c->sm, &c->slots_n))
+  if (!kie::plan_smem(c->shape, grid, c->chunk_bytes, smem_optin, c->hranges, &c->sm,
+                      &c->ring_bytes))
     return fail(KIE_ERR_UNSUPPORTED);
   c->smem = c->sm.total;
   int per_sm = 0;
   if (cuda_bad(kie::mono_configure(d->head_dim, c->smem, &per_sm))) return fail(KIE_ERR_CUDA);
   if (per_sm < 1) return fail(KIE_ERR_UNSUPPORTED);
-  c->max_split = std::max(1, grid / d->n_kv_heads);
+  c->max_split = std::max(1, std::min(grid / d->n_kv_heads, kie::kMaxSplitCombine));
 
   const int G = d->n_heads / d->n_kv_heads;
   const size_t qd = (size_t)d->n_heads * d->head_dim, kvd = (size_t)d->n_kv_heads * d->head_dim;
@@ -340,7 +391,7 @@ kie_status kie_create(const kie_model_desc* d, const kie_weights* w, void* kv_ca
       cuda_bad(cudaMalloc(&c->att_ctr, sizeof(unsigned) * d->n_layers * d->n_kv_heads)) ||
       cuda_bad(cudaMalloc(&c->d_ids, sizeof(int32_t) * d->max_seq)) ||
       cuda_bad(cudaMalloc(&c->d_io, kStatusBytes + sizeof(int32_t) * d->max_seq)) ||
-      cuda_bad(cudaMalloc(&c->cta_stats, sizeof(unsigned long long) * 4 * grid)) ||
+      cuda_bad(cudaMalloc(&c->cta_stats, sizeof(unsigned long long) * kie::kStatsPerCta * grid)) ||
       cuda_bad(cudaMallocHost(&c->h_io, kStatusBytes + sizeof(int32_t) * d->max_seq)) ||
       cuda_bad(cudaEventCreate(&c->ev0)) || cuda_bad(cudaEventCreate(&c->ev1)))
     return fail(KIE_ERR_CUDA);
@@ -361,14 +412,15 @@ kie_status kie_create(const kie_model_desc* d, const kie_weights* w, void* kv_ca
       cuda_bad(cudaMemsetAsync(c->tagged, 0, 8 * c->tagged_words, c->stream)) ||
       cuda_bad(cudaMemsetAsync(c->att_ctr, 0, sizeof(unsigned) * d->n_layers * d->n_kv_heads,
                                c->stream)) ||
-      cuda_bad(cudaMemsetAsync(c->cta_stats, 0, sizeof(unsigned long long) * 4 * grid,
+      cuda_bad(cudaMemsetAsync(c->cta_stats, 0, sizeof(unsigned long long) * kie::kStatsPerCta * grid,
                                c->stream)) ||
       cuda_bad(cudaStreamSynchronize(c->stream)))
     return fail(KIE_ERR_CUDA);
 
+  if (repack(c) != KIE_OK) return fail(KIE_ERR_CUDA);
   c->stats.grid = grid;
-  c->stats.ring_slots = c->slots_n;
-  c->stats.slot_bytes = c->slot_bytes;
+  c->stats.ring_bytes = c->ring_bytes;
+  c->stats.chunk_bytes = c->chunk_bytes;
   c->stats.smem_bytes = c->smem;
   *out = c;
   return KIE_OK;
@@ -462,6 +514,147 @@ kie_status kie_set_logits_capture(kie_ctx* c, float* dev_logits, int32_t rows) {
   return KIE_OK;
 }
 
+kie_status kie_gemv_f16(const void* W, const float* x, float* y, int32_t N, int32_t K,
+                        int32_t iters, int32_t mode, int32_t chunk_bytes, void* stream,
+                        float* ms_out, double* stats_out) {
+  if (!W || !x || (!y && mode == 1) || N < 1 || K < 256 || K % 256 || iters < 1 ||
+      (mode != 0 && mode != 1) || chunk_bytes < 8192 || chunk_bytes % 512)
+    return KIE_ERR_INVALID_ARG;
+  if (!aligned16(W) || !aligned16(x)) return KIE_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int dev = 0, n_sm = 0, smem_optin = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) !=
+          cudaSuccess)
+    return KIE_ERR_CUDA;
+  const int grid = std::min(n_sm, N);
+  // one layer whose four layer stages own no rows; the LM-head stage is W
+  kie::Shape sh{1, K, 1, 1, 64, 256, N};
+  std::vector<std::vector<int2>> ranges(kie::N_STAGES, std::vector<int2>(grid, make_int2(0, 0)));
+  ranges[kie::ST_LM] = kie::partition(sh, grid, kie::ST_LM);
+  std::vector<int2> flat;
+  for (auto& v : ranges) flat.insert(flat.end(), v.begin(), v.end());
+  int maxrows = 0;
+  std::vector<unsigned long long> off(grid);
+  size_t total = 0;
+  for (int c = 0; c < grid; ++c) {
+    maxrows = std::max(maxrows, ranges[kie::ST_LM][c].y - ranges[kie::ST_LM][c].x);
+    off[c] = total;
+    total += (size_t)(ranges[kie::ST_LM][c].y - ranges[kie::ST_LM][c].x) * K * 2;
+  }
+  kie::SmemLayout L{};
+  L.xs_bytes = (K * 4 + 127) / 128 * 128;
+  L.rowacc_rows = maxrows;
+  L.resid_rows = 0;
+  const int fixed = 256 + L.xs_bytes + (maxrows * 4 + 127) / 128 * 128 + 256;
+  const int ring = (smem_optin - fixed) / 512 * 512;
+  if (ring < 2 * chunk_bytes) return KIE_ERR_UNSUPPORTED;
+  L.ring_off = 0;
+  L.bar_off = ring;
+  L.xs_off = L.bar_off + 256;
+  L.rowacc_off = L.xs_off + L.xs_bytes;
+  L.misc_off = L.rowacc_off + (maxrows * 4 + 127) / 128 * 128;
+  L.total = L.misc_off + 256;
+
+  int2* d_ranges = nullptr;
+  DevStatus* d_status = nullptr;
+  unsigned long long* d_stats = nullptr;
+  unsigned long long* d_off = nullptr;
+  unsigned char* d_packed = nullptr;
+  LayerW* d_layer = nullptr;
+  cudaEvent_t e0 = nullptr, e1 = nullptr;
+  kie_status ret = KIE_OK;
+  if (cudaMalloc(&d_ranges, sizeof(int2) * flat.size()) != cudaSuccess ||
+      cudaMalloc(&d_status, sizeof(DevStatus)) != cudaSuccess ||
+      cudaMalloc(&d_stats, sizeof(unsigned long long) * kie::kStatsPerCta * grid) != cudaSuccess ||
+      cudaMalloc(&d_off, sizeof(unsigned long long) * grid) != cudaSuccess ||
+      cudaMalloc(&d_packed, total) != cudaSuccess ||
+      cudaMalloc(&d_layer, sizeof(LayerW)) != cudaSuccess ||
+      cudaEventCreate(&e0) != cudaSuccess || cudaEventCreate(&e1) != cudaSuccess) {
+    ret = KIE_ERR_CUDA;
+  }
+  MonoParams p{};
+  if (ret == KIE_OK) {
+    p.L = 1;
+    p.d = K;
+    p.H = 1;
+    p.KV = 1;
+    p.hd = 64;
+    p.F = 256;
+    p.V = N;
+    p.G = 1;
+    p.layers = d_layer;
+    p.lm_head = static_cast<const __half*>(W);
+    p.ranges = d_ranges;
+    p.grid = grid;
+    p.ring_bytes = ring;
+    p.chunk_bytes = chunk_bytes;
+    p.packed = d_packed;
+    p.packed_off = d_off;
+    p.sm = L;
+    p.status = d_status;
+    p.cta_stats = d_stats;
+    p.timeout_ns = 2000000000LL;
+    p.poll_ns = 128;
+    p.fault_cta = -1;
+    if (cudaMemcpyAsync(d_ranges, flat.data(), sizeof(int2) * flat.size(),
+                        cudaMemcpyHostToDevice, st) != cudaSuccess ||
+        cudaMemcpyAsync(d_off, off.data(), sizeof(unsigned long long) * grid,
+                        cudaMemcpyHostToDevice, st) != cudaSuccess ||
+        cudaMemsetAsync(d_status, 0, sizeof(DevStatus), st) != cudaSuccess ||
+        cudaMemsetAsync(d_stats, 0, sizeof(unsigned long long) * kie::kStatsPerCta * grid, st) !=
+            cudaSuccess ||
+        cudaMemsetAsync(d_layer, 0, sizeof(LayerW), st) != cudaSuccess ||
+        kie::repack_launch(p, d_packed, st) != cudaSuccess ||
+        kie::gemv_configure(L.total) != cudaSuccess || cudaEventRecord(e0, st) != cudaSuccess ||
+        kie::gemv_launch(p, mode, x, y, iters, grid, L.total, st) != cudaSuccess ||
+        cudaEventRecord(e1, st) != cudaSuccess || cudaStreamSynchronize(st) != cudaSuccess)
+      ret = KIE_ERR_CUDA;
+  }
+  if (ret == KIE_OK) {
+    float ms = 0.f;
+    cudaEventElapsedTime(&ms, e0, e1);
+    if (ms_out) *ms_out = ms;
+    DevStatus hs{};
+    cudaMemcpy(&hs, d_status, sizeof hs, cudaMemcpyDeviceToHost);
+    if (hs.code != kie::DEV_OK) ret = hs.code == kie::DEV_TIMEOUT ? KIE_ERR_TIMEOUT : KIE_ERR_PROTOCOL;
+    if (stats_out) {
+      std::vector<unsigned long long> h((size_t)kie::kStatsPerCta * grid);
+      cudaMemcpy(h.data(), d_stats, sizeof(unsigned long long) * h.size(), cudaMemcpyDeviceToHost);
+      double stream = 0, prod = 0;
+      for (int c = 0; c < grid; ++c) {
+        stream += (double)h[(size_t)kie::kStatsPerCta * c + 2];
+        prod += (double)h[(size_t)kie::kStatsPerCta * c + 3];
+      }
+      stats_out[0] = stream / grid;
+      stats_out[1] = prod / grid;
+      stats_out[2] = grid;
+      stats_out[3] = ring;
+    }
+  }
+  cudaFree(d_ranges);
+  cudaFree(d_status);
+  cudaFree(d_stats);
+  cudaFree(d_off);
+  cudaFree(d_packed);
+  cudaFree(d_layer);
+  if (e0) cudaEventDestroy(e0);
+  if (e1) cudaEventDestroy(e1);
+  return ret;
+}
+
+kie_status kie_set_trace(kie_ctx* c, uint64_t* dev_buf, int32_t capacity, int32_t cta) {
+  if (!c) return KIE_ERR_INVALID_ARG;
+  if (dev_buf && (capacity < 1 || cta < 0 || cta >= c->grid))
+    return set_err(c, KIE_ERR_INVALID_ARG, "bad trace buffer or CTA");
+  const int per = c->desc.n_layers * kie::kTracePerLayer + 4;
+  c->trace = reinterpret_cast<unsigned long long*>(dev_buf);
+  c->trace_cta = cta;
+  c->trace_steps = dev_buf ? capacity / per : 0;
+  return KIE_OK;
+}
+
 kie_status kie_set_option(kie_ctx* c, kie_option opt, int64_t v) {
   if (!c) return KIE_ERR_INVALID_ARG;
   switch (opt) {
@@ -469,31 +662,39 @@ kie_status kie_set_option(kie_ctx* c, kie_option opt, int64_t v) {
       if (v < 1000) return KIE_ERR_INVALID_ARG;
       c->timeout_ns = v;
       return KIE_OK;
-    case KIE_OPT_SLOT_BYTES: {
-      if (v < 4096 || v % 4096 || v > (1 << 20)) return KIE_ERR_INVALID_ARG;
+    case KIE_OPT_CHUNK_BYTES: {
+      if (c->failed) return set_err(c, KIE_ERR_STATE, "context failed earlier; destroy it");
+      if (v < 8192 || v % 512 || v > (1 << 20)) return KIE_ERR_INVALID_ARG;
       int smem_optin = 0;
       if (cudaDeviceGetAttribute(&smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin,
                                  c->device) != cudaSuccess)
         return set_err(c, KIE_ERR_CUDA, "device attribute query failed");
       kie::SmemLayout sm{};
-      int slots = 0;
-      if (!kie::plan_smem(c->shape, c->grid, (int)v, smem_optin, c->hranges, &sm, &slots))
-        return set_err(c, KIE_ERR_UNSUPPORTED, "slot size does not fit shared memory");
+      int ring = 0;
+      if (!kie::plan_smem(c->shape, c->grid, (int)v, smem_optin, c->hranges, &sm, &ring))
+        return set_err(c, KIE_ERR_UNSUPPORTED, "chunk size does not fit shared memory");
       int per_sm = 0;
       if (kie::mono_configure(c->desc.head_dim, sm.total, &per_sm) != cudaSuccess || per_sm < 1)
-        return set_err(c, KIE_ERR_UNSUPPORTED, "kernel does not fit with this slot size");
-      c->slot_bytes = (int)v;
+        return set_err(c, KIE_ERR_UNSUPPORTED, "kernel does not fit with this chunk size");
+      c->chunk_bytes = (int)v;
       c->sm = sm;
-      c->slots_n = slots;
+      c->ring_bytes = ring;
       c->smem = sm.total;
-      c->stats.ring_slots = slots;
-      c->stats.slot_bytes = (int)v;
+      c->stats.ring_bytes = ring;
+      c->stats.chunk_bytes = (int)v;
       c->stats.smem_bytes = sm.total;
-      return KIE_OK;
+      return repack(c);
     }
     case KIE_OPT_MIN_SPLIT_LEN:
       if (v < 1 || v > (1 << 20)) return KIE_ERR_INVALID_ARG;
       c->min_split_len = (int)v;
+      return KIE_OK;
+    case KIE_OPT_TRACE_CLOCK:
+      c->trace_clock = v ? 1 : 0;
+      return KIE_OK;
+    case KIE_OPT_POLL_BACKOFF_NS:
+      if (v < 0 || v > 100000) return KIE_ERR_INVALID_ARG;
+      c->poll_ns = (unsigned)v;
       return KIE_OK;
     case KIE_OPT_FAULT_CTA: c->fault_cta = (int)v; return KIE_OK;
     case KIE_OPT_FAULT_STEP: c->fault_step = (int)v; return KIE_OK;
@@ -508,19 +709,22 @@ kie_status kie_get_stats(const kie_ctx* cc, kie_stats* out) {
   kie_ctx* c = const_cast<kie_ctx*>(cc);
   *out = c->stats;
   if (c->stats.launches > 0 && c->cta_stats) {
-    std::vector<unsigned long long> st((size_t)4 * c->grid);
+    const int K = kie::kStatsPerCta;
+    std::vector<unsigned long long> st((size_t)K * c->grid);
     if (cudaMemcpy(st.data(), c->cta_stats, sizeof(unsigned long long) * st.size(),
                    cudaMemcpyDeviceToHost) == cudaSuccess) {
-      double loop = 0, sync = 0, stream = 0, mx = 0;
+      double loop = 0, sync = 0, stream = 0, prod = 0, mx = 0;
       for (int i = 0; i < c->grid; ++i) {
-        loop += (double)st[4 * i];
-        sync += (double)st[4 * i + 1];
-        stream += (double)st[4 * i + 2];
-        if (st[4 * i] > 0) mx = std::max(mx, (double)st[4 * i + 1] / (double)st[4 * i]);
+        loop += (double)st[K * i];
+        sync += (double)st[K * i + 1];
+        stream += (double)st[K * i + 2];
+        prod += (double)st[K * i + 3];
+        if (st[K * i] > 0) mx = std::max(mx, (double)st[K * i + 1] / (double)st[K * i]);
       }
       out->loop_cycles = loop / c->grid;
       out->sync_wait_cycles = sync / c->grid;
       out->stream_wait_cycles = stream / c->grid;
+      out->producer_wait_cycles = prod / c->grid;
       out->sync_wait_max_frac = mx;
     }
   }

@@ -46,38 +46,51 @@ using u64 = unsigned long long;
 
 namespace {
 
-enum : int { F_ABORT = 0, F_STOP = 1, F_LAST = 2 };
+enum : int { F_ABORT = 0, F_STOP = 1, F_LAST = 2, F_KVSTEP = 3 };
 
-struct Smem {
-  unsigned char* ring;
-  uint32_t ring_s;
-  uint32_t full_s, empty_s;
-  float* xs;
-  float* rowacc;
-  float* part;        // [8] tail-group partial sums
-  float* red;         // [8] reduction scratch
-  float* red2;        // [8]
-  int* redi;          // [8]
-  int* redi2;         // [8]
-  volatile int* flags;
-};
+// The dynamic shared-memory block.  Pointers derived from it directly keep
+// their address space, so the compiler emits shared-memory loads for them.
+extern __shared__ __align__(128) unsigned char kie_smem[];
 
-__device__ __forceinline__ Smem carve(const MonoParams& p, unsigned char* base) {
-  Smem S;
-  S.ring = base + p.sm.ring_off;
-  S.ring_s = dev::smem_u32(S.ring);
-  S.full_s = dev::smem_u32(base + p.sm.bar_off);
-  S.empty_s = S.full_s + 8 * kMaxSlots;
-  S.xs = reinterpret_cast<float*>(base + p.sm.xs_off);
-  S.rowacc = reinterpret_cast<float*>(base + p.sm.rowacc_off);
-  float* m = reinterpret_cast<float*>(base + p.sm.misc_off);
-  S.part = m;
-  S.red = m + 8;
-  S.red2 = m + 16;
-  S.redi = reinterpret_cast<int*>(m + 24);
-  S.redi2 = reinterpret_cast<int*>(m + 32);
-  S.flags = reinterpret_cast<volatile int*>(m + 40);
-  return S;
+// Views of the dynamic shared memory, always derived from the __shared__
+// symbol so that every access compiles to a shared-memory instruction.
+__device__ __forceinline__ float* sm_xs(const MonoParams& p) {
+  return reinterpret_cast<float*>(kie_smem + p.sm.xs_off);
+}
+__device__ __forceinline__ float* sm_rowacc(const MonoParams& p) {
+  return reinterpret_cast<float*>(kie_smem + p.sm.rowacc_off);
+}
+__device__ __forceinline__ float* sm_misc(const MonoParams& p) {
+  return reinterpret_cast<float*>(kie_smem + p.sm.misc_off);
+}
+__device__ __forceinline__ float* sm_part(const MonoParams& p) { return sm_misc(p); }       // [8]
+__device__ __forceinline__ float* sm_red(const MonoParams& p) { return sm_misc(p) + 8; }    // [8]
+__device__ __forceinline__ float* sm_red2(const MonoParams& p) { return sm_misc(p) + 16; }  // [8]
+__device__ __forceinline__ int* sm_redi(const MonoParams& p) {
+  return reinterpret_cast<int*>(sm_misc(p) + 24);
+}
+__device__ __forceinline__ int* sm_redi2(const MonoParams& p) {
+  return reinterpret_cast<int*>(sm_misc(p) + 32);
+}
+__device__ __forceinline__ volatile int* sm_flags(const MonoParams& p) {
+  return reinterpret_cast<volatile int*>(sm_misc(p) + 40);
+}
+// residual stream rows this CTA owns (O / down stages)
+__device__ __forceinline__ float* sm_res_attn(const MonoParams& p) { return sm_misc(p) + 64; }
+__device__ __forceinline__ float* sm_res_ffn(const MonoParams& p) {
+  return sm_misc(p) + 64 + p.sm.resid_rows;
+}
+__device__ __forceinline__ const unsigned char* sm_ring(const MonoParams& p) {
+  return kie_smem + p.sm.ring_off;
+}
+__device__ __forceinline__ uint32_t sm_ring_s(const MonoParams& p) {
+  return dev::smem_u32(kie_smem + p.sm.ring_off);
+}
+__device__ __forceinline__ uint32_t sm_full_s(const MonoParams& p) {
+  return dev::smem_u32(kie_smem + p.sm.bar_off);
+}
+__device__ __forceinline__ uint32_t sm_empty_s(const MonoParams& p) {
+  return sm_full_s(p) + 8 * kRingBars;
 }
 
 // ------------------------------------------------------------ stage geometry
@@ -138,21 +151,58 @@ __device__ __forceinline__ const __half* row_ptr(const MonoParams& p, int st, co
   }
 }
 
-// k-chunking of one group of rg (<= 8) rows with kp pieces per row: chunk kc
-// covers pieces [first(kc), first(kc+1)) of every row of the group.
+// k-chunking of one group of rg (<= kGroupRows) rows with kp pieces per row into nk
+// chunks of at most chunk_bytes: chunk kc holds count(kc) pieces of every
+// row of the group, starting at piece first(kc).  Stored [row][piece][512 B].
 struct Chunking {
-  int kp, nk;
-  __device__ __forceinline__ int first(int kc) const {
-    return (int)(((long long)kc * kp) / nk);
-  }
+  int nk, base, rem;
+  __device__ __forceinline__ int first(int kc) const { return kc * base + min(kc, rem); }
+  __device__ __forceinline__ int count(int kc) const { return base + (kc < rem ? 1 : 0); }
 };
-__device__ __forceinline__ Chunking chunking(int rg, int kp, int slot_bytes) {
-  int mp = slot_bytes / (rg * kPieceBytes);
+__device__ __forceinline__ Chunking chunking(int rg, int kp, int chunk_bytes) {
+  int mp = chunk_bytes / (rg * kPieceBytes);
   if (mp < 1) mp = 1;
   Chunking c;
-  c.kp = kp;
   c.nk = (kp + mp - 1) / mp;
+  c.base = kp / c.nk;
+  c.rem = kp - c.base * c.nk;
   return c;
+}
+
+// Byte ring placement shared by producer and consumers: a chunk goes right
+// after the previous one, or back to offset 0 when it would not fit.
+__device__ __forceinline__ uint32_t ring_place(uint32_t& wend, uint32_t sz, uint32_t ring_bytes) {
+  const uint32_t off = (wend + sz <= ring_bytes) ? wend : 0u;
+  wend = off + sz;
+  return off;
+}
+
+// This CTA's attention work item at position pos: KV head j, positions
+// [t0, t1) of 0..pos.  Items are (KV head, split) pairs, item = CTA index.
+struct AttnItem {
+  int j, t0, t1, nsplit;
+  bool valid;
+};
+__device__ __forceinline__ AttnItem attn_item(const MonoParams& p, int pos) {
+  const int n_pos = pos + 1;
+  int nsplit = (n_pos + p.min_split_len - 1) / p.min_split_len;
+  if (nsplit > p.max_split) nsplit = p.max_split;
+  AttnItem a;
+  a.nsplit = nsplit;
+  const int it = blockIdx.x;
+  a.valid = it < p.KV * nsplit;
+  a.j = it / nsplit;
+  const int s = it - a.j * nsplit;
+  a.t0 = (int)(((long long)s * n_pos) / nsplit);
+  a.t1 = (int)(((long long)(s + 1) * n_pos) / nsplit);
+  return a;
+}
+// Positions per attention block (one K chunk and one V chunk in the ring).
+__device__ __forceinline__ int attn_block(const MonoParams& p) {
+  return min(kAttnBlock, p.chunk_bytes / (p.hd * 2));
+}
+__device__ __forceinline__ const __half* kv_rows(const MonoParams& p, int layer, int kv, int j) {
+  return p.kv + (((size_t)layer * 2 + kv) * p.KV + j) * (size_t)p.max_seq * p.hd;
 }
 
 __device__ __forceinline__ unsigned epoch_of(const MonoParams& p, int step, int layer) {
@@ -178,72 +228,136 @@ __device__ __forceinline__ bool global_error(const MonoParams& p) {
 
 struct Producer {
   const MonoParams& p;
-  const Smem& S;
   uint64_t pol;
-  int slot;
-  unsigned round;
-  unsigned used_mask, par_mask;
+  uint32_t idx;    // chunks issued
+  uint32_t cons;   // chunks known to be consumed
+  uint32_t wend;   // ring write position
+  uint32_t live_off[kRingBars], live_end[kRingBars];
+  long long t_wait;  // cycles spent waiting for ring space
 
-  __device__ Producer(const MonoParams& pp, const Smem& ss)
-      : p(pp), S(ss), pol(dev::policy_evict_first()), slot(0), round(0), used_mask(0),
-        par_mask(0) {}
+  __device__ explicit Producer(const MonoParams& pp)
+      : p(pp), pol(dev::policy_evict_first()), idx(0), cons(0), wend(0), t_wait(0) {}
 
-  // Waits for the consumers to free the current slot; false = stop.
-  __device__ bool wait_free() {
-    if (round == 0) return true;
-    const uint32_t bar = S.empty_s + 8 * slot;
-    const uint32_t par = (round - 1) & 1u;
-    if (dev::mbar_try_wait(bar, par)) return true;
+  // Waits until chunk i has been consumed; false = stop.
+  __device__ bool wait_consumed(uint32_t i) {
+    const uint32_t bar = sm_empty_s(p) + 8 * (i & (kRingBars - 1));
+    const uint32_t par = (i / kRingBars) & 1u;
+    if (dev::mbar_test_wait(bar, par)) return true;
+    const long long c0 = clock64();
     const long long t0 = dev::globaltimer();
+    bool ok = true;
     for (unsigned it = 1;; ++it) {
-      if (S.flags[F_STOP]) return false;
-      if (dev::mbar_try_wait(bar, par)) return true;
+      if (sm_flags(p)[F_STOP]) {
+        ok = false;
+        break;
+      }
+      if (dev::mbar_try_wait(bar, par)) break;
       if ((it & 15u) == 0u && dev::globaltimer() - t0 > p.timeout_ns) {
         raise_error(p, DEV_TIMEOUT, -1, -1, -1, 1);
-        return false;
+        ok = false;
+        break;
       }
     }
+    t_wait += clock64() - c0;
+    return ok;
   }
 
-  __device__ bool stage(int st, int layer) {
-    const LayerW& w = p.layers[layer];
-    const int2 r = p.ranges[st * p.grid + blockIdx.x];
-    const int R = range_rows(p, st, r.x, r.y);
-    const int K = stage_k(p, st);
-    const int kp = K / kPieceElems;
-    for (int g0 = 0; g0 < R; g0 += 8) {
-      const int rg = min(8, R - g0);
-      const Chunking ch = chunking(rg, kp, p.slot_bytes);
-      for (int kc = 0; kc < ch.nk; ++kc) {
-        if (S.flags[F_STOP]) return false;
-        if (!wait_free()) return false;
-        const int p0 = ch.first(kc), n = ch.first(kc + 1) - p0;
-        const uint32_t bytes = (uint32_t)(n * kPieceBytes);
-        const uint32_t full = S.full_s + 8 * slot;
-        dev::mbar_arrive_expect_tx(full, bytes * rg);
-        const uint32_t dst = S.ring_s + (uint32_t)slot * (uint32_t)p.slot_bytes;
-        for (int j = 0; j < rg; ++j) {
-          const __half* src = row_ptr(p, st, w, r.x, r.y, g0 + j) + (size_t)p0 * kPieceElems;
-          dev::bulk_g2s(dst + (uint32_t)j * bytes, src, bytes, full, pol);
-        }
-        used_mask |= 1u << slot;
-        par_mask = (par_mask & ~(1u << slot)) | ((round & 1u) << slot);
-        if (++slot == p.ring_slots) {
-          slot = 0;
-          ++round;
-        }
+  // Frees ring bytes [off, end) and a barrier pair for the next chunk:
+  // waits, oldest first, until no live chunk overlaps the range and fewer
+  // than kRingBars chunks are live.  (When both the live region and the new
+  // chunk wrap, the overlapped chunks are not the oldest, so every live
+  // chunk is checked.)
+  __device__ bool acquire(uint32_t off, uint32_t end) {
+    while (cons < idx) {
+      bool blocked = idx - cons >= (uint32_t)kRingBars;
+      for (uint32_t j = cons; j < idx && !blocked; ++j) {
+        const uint32_t b = j & (kRingBars - 1);
+        blocked = off < live_end[b] && live_off[b] < end;
       }
+      if (!blocked) break;
+      if (!wait_consumed(cons)) return false;
+      ++cons;
     }
     return true;
   }
 
-  // Waits until every copy this producer issued has landed.
+  // One chunk = one bulk copy of the next `sz` bytes of the CTA's stream.
+  __device__ bool chunk(const unsigned char*& src, uint32_t sz) {
+    if (sm_flags(p)[F_STOP]) return false;
+    const uint32_t off = ring_place(wend, sz, (uint32_t)p.ring_bytes);
+    if (!acquire(off, off + sz)) return false;
+    const uint32_t b = idx & (kRingBars - 1);
+    const uint32_t full = sm_full_s(p) + 8 * b;
+    dev::mbar_arrive_expect_tx(full, sz);
+    dev::bulk_g2s(sm_ring_s(p) + off, src, sz, full, pol);
+    live_off[b] = off;
+    live_end[b] = off + sz;
+    src += sz;
+    ++idx;
+    return true;
+  }
+
+  __device__ bool stage(int st, const unsigned char*& src) {
+    const int2 r = p.ranges[st * p.grid + blockIdx.x];
+    const int R = range_rows(p, st, r.x, r.y);
+    const int kp = stage_k(p, st) / kPieceElems;
+    for (int g0 = 0; g0 < R; g0 += kGroupRows) {
+      const int rg = min(kGroupRows, R - g0);
+      const Chunking ch = chunking(rg, kp, p.chunk_bytes);
+      for (int kc = 0; kc < ch.nk; ++kc)
+        if (!chunk(src, (uint32_t)(rg * ch.count(kc) * kPieceBytes))) return false;
+    }
+    return true;
+  }
+
+  // K and V blocks of this CTA's attention item at step i, layer l, for the
+  // positions before pos (the current position's k/v arrive as tagged
+  // words).  The rows were written by other CTAs in earlier steps: before
+  // the first such copy of step i the producer waits until its consumers
+  // have passed step i-1's fenced publish, then orders that view before its
+  // bulk copies with a proxy fence.
+  __device__ bool attn(int i, int l) {
+    const int pos = p.pos0 + i;
+    const AttnItem it = attn_item(p, pos);
+    if (!it.valid) return true;
+    if (l == 0 && i > 0) {
+      if (dev::ld_acquire_cta(sm_flags(p) + F_KVSTEP) < i) {
+        const long long c0 = clock64();
+        const long long t0 = dev::globaltimer();
+        for (unsigned n = 1;; ++n) {
+          if (sm_flags(p)[F_STOP]) return false;
+          if (dev::ld_acquire_cta(sm_flags(p) + F_KVSTEP) >= i) break;
+          if ((n & 63u) == 0u && dev::globaltimer() - t0 > p.timeout_ns) {
+            raise_error(p, DEV_TIMEOUT, i, l, 5, 4);
+            return false;
+          }
+        }
+        t_wait += clock64() - c0;
+      }
+      dev::fence_proxy_async_global();
+    }
+    const int tb = attn_block(p);
+    const unsigned char* K = reinterpret_cast<const unsigned char*>(kv_rows(p, l, 0, it.j));
+    const unsigned char* V = reinterpret_cast<const unsigned char*>(kv_rows(p, l, 1, it.j));
+    const size_t row = (size_t)p.hd * 2;
+    for (int b0 = it.t0; b0 < it.t1; b0 += tb) {
+      const int nc = min(min(it.t1, b0 + tb), pos) - b0;
+      if (nc <= 0) continue;
+      const unsigned char* k = K + b0 * row;
+      const unsigned char* v = V + b0 * row;
+      if (!chunk(k, (uint32_t)(nc * row)) || !chunk(v, (uint32_t)(nc * row))) return false;
+    }
+    return true;
+  }
+
+  // Waits until every copy this producer issued has landed (the last
+  // kRingBars chunks; older ones were consumed before their barrier was
+  // reused).
   __device__ void drain() {
     const long long t0 = dev::globaltimer();
-    for (int s = 0; s < p.ring_slots; ++s) {
-      if (!((used_mask >> s) & 1u)) continue;
-      const uint32_t bar = S.full_s + 8 * s;
-      const uint32_t par = (par_mask >> s) & 1u;
+    for (uint32_t i = idx > (uint32_t)kRingBars ? idx - kRingBars : 0u; i < idx; ++i) {
+      const uint32_t bar = sm_full_s(p) + 8 * (i & (kRingBars - 1));
+      const uint32_t par = (i / kRingBars) & 1u;
       while (!dev::mbar_try_wait(bar, par)) {
         if (dev::globaltimer() - t0 > p.timeout_ns) {
           raise_error(p, DEV_TIMEOUT, -1, -1, -1, 2);
@@ -253,39 +367,85 @@ struct Producer {
     }
   }
 
+  // The whole call's stream: per step the CTA's packed layers, then the LM
+  // head on steps that pick an id.
   __device__ void run() {
-    for (int i = 0; i < p.n_steps; ++i) {
-      for (int l = 0; l < p.L; ++l) {
-        if (!stage(ST_QKV, l) || !stage(ST_O, l) || !stage(ST_GU, l) || !stage(ST_DOWN, l)) {
-          drain();
-          return;
-        }
-      }
-      if (i >= p.lm_from && !stage(ST_LM, 0)) {
-        drain();
-        return;
-      }
+    bool ok = true;
+    const unsigned char* base = p.packed + p.packed_off[blockIdx.x];
+    for (int i = 0; i < p.n_steps && ok; ++i) {
+      const unsigned char* src = base;
+      for (int l = 0; l < p.L && ok; ++l)
+        ok = stage(ST_QKV, src) && attn(i, l) && stage(ST_O, src) && stage(ST_GU, src) &&
+             stage(ST_DOWN, src);
+      if (ok && i >= p.lm_from) ok = stage(ST_LM, src);
     }
     drain();
+    p.cta_stats[kStatsPerCta * blockIdx.x + 3] = (unsigned long long)t_wait;
   }
 };
+
+// Lays out CTA blockIdx.x's one-token weight stream in the order Producer
+// streams it: per layer the QKV, O, gate/up and down chunks, then the LM
+// head, each chunk [row][piece][512 B].  Run once per model.
+__device__ void repack_stage(const MonoParams& p, int st, const LayerW& w, unsigned char*& dst) {
+  const int2 r = p.ranges[st * p.grid + blockIdx.x];
+  const int R = range_rows(p, st, r.x, r.y);
+  const int kp = stage_k(p, st) / kPieceElems;
+  for (int g0 = 0; g0 < R; g0 += kGroupRows) {
+    const int rg = min(kGroupRows, R - g0);
+    const Chunking ch = chunking(rg, kp, p.chunk_bytes);
+    for (int kc = 0; kc < ch.nk; ++kc) {
+      const int n = ch.count(kc), p0 = ch.first(kc);
+      const int n16 = n * kPieceBytes / 16;
+      uint4* d = reinterpret_cast<uint4*>(dst);
+      for (int e = threadIdx.x; e < rg * n16; e += blockDim.x) {
+        const int j = e / n16, q = e - j * n16;
+        const uint4* src = reinterpret_cast<const uint4*>(row_ptr(p, st, w, r.x, r.y, g0 + j) +
+                                                          (size_t)p0 * kPieceElems);
+        d[e] = src[q];
+      }
+      dst += (size_t)rg * n * kPieceBytes;
+    }
+  }
+}
 
 // ----------------------------------------------------------------- consumer
 
 struct Consumer {
   const MonoParams& p;
-  const Smem& S;
   int tid, warp, lane;
-  int slot;
-  unsigned round;
+  uint32_t cidx;   // next chunk to wait for
+  uint32_t crel;   // next chunk to release (chunks are released in order)
+  uint32_t cend;   // ring read position (mirrors the producer's placement)
   long long t_sync, t_stream;
   int step, layer, stage;  // for error reports
 
-  __device__ Consumer(const MonoParams& pp, const Smem& ss)
-      : p(pp), S(ss), slot(0), round(0), t_sync(0), t_stream(0), step(0), layer(0), stage(0) {
+  __device__ explicit Consumer(const MonoParams& pp)
+      : p(pp), cidx(0), crel(0), cend(0), t_sync(0), t_stream(0), step(0), layer(0), stage(0) {
     tid = threadIdx.x;
     warp = tid >> 5;
     lane = tid & 31;
+  }
+
+  // Stage-boundary timestamps of one CTA (measurement): per step
+  // 10 per layer (QKV begin/loaded/done, attention done, O loaded/done,
+  // gate-up loaded/done, down loaded/done) + 4 for the LM head.
+  __device__ __forceinline__ void trace(int ev) const {
+    if (p.trace && tid == 0 && (int)blockIdx.x == p.trace_cta && step < p.trace_steps) {
+      const int per = p.L * kTracePerLayer + 4;
+      const int idx = step * per + (layer < p.L ? layer * kTracePerLayer : p.L * kTracePerLayer) + ev;
+      p.trace[idx] = p.trace_clock ? (unsigned long long)clock64()
+                                   : (unsigned long long)dev::globaltimer();
+    }
+  }
+  __device__ __forceinline__ void trace_loaded() const {
+    switch (stage) {
+      case ST_QKV: trace(1); break;
+      case ST_O: trace(4); break;
+      case ST_GU: trace(6); break;
+      case ST_DOWN: trace(8); break;
+      default: trace(1); break;
+    }
   }
 
   __device__ __forceinline__ bool fault_here(int st) const {
@@ -293,68 +453,26 @@ struct Consumer {
            p.fault_stage == st;
   }
 
-  // ---- tagged-word polling
-  __device__ __noinline__ bool wait_tag_slow(const u64* a, unsigned tag, unsigned& out,
-                                             int where) {
-    const long long t0 = dev::globaltimer();
-    for (unsigned it = 1;; ++it) {
-      const u64 v = dev::ld_relaxed_u64(a);
-      const unsigned tg = (unsigned)(v >> 32);
-      if (tg == tag) {
-        out = (unsigned)v;
-        return true;
-      }
-      if (tg != 0u && (int)(tg - tag) > 0) {
-        raise_error(p, DEV_PROTOCOL, step, layer, stage, where);
-        S.flags[F_ABORT] = 1;
-        return false;
-      }
-      if ((it & 31u) == 0u) {
-        if (S.flags[F_ABORT] || global_error(p)) {
-          S.flags[F_ABORT] = 1;
-          return false;
-        }
-        if (dev::globaltimer() - t0 > p.timeout_ns) {
-          raise_error(p, DEV_TIMEOUT, step, layer, stage, where);
-          S.flags[F_ABORT] = 1;
-          return false;
-        }
-      }
-    }
-  }
-  __device__ __forceinline__ bool wait_tag(const u64* a, unsigned tag, unsigned& out, int where) {
-    const u64 v = dev::ld_relaxed_u64(a);
-    if ((unsigned)(v >> 32) == tag) {
-      out = (unsigned)v;
-      return true;
-    }
-    return wait_tag_slow(a, tag, out, where);
-  }
-  __device__ __forceinline__ bool wait_f(const u64* a, unsigned tag, float& out, int where) {
-    unsigned u;
-    const bool ok = wait_tag(a, tag, u, where);
-    out = __uint_as_float(u);
-    return ok;
-  }
-
-  // ---- ring
-  __device__ __forceinline__ bool wait_full() {
-    const uint32_t bar = S.full_s + 8 * slot;
-    const uint32_t par = round & 1u;
-    if (dev::mbar_try_wait(bar, par)) return true;
+  // ---- ring: waits for the next chunk (sz bytes) and returns its offset
+  __device__ __forceinline__ bool wait_chunk(uint32_t sz, uint32_t& off) {
+    off = ring_place(cend, sz, (uint32_t)p.ring_bytes);
+    const uint32_t bar = sm_full_s(p) + 8 * (cidx & (kRingBars - 1));
+    const uint32_t par = (cidx / kRingBars) & 1u;
+    ++cidx;
+    if (dev::mbar_test_wait(bar, par)) return true;
     const long long c0 = clock64();
     const long long t0 = dev::globaltimer();
     bool ok = true;
     for (unsigned it = 1;; ++it) {
       if (dev::mbar_try_wait(bar, par)) break;
       if ((it & 15u) == 0u) {
-        if (S.flags[F_ABORT]) {
+        if (sm_flags(p)[F_ABORT]) {
           ok = false;
           break;
         }
         if (dev::globaltimer() - t0 > p.timeout_ns) {
           raise_error(p, DEV_TIMEOUT, step, layer, stage, 3);
-          S.flags[F_ABORT] = 1;
+          sm_flags(p)[F_ABORT] = 1;
           ok = false;
           break;
         }
@@ -363,13 +481,11 @@ struct Consumer {
     if (tid == 0) t_stream += clock64() - c0;
     return ok;
   }
-  __device__ __forceinline__ void release_slot() {
+  // Releases the oldest chunk this warp waited for and has not released.
+  __device__ __forceinline__ void release_chunk() {
     __syncwarp();
-    if (lane == 0) dev::mbar_arrive(S.empty_s + 8 * slot);
-    if (++slot == p.ring_slots) {
-      slot = 0;
-      ++round;
-    }
+    if (lane == 0) dev::mbar_arrive(sm_empty_s(p) + 8 * (crel & (kRingBars - 1)));
+    ++crel;
   }
 
   // ---- permuted activation layout: element k of a K-vector sits where
@@ -380,95 +496,248 @@ struct Consumer {
     return (e < 4 ? 0 : (K >> 1)) + ((piece * 32 + ln) << 2) + (e & 3);
   }
 
+  // Polls NB pairs of tagged words (pair b at src + 2*k2[b], used when
+  // k2[b] < n2) until every word carries `tag`.  All pending pairs are
+  // re-read together, so a round costs one L2 round trip; rounds after the
+  // first back off for kPollBackoffNs so that waiting CTAs do not flood L2
+  // while their producers work.  Returns false on abort, timeout or a word
+  // that carries a newer tag (protocol violation).
+  template <int NB>
+  __device__ __forceinline__ bool poll_pairs(const u64* src, const int (&k2)[NB], int n2,
+                                             unsigned tag, ulonglong2 (&v)[NB], int where) {
+    unsigned pend = 0;
+#pragma unroll
+    for (int b = 0; b < NB; ++b)
+      if (k2[b] < n2) {
+        v[b] = dev::ld_relaxed_v2_u64(src + 2 * k2[b]);
+        pend |= 1u << b;
+      }
+    long long t0 = 0;
+    for (unsigned it = 0;; ++it) {
+      bool newer = false;
+#pragma unroll
+      for (int b = 0; b < NB; ++b) {
+        if ((pend >> b) & 1u) {
+          const unsigned tx = (unsigned)(v[b].x >> 32), ty = (unsigned)(v[b].y >> 32);
+          if (tx == tag && ty == tag) pend &= ~(1u << b);
+          newer |= (tx != 0u && (int)(tx - tag) > 0) || (ty != 0u && (int)(ty - tag) > 0);
+        }
+      }
+      if (!pend) return true;
+      if (newer) {
+        raise_error(p, DEV_PROTOCOL, step, layer, stage, where);
+        sm_flags(p)[F_ABORT] = 1;
+        return false;
+      }
+      if (it == 0) {
+        t0 = dev::globaltimer();
+      } else if ((it & 7u) == 0u) {
+        if (sm_flags(p)[F_ABORT] || global_error(p)) {
+          sm_flags(p)[F_ABORT] = 1;
+          return false;
+        }
+        if (dev::globaltimer() - t0 > p.timeout_ns) {
+          raise_error(p, DEV_TIMEOUT, step, layer, stage, where);
+          sm_flags(p)[F_ABORT] = 1;
+          return false;
+        }
+      }
+      __nanosleep(p.poll_ns);
+#pragma unroll
+      for (int b = 0; b < NB; ++b)
+        if ((pend >> b) & 1u) v[b] = dev::ld_relaxed_v2_u64(src + 2 * k2[b]);
+    }
+  }
+
+  // Stores elements 2*k2 and 2*k2+1 of a K-vector into xs (times the gain
+  // when given); adds their squares to acc.
+  __device__ __forceinline__ void store_pair(int k2, float a, float b, int K, const __half* gain,
+                                             float& acc) {
+    acc = fmaf(a, a, acc);
+    acc = fmaf(b, b, acc);
+    if (gain) {
+      const float2 g = __half22float2(reinterpret_cast<const __half2*>(gain)[k2]);
+      a *= g.x;
+      b *= g.y;
+    }
+    *reinterpret_cast<float2*>(sm_xs(p) + perm(2 * k2, K)) = make_float2(a, b);
+  }
+
   // Loads a K-vector into xs (times `gain` if given) and returns in `ss` the
   // sum of squares of the raw values.  Source: tagged words, or an fp16
-  // embedding row.  Returns false (uniformly) on abort.
-  __device__ bool load_vec(const u64* src, unsigned tag, const __half* emb, int K,
+  // embedding row.  The polls of one thread are issued in batches of 16-byte
+  // loads so that their L2 round trips overlap.  Returns false (uniformly)
+  // on abort.
+  __device__ __noinline__ bool load_vec(const u64* src, unsigned tag, const __half* emb, int K,
                            const __half* gain, float& ss, int where) {
+    constexpr int NB = 4;
     const long long c0 = clock64();
     float acc = 0.f;
     bool bad = false;
-    for (int k = tid; k < K; k += kConsumerThreads) {
-      float v;
-      if (emb) {
-        v = __half2float(emb[k]);
-      } else if (!wait_f(src + k, tag, v, where)) {
-        bad = true;
-        break;
+    const int K2 = K >> 1;
+    if (emb) {
+      const __half2* e2 = reinterpret_cast<const __half2*>(emb);
+      for (int k2 = tid; k2 < K2; k2 += kConsumerThreads) {
+        const float2 v = __half22float2(e2[k2]);
+        store_pair(k2, v.x, v.y, K, gain, acc);
       }
-      acc = fmaf(v, v, acc);
-      S.xs[perm(k, K)] = gain ? v * __half2float(gain[k]) : v;
+    } else {
+      for (int base = tid; base < K2 && !bad; base += kConsumerThreads * NB) {
+        ulonglong2 v[NB];
+        int k2[NB];
+#pragma unroll
+        for (int b = 0; b < NB; ++b) k2[b] = base + b * kConsumerThreads;
+        if (!poll_pairs<NB>(src, k2, K2, tag, v, where)) {
+          bad = true;
+          break;
+        }
+#pragma unroll
+        for (int b = 0; b < NB; ++b)
+          if (k2[b] < K2)
+            store_pair(k2[b], __uint_as_float((unsigned)v[b].x), __uint_as_float((unsigned)v[b].y),
+                       K, gain, acc);
+      }
     }
     acc = dev::warp_sum(acc);
-    if (lane == 0) S.red[warp] = acc;
+    if (lane == 0) sm_red(p)[warp] = acc;
     bad = dev::consumer_sync_or(bad);
     float t = 0.f;
 #pragma unroll
-    for (int w = 0; w < kConsumerWarps; ++w) t += S.red[w];
+    for (int w = 0; w < kConsumerWarps; ++w) t += sm_red(p)[w];
     ss = t;
     if (tid == 0) t_sync += clock64() - c0;
+    trace_loaded();
     return !bad;
   }
 
+  // Polls n2 pairs of tagged words into dst[0 .. 2*n2) (times `scale`).
+  __device__ __noinline__ bool load_pairs(const u64* src, unsigned tag, int n2, float* dst,
+                                          float scale, int where) {
+    constexpr int NB = 4;
+    for (int base = tid; base < n2; base += kConsumerThreads * NB) {
+      ulonglong2 v[NB];
+      int k2[NB];
+#pragma unroll
+      for (int b = 0; b < NB; ++b) k2[b] = base + b * kConsumerThreads;
+      if (!poll_pairs<NB>(src, k2, n2, tag, v, where)) return false;
+#pragma unroll
+      for (int b = 0; b < NB; ++b)
+        if (k2[b] < n2) {
+          dst[2 * k2[b]] = __uint_as_float((unsigned)v[b].x) * scale;
+          dst[2 * k2[b] + 1] = __uint_as_float((unsigned)v[b].y) * scale;
+        }
+    }
+    return true;
+  }
+
   // ---- GEMV of this CTA's rows of a stage into rowacc (raw dot products).
-  __device__ bool gemv(int st, const LayerW& w, int ub, int ue) {
+  // A group of up to 16 rows streams as k-chunks.  In a full group warp w
+  // owns rows w and w+8 for all of the group's chunks (one activation load
+  // serves two rows) and keeps its partial sums in registers.  A group of
+  // at most 8 rows gives each row 8/rg (power of two) warps that split its
+  // pieces and are summed in a fixed order, so results do not depend on
+  // timing.
+  __device__ __forceinline__ static void dot_piece(const uint4& w, const float4& a,
+                                                   const float4& b, float2 (&c)[4]) {
+    c[0] = dev::ffma2(__half22float2(*reinterpret_cast<const __half2*>(&w.x)),
+                      make_float2(a.x, a.y), c[0]);
+    c[1] = dev::ffma2(__half22float2(*reinterpret_cast<const __half2*>(&w.y)),
+                      make_float2(a.z, a.w), c[1]);
+    c[2] = dev::ffma2(__half22float2(*reinterpret_cast<const __half2*>(&w.z)),
+                      make_float2(b.x, b.y), c[2]);
+    c[3] = dev::ffma2(__half22float2(*reinterpret_cast<const __half2*>(&w.w)),
+                      make_float2(b.z, b.w), c[3]);
+  }
+  __device__ __forceinline__ static float sum4(const float2 (&c)[4]) {
+    return ((c[0].x + c[0].y) + (c[1].x + c[1].y)) + ((c[2].x + c[2].y) + (c[3].x + c[3].y));
+  }
+
+  __device__ __noinline__ bool gemv(int st, int ub, int ue) {
     const int R = range_rows(p, st, ub, ue);
     const int K = stage_k(p, st);
     const int kp = K / kPieceElems;
-    const float4* xlo = reinterpret_cast<const float4*>(S.xs);
-    const float4* xhi = reinterpret_cast<const float4*>(S.xs + (K >> 1));
+    const unsigned char* ring = sm_ring(p);
+    const float4* xlo = reinterpret_cast<const float4*>(kie_smem + p.sm.xs_off) + lane;
+    const float4* xhi = xlo + (K >> 3);   // + K/2 floats
+    float* rowacc = sm_rowacc(p);
+    const Chunking chf = chunking(kGroupRows, kp, p.chunk_bytes);
     bool bad = false;
-    for (int g0 = 0; g0 < R; g0 += 8) {
-      const int rg = min(8, R - g0);
-      const Chunking ch = chunking(rg, kp, p.slot_bytes);
-      const int wpr = kConsumerWarps / rg;
-      const bool active = warp < rg * wpr;
-      const int r = warp / wpr, part = warp - (warp / wpr) * wpr;
-      float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-      for (int kc = 0; kc < ch.nk; ++kc) {
-        if (!bad && !wait_full()) bad = true;
-        if (active && !bad) {
-          const int p0 = ch.first(kc), n = ch.first(kc + 1) - p0;
-          const int pa = (part * n) / wpr, pb = ((part + 1) * n) / wpr;
-          const uint4* wrow = reinterpret_cast<const uint4*>(
-                                  S.ring + (size_t)slot * p.slot_bytes + (size_t)r * n * kPieceBytes) +
-                              lane;
-          const float4* xl = xlo + (size_t)p0 * 32 + lane;
-          const float4* xh = xhi + (size_t)p0 * 32 + lane;
+    for (int g0 = 0; g0 < R; g0 += kGroupRows) {
+      const int rg = min(kGroupRows, R - g0);
+      const Chunking ch = rg == kGroupRows ? chf : chunking(rg, kp, p.chunk_bytes);
+      if (rg > kConsumerWarps) {
+        // two rows per warp: w and w+8 (the second may be missing)
+        const bool two = warp + kConsumerWarps < rg;
+        float2 c0[4], c1[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) c0[i] = c1[i] = make_float2(0.f, 0.f);
+        for (int kc = 0; kc < ch.nk; ++kc) {
+          const int n = ch.count(kc), p0 = ch.first(kc);
+          uint32_t off;
+          if (!wait_chunk((uint32_t)(rg * n * kPieceBytes), off) && !bad) bad = true;
+          if (!bad) {
+            const uint4* w0 =
+                reinterpret_cast<const uint4*>(ring + off + (size_t)warp * n * kPieceBytes) + lane;
+            const uint4* w1 = w0 + (size_t)kConsumerWarps * n * 32;
+            const float4* xl = xlo + (size_t)p0 * 32;
+            const float4* xh = xhi + (size_t)p0 * 32;
+            if (two) {
+#pragma unroll 4
+              for (int q = 0; q < n; ++q) {
+                const float4 a = xl[q * 32], b = xh[q * 32];
+                const uint4 u0 = w0[q * 32], u1 = w1[q * 32];
+                dot_piece(u0, a, b, c0);
+                dot_piece(u1, a, b, c1);
+              }
+            } else {
 #pragma unroll 2
-          for (int q = pa; q < pb; ++q) {
-            const uint4 wv = wrow[q * 32];
-            const float4 xa = xl[q * 32];
-            const float4 xb = xh[q * 32];
-            const float2 f0 = __half22float2(*reinterpret_cast<const __half2*>(&wv.x));
-            const float2 f1 = __half22float2(*reinterpret_cast<const __half2*>(&wv.y));
-            const float2 f2 = __half22float2(*reinterpret_cast<const __half2*>(&wv.z));
-            const float2 f3 = __half22float2(*reinterpret_cast<const __half2*>(&wv.w));
-            a0 = fmaf(f0.x, xa.x, a0);
-            a1 = fmaf(f0.y, xa.y, a1);
-            a2 = fmaf(f1.x, xa.z, a2);
-            a3 = fmaf(f1.y, xa.w, a3);
-            a0 = fmaf(f2.x, xb.x, a0);
-            a1 = fmaf(f2.y, xb.y, a1);
-            a2 = fmaf(f3.x, xb.z, a2);
-            a3 = fmaf(f3.y, xb.w, a3);
+              for (int q = 0; q < n; ++q) dot_piece(w0[q * 32], xl[q * 32], xh[q * 32], c0);
+            }
+          }
+          release_chunk();
+        }
+        const float s0 = dev::warp_sum(sum4(c0));
+        const float s1 = dev::warp_sum(sum4(c1));
+        if (lane == 0) {
+          rowacc[g0 + warp] = s0;
+          if (two) rowacc[g0 + warp + kConsumerWarps] = s1;
+        }
+      } else {
+        const int lw = rg == 1 ? 3 : rg == 2 ? 2 : rg <= 4 ? 1 : 0;   // log2(warps per row)
+        const int r = warp >> lw, part = warp & ((1 << lw) - 1);
+        const bool active = r < rg;
+        float2 c0[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) c0[i] = make_float2(0.f, 0.f);
+        for (int kc = 0; kc < ch.nk; ++kc) {
+          const int n = ch.count(kc), p0 = ch.first(kc);
+          uint32_t off;
+          if (!wait_chunk((uint32_t)(rg * n * kPieceBytes), off) && !bad) bad = true;
+          if (active && !bad) {
+            const int pa = (part * n) >> lw, pb = ((part + 1) * n) >> lw;
+            const uint4* wr =
+                reinterpret_cast<const uint4*>(ring + off + (size_t)r * n * kPieceBytes) + lane;
+            const float4* xl = xlo + (size_t)p0 * 32;
+            const float4* xh = xhi + (size_t)p0 * 32;
+#pragma unroll 2
+            for (int q = pa; q < pb; ++q) dot_piece(wr[q * 32], xl[q * 32], xh[q * 32], c0);
+          }
+          release_chunk();
+        }
+        if (active) {
+          const float s = dev::warp_sum(sum4(c0));
+          if (lane == 0) {
+            if (lw == 0) rowacc[g0 + r] = s;
+            else sm_part(p)[warp] = s;
           }
         }
-        release_slot();
-      }
-      if (active) {
-        const float s = dev::warp_sum((a0 + a1) + (a2 + a3));
-        if (lane == 0) {
-          if (wpr == 1) S.rowacc[g0 + r] = s;
-          else S.part[warp] = s;
-        }
-      }
-      if (wpr > 1) {
-        dev::consumer_sync();
-        if (tid < rg) {
-          float s = 0.f;
-          for (int q = 0; q < wpr; ++q) s += S.part[tid * wpr + q];
-          S.rowacc[g0 + tid] = s;
+        if (lw > 0) {
+          dev::consumer_sync();
+          if (tid < rg) {
+            float s = 0.f;
+            for (int q = 0; q < (1 << lw); ++q) s += sm_part(p)[(tid << lw) + q];
+            rowacc[g0 + tid] = s;
+          }
         }
       }
     }
@@ -482,14 +751,14 @@ struct Consumer {
   // ---- stage bodies -------------------------------------------------------
 
   // RMSNorm + QKV GEMV + RoPE + KV append.
-  __device__ bool stage_qkv(const LayerW& w, int tok, int pos, unsigned tag) {
+  __device__ __noinline__ bool stage_qkv(const LayerW& w, int tok, int pos, unsigned tag) {
     stage = ST_QKV;
     const int2 r = p.ranges[ST_QKV * p.grid + blockIdx.x];
     float ss;
     const __half* emb = layer == 0 ? p.tok_emb + (size_t)tok * p.d : nullptr;
     if (r.y > r.x) {
       if (!load_vec(p.x_attn, tag, emb, p.d, w.attn_norm, ss, 10)) return false;
-      if (!gemv(ST_QKV, w, r.x, r.y)) return false;
+      if (!gemv(ST_QKV, r.x, r.y)) return false;
     } else {
       return true;
     }
@@ -504,7 +773,7 @@ struct Consumer {
     for (int u = r.x + tid; u < r.y; u += kConsumerThreads) {
       const int k = u - r.x;
       if (u < np_all) {
-        const float a = S.rowacc[2 * k] * rs, b = S.rowacc[2 * k + 1] * rs;
+        const float a = sm_rowacc(p)[2 * k] * rs, b = sm_rowacc(p)[2 * k + 1] * rs;
         const bool isq = u < nqp;
         const int uu = isq ? u : u - nqp;
         const int h = uu / half, i = uu - h * half;
@@ -525,7 +794,7 @@ struct Consumer {
       } else {
         const int vr = u - np_all;
         const int lr = 2 * np + (k - np);
-        const __half vh = __float2half_rn(S.rowacc[lr] * rs);
+        const __half vh = __float2half_rn(sm_rowacc(p)[lr] * rs);
         const int h = vr / p.hd, e = vr - h * p.hd;
         vbase[((size_t)h * p.max_seq + pos) * p.hd + e] = vh;
         put(p.kvnew + p.KV * p.hd + vr, tag, __half2float(vh), skip);
@@ -534,102 +803,150 @@ struct Consumer {
     return true;
   }
 
-  // Split-K attention over positions 0..pos, GQA group of one KV head per
-  // work item; the last item of a KV head combines the partials.
+  // Split-K attention over positions 0..pos for the G query heads of one
+  // KV head; the last item of a KV head combines the partials.  K and V
+  // blocks arrive through the ring (issued by the producer before q is
+  // ready); the current position's k and v come from the tagged words.
+  //   scores: P = 1, 2 or 4 threads per position split the HD/8 16-byte
+  //           chunks of the K row: part p of position t reads chunk
+  //           (p + P*(i + t)) mod HD/8 at step i, so the 8 lanes of a load
+  //           phase read chunks with 8 different residues mod 8 (8 bank
+  //           groups); q sits chunk-major with an odd multiple of 4 floats
+  //           per chunk row, so the same rotated reads of q are
+  //           conflict-free too;
+  //   P.V:    thread (head g, 4 dims) runs over the block's positions with
+  //           four independent accumulators.
   template <int HD>
-  __device__ bool stage_attn(int pos, unsigned tag) {
+  __device__ __noinline__ bool stage_attn(int pos, unsigned tag) {
     stage = 5;
-    const int n_pos = pos + 1;
-    int nsplit = (n_pos + p.min_split_len - 1) / p.min_split_len;
-    if (nsplit > p.max_split) nsplit = p.max_split;
-    const int items = p.KV * nsplit;
-    const int it = blockIdx.x;
-    if (it >= items) return true;
+    const AttnItem it = attn_item(p, pos);
+    if (!it.valid) return true;
+    constexpr int NCH = HD / 8;        // 16-byte K chunks per row
+    constexpr int DQ = HD / 4;         // dim quads per head
     const int G = p.G;
-    const int j = it / nsplit, s = it - (it / nsplit) * nsplit;
-    const int t0 = (int)(((long long)s * n_pos) / nsplit);
-    const int t1 = (int)(((long long)(s + 1) * n_pos) / nsplit);
-    constexpr int NGRP = kConsumerThreads / (HD / 2);
-    float* qs = S.xs;
-    float* sc = qs + G * HD;
+    const int QST = G * 8 + 4;         // floats per q chunk row (padded)
+    const int j = it.j;
+    float* qc = sm_xs(p);              // [NCH][QST]: q chunk c of head g at c*QST + g*8
+    float* sc = qc + NCH * QST;        // [G][kAttnBlock]
     float* kn = sc + G * kAttnBlock;
     float* vn = kn + HD;
-    float* red = vn + HD;
-    float* orun = red + NGRP * G * HD;
+    float* orun = vn + HD;
     float* mrun = orun + G * HD;
     float* lrun = mrun + kMaxGroup;
     float* alpha = lrun + kMaxGroup;
     const float scale = 1.0f / sqrtf((float)HD);
     const long long c0 = clock64();
+    // q (tagged), scaled, stored chunk-major
     bool bad = false;
-    for (int e = tid; e < G * HD && !bad; e += kConsumerThreads) {
-      float v;
-      if (!wait_f(p.qbuf + (size_t)j * G * HD + e, tag, v, 20)) bad = true;
-      qs[e] = v * scale;
-      orun[e] = 0.f;
-    }
-    if (t1 > pos) {
-      for (int e = tid; e < 2 * HD && !bad; e += kConsumerThreads) {
-        float v;
-        const u64* src = e < HD ? p.kvnew + j * HD + e : p.kvnew + p.KV * HD + j * HD + (e - HD);
-        if (!wait_f(src, tag, v, 21)) bad = true;
-        if (e < HD) kn[e] = v;
-        else vn[e - HD] = v;
+    {
+      const u64* src = p.qbuf + (size_t)j * G * HD;
+      const int n2 = G * HD / 2;
+      constexpr int NB = 4;
+      for (int base = tid; base < n2 && !bad; base += kConsumerThreads * NB) {
+        ulonglong2 v[NB];
+        int k2[NB];
+#pragma unroll
+        for (int b = 0; b < NB; ++b) k2[b] = base + b * kConsumerThreads;
+        if (!poll_pairs<NB>(src, k2, n2, tag, v, 20)) {
+          bad = true;
+          break;
+        }
+#pragma unroll
+        for (int b = 0; b < NB; ++b) {
+          if (k2[b] < n2) {
+            const int e = 2 * k2[b], g = e / HD, d = e - g * HD;
+            qc[(d >> 3) * QST + g * 8 + (d & 7)] = __uint_as_float((unsigned)v[b].x) * scale;
+            qc[(d >> 3) * QST + g * 8 + (d & 7) + 1] = __uint_as_float((unsigned)v[b].y) * scale;
+          }
+        }
       }
     }
+    if (it.t1 > pos && !bad) {
+      bad = !load_pairs(p.kvnew + j * HD, tag, HD / 2, kn, 1.0f, 21) ||
+            !load_pairs(p.kvnew + p.KV * HD + j * HD, tag, HD / 2, vn, 1.0f, 22);
+    }
+    for (int e = tid; e < G * HD; e += kConsumerThreads) orun[e] = 0.f;
     if (tid < kMaxGroup) {
       mrun[tid] = -INFINITY;
       lrun[tid] = 0.f;
     }
     if (dev::consumer_sync_or(bad)) return false;
     if (tid == 0) t_sync += clock64() - c0;
+    trace(10);
 
-    const __half* Kc = p.kv + (((size_t)layer * 2 + 0) * p.KV + j) * (size_t)p.max_seq * HD;
-    const __half* Vc = p.kv + (((size_t)layer * 2 + 1) * p.KV + j) * (size_t)p.max_seq * HD;
-    for (int b0 = t0; b0 < t1; b0 += kAttnBlock) {
-      const int nb = min(kAttnBlock, t1 - b0);
-      // scores of the block: one thread per position, all G heads
-      if (tid < nb) {
-        const int u = b0 + tid;
-        float sg[kMaxGroup];
+    const unsigned char* ring = sm_ring(p);
+    const int tb = attn_block(p);
+    const int g_pv = tid / DQ, dq = tid - (tid / DQ) * DQ;   // P.V thread role
+    for (int b0 = it.t0; b0 < it.t1; b0 += tb) {
+      const int nb = min(it.t1, b0 + tb) - b0;
+      const int nc = min(b0 + nb, pos) - b0;    // rows that came through the ring
+      uint32_t offk = 0, offv = 0;
+      bool badc = false;
+      if (nc > 0) {
+        const uint32_t sz = (uint32_t)(nc * HD * 2);
+        if (!wait_chunk(sz, offk)) badc = true;
+        if (!wait_chunk(sz, offv)) badc = true;
+      }
+      if (b0 == it.t0) trace(14);
+      if (!badc) {
+        // threads per position: 4, 2 or 1
+        const int lp = nb <= kConsumerThreads / 4 ? 2 : nb <= kConsumerThreads / 2 ? 1 : 0;
+        const int P = 1 << lp;
+        const int cper = NCH >> lp;                    // chunks per thread
+        const uint4* Krows = reinterpret_cast<const uint4*>(ring + offk);
+        for (int base = 0; base < nb * P; base += kConsumerThreads) {
+          const int e = base + tid;
+          const int t = e >> lp, part = e & (P - 1);
+          float sg[kMaxGroup];
 #pragma unroll
-        for (int g = 0; g < kMaxGroup; ++g) sg[g] = 0.f;
-        const uint4* krow = reinterpret_cast<const uint4*>(Kc + (size_t)u * HD);
-#pragma unroll 4
-        for (int c = 0; c < HD / 8; ++c) {
-          float kf[8];
-          if (u == pos) {
+          for (int g = 0; g < kMaxGroup; ++g) sg[g] = 0.f;
+          if (t < nb) {
+            const bool cur = t >= nc;
+            for (int i = 0; i < cper; ++i) {
+              const int c = (part + P * (i + t)) & (NCH - 1);
+              float kf[8];
+              if (!cur) {
+                const uint4 kv = Krows[(size_t)t * NCH + c];
+                const float2 a = __half22float2(*reinterpret_cast<const __half2*>(&kv.x));
+                const float2 b = __half22float2(*reinterpret_cast<const __half2*>(&kv.y));
+                const float2 cc = __half22float2(*reinterpret_cast<const __half2*>(&kv.z));
+                const float2 d = __half22float2(*reinterpret_cast<const __half2*>(&kv.w));
+                kf[0] = a.x; kf[1] = a.y; kf[2] = b.x; kf[3] = b.y;
+                kf[4] = cc.x; kf[5] = cc.y; kf[6] = d.x; kf[7] = d.y;
+              } else {
 #pragma unroll
-            for (int e = 0; e < 8; ++e) kf[e] = kn[c * 8 + e];
-          } else {
-            const uint4 kv = krow[c];
-            const float2 a = __half22float2(*reinterpret_cast<const __half2*>(&kv.x));
-            const float2 b = __half22float2(*reinterpret_cast<const __half2*>(&kv.y));
-            const float2 cc = __half22float2(*reinterpret_cast<const __half2*>(&kv.z));
-            const float2 d = __half22float2(*reinterpret_cast<const __half2*>(&kv.w));
-            kf[0] = a.x; kf[1] = a.y; kf[2] = b.x; kf[3] = b.y;
-            kf[4] = cc.x; kf[5] = cc.y; kf[6] = d.x; kf[7] = d.y;
+                for (int q = 0; q < 8; ++q) kf[q] = kn[c * 8 + q];
+              }
+              const float* qrow = qc + c * QST;
+#pragma unroll
+              for (int g = 0; g < kMaxGroup; ++g) {
+                if (g < G) {
+                  const float4 qa = *reinterpret_cast<const float4*>(qrow + g * 8);
+                  const float4 qb = *reinterpret_cast<const float4*>(qrow + g * 8 + 4);
+                  float s2 = sg[g];
+                  s2 = fmaf(qa.x, kf[0], s2); s2 = fmaf(qa.y, kf[1], s2);
+                  s2 = fmaf(qa.z, kf[2], s2); s2 = fmaf(qa.w, kf[3], s2);
+                  s2 = fmaf(qb.x, kf[4], s2); s2 = fmaf(qb.y, kf[5], s2);
+                  s2 = fmaf(qb.z, kf[6], s2); s2 = fmaf(qb.w, kf[7], s2);
+                  sg[g] = s2;
+                }
+              }
+            }
           }
+          // sum the P parts of a position (adjacent lanes)
 #pragma unroll
           for (int g = 0; g < kMaxGroup; ++g) {
             if (g < G) {
-              const float4 qa = *reinterpret_cast<const float4*>(qs + g * HD + c * 8);
-              const float4 qb = *reinterpret_cast<const float4*>(qs + g * HD + c * 8 + 4);
-              float t = sg[g];
-              t = fmaf(qa.x, kf[0], t); t = fmaf(qa.y, kf[1], t);
-              t = fmaf(qa.z, kf[2], t); t = fmaf(qa.w, kf[3], t);
-              t = fmaf(qb.x, kf[4], t); t = fmaf(qb.y, kf[5], t);
-              t = fmaf(qb.z, kf[6], t); t = fmaf(qb.w, kf[7], t);
-              sg[g] = t;
+              float v = sg[g];
+              if (lp >= 2) v += __shfl_xor_sync(0xffffffffu, v, 2);
+              if (lp >= 1) v += __shfl_xor_sync(0xffffffffu, v, 1);
+              if (t < nb && part == 0) sc[g * kAttnBlock + t] = v;
             }
           }
         }
-#pragma unroll
-        for (int g = 0; g < kMaxGroup; ++g)
-          if (g < G) sc[g * kAttnBlock + tid] = sg[g];
       }
-      dev::consumer_sync();
-      // online softmax: warp g owns head g
+      if (dev::consumer_sync_or(badc)) return false;
+      // online softmax over the block: warp g owns head g
       if (warp < G) {
         float* row = sc + warp * kAttnBlock;
         float mx = -INFINITY;
@@ -652,45 +969,61 @@ struct Consumer {
         }
       }
       dev::consumer_sync();
-      // P.V: thread (dim pair dp, position group tg)
-      {
-        const int dp = tid % (HD / 2), tg = tid / (HD / 2);
-        float2 acc[kMaxGroup];
+      if (b0 == it.t0) trace(15);
+      if (g_pv < G) {
+        const uint2* Vrows = reinterpret_cast<const uint2*>(ring + offv);
+        const float* pr = sc + g_pv * kAttnBlock;
+        float4 acc[4];
 #pragma unroll
-        for (int g = 0; g < kMaxGroup; ++g) acc[g] = make_float2(0.f, 0.f);
-        for (int t = tg; t < nb; t += NGRP) {
-          const int u = b0 + t;
-          float2 v;
-          if (u == pos) v = make_float2(vn[2 * dp], vn[2 * dp + 1]);
-          else v = __half22float2(reinterpret_cast<const __half2*>(Vc + (size_t)u * HD)[dp]);
+        for (int u = 0; u < 4; ++u) acc[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+        int t = 0;
+        for (; t + 4 <= nc; t += 4) {
 #pragma unroll
-          for (int g = 0; g < kMaxGroup; ++g) {
-            if (g < G) {
-              const float pr = sc[g * kAttnBlock + t];
-              acc[g].x = fmaf(pr, v.x, acc[g].x);
-              acc[g].y = fmaf(pr, v.y, acc[g].y);
-            }
+          for (int u = 0; u < 4; ++u) {
+            const uint2 raw = Vrows[(size_t)(t + u) * DQ + dq];
+            const float2 a = __half22float2(*reinterpret_cast<const __half2*>(&raw.x));
+            const float2 b = __half22float2(*reinterpret_cast<const __half2*>(&raw.y));
+            const float w = pr[t + u];
+            acc[u].x = fmaf(w, a.x, acc[u].x);
+            acc[u].y = fmaf(w, a.y, acc[u].y);
+            acc[u].z = fmaf(w, b.x, acc[u].z);
+            acc[u].w = fmaf(w, b.y, acc[u].w);
           }
         }
-#pragma unroll
-        for (int g = 0; g < kMaxGroup; ++g) {
-          if (g < G) {
-            red[(tg * G + g) * HD + 2 * dp] = acc[g].x;
-            red[(tg * G + g) * HD + 2 * dp + 1] = acc[g].y;
+        for (; t < nb; ++t) {
+          float4 v;
+          if (t < nc) {
+            const uint2 raw = Vrows[(size_t)t * DQ + dq];
+            const float2 a = __half22float2(*reinterpret_cast<const __half2*>(&raw.x));
+            const float2 b = __half22float2(*reinterpret_cast<const __half2*>(&raw.y));
+            v = make_float4(a.x, a.y, b.x, b.y);
+          } else {
+            v = *reinterpret_cast<const float4*>(vn + dq * 4);
           }
+          const float w = pr[t];
+          acc[0].x = fmaf(w, v.x, acc[0].x);
+          acc[0].y = fmaf(w, v.y, acc[0].y);
+          acc[0].z = fmaf(w, v.z, acc[0].z);
+          acc[0].w = fmaf(w, v.w, acc[0].w);
         }
+        float4* o = reinterpret_cast<float4*>(orun + g_pv * HD + dq * 4);
+        const float a = alpha[g_pv];
+        float4 cur = *o;
+        cur.x = fmaf(cur.x, a, (acc[0].x + acc[1].x) + (acc[2].x + acc[3].x));
+        cur.y = fmaf(cur.y, a, (acc[0].y + acc[1].y) + (acc[2].y + acc[3].y));
+        cur.z = fmaf(cur.z, a, (acc[0].z + acc[1].z) + (acc[2].z + acc[3].z));
+        cur.w = fmaf(cur.w, a, (acc[0].w + acc[1].w) + (acc[2].w + acc[3].w));
+        *o = cur;
       }
       dev::consumer_sync();
-      for (int e = tid; e < G * HD; e += kConsumerThreads) {
-        const int g = e / HD, dd = e - g * HD;
-        float sum = 0.f;
-        for (int q = 0; q < NGRP; ++q) sum += red[(q * G + g) * HD + dd];
-        orun[e] = orun[e] * alpha[g] + sum;
+      if (nc > 0) {
+        release_chunk();
+        release_chunk();
       }
-      dev::consumer_sync();
     }
+    trace(11);
     // publish this item's partial (m, l, unnormalised o)
-    float* part = p.partials + (size_t)it * G * (HD + 2);
+    float* part = p.partials + (size_t)blockIdx.x * G * (HD + 2);
     for (int e = tid; e < G * HD; e += kConsumerThreads) {
       const int g = e / HD, dd = e - g * HD;
       part[g * (HD + 2) + 2 + dd] = orun[e];
@@ -700,30 +1033,52 @@ struct Consumer {
       part[tid * (HD + 2) + 1] = lrun[tid];
     }
     dev::consumer_sync();
+    const int nsplit = it.nsplit;
     if (tid == 0) {
       dev::fence_acq_rel_gpu();
       const unsigned old = atomicAdd(p.att_ctr + layer * p.KV + j, 1u);
-      S.flags[F_LAST] = (old == (unsigned)(nsplit - 1)) ? 1 : 0;
+      sm_flags(p)[F_LAST] = (old == (unsigned)(nsplit - 1)) ? 1 : 0;
     }
     dev::consumer_sync();
-    if (S.flags[F_LAST]) {
+    trace(12);
+    if (sm_flags(p)[F_LAST]) {
       dev::fence_acq_rel_gpu();
+      // the last item of KV head j combines all nsplit partials:
+      // weights w_q = exp(m_q - M) / sum_q exp(m_q - M) l_q per head
       const float* base = p.partials + (size_t)(j * nsplit) * G * (HD + 2);
+      float* wq = sc;                                   // [nsplit][G]
+      float* mq = sc + kMaxSplitCombine * kMaxGroup;    // [nsplit][G] m, then l
+      for (int e = tid; e < nsplit * G; e += kConsumerThreads) {
+        const int q = e / G, g = e - (e / G) * G;
+        const float2 ml = *reinterpret_cast<const float2*>(base + ((size_t)q * G + g) * (HD + 2));
+        mq[2 * e] = ml.x;
+        mq[2 * e + 1] = ml.y;
+      }
+      dev::consumer_sync();
+      if (tid < G) {
+        float M = -INFINITY;
+        for (int q = 0; q < nsplit; ++q) M = fmaxf(M, mq[2 * (q * G + tid)]);
+        float Lsum = 0.f;
+        for (int q = 0; q < nsplit; ++q) {
+          const float f = expf(mq[2 * (q * G + tid)] - M);
+          wq[q * G + tid] = f;
+          Lsum = fmaf(f, mq[2 * (q * G + tid) + 1], Lsum);
+        }
+        const float inv = 1.0f / Lsum;
+        for (int q = 0; q < nsplit; ++q) wq[q * G + tid] *= inv;
+      }
+      dev::consumer_sync();
       const bool skip = fault_here(1);
       for (int e = tid; e < G * HD; e += kConsumerThreads) {
         const int g = e / HD, dd = e - g * HD;
-        float M = -INFINITY;
-        for (int q = 0; q < nsplit; ++q) M = fmaxf(M, base[((size_t)q * G + g) * (HD + 2)]);
-        float Lsum = 0.f, O = 0.f;
-        for (int q = 0; q < nsplit; ++q) {
-          const float* pq = base + ((size_t)q * G + g) * (HD + 2);
-          const float f = expf(pq[0] - M);
-          Lsum = fmaf(f, pq[1], Lsum);
-          O = fmaf(f, pq[2 + dd], O);
-        }
-        put(p.obuf + ((size_t)j * G + g) * HD + dd, tag, O / Lsum, skip);
+        float O = 0.f;
+#pragma unroll 4
+        for (int q = 0; q < nsplit; ++q)
+          O = fmaf(wq[q * G + g], base[((size_t)q * G + g) * (HD + 2) + 2 + dd], O);
+        put(p.obuf + ((size_t)j * G + g) * HD + dd, tag, O, skip);
       }
       if (tid == 0) p.att_ctr[layer * p.KV + j] = 0u;
+      trace(13);
     }
     return true;
   }
@@ -735,16 +1090,16 @@ struct Consumer {
     if (r.y <= r.x) return true;
     float ss;
     if (!load_vec(p.obuf, tag, nullptr, p.H * p.hd, nullptr, ss, 30)) return false;
-    if (!gemv(ST_O, w, r.x, r.y)) return false;
+    if (!gemv(ST_O, r.x, r.y)) return false;
     const bool skip = fault_here(ST_O);
-    bool bad = false;
     for (int u = r.x + tid; u < r.y; u += kConsumerThreads) {
-      float res;
-      if (layer == 0) res = __half2float(p.tok_emb[(size_t)tok * p.d + u]);
-      else if (!wait_f(p.x_attn + u, tag, res, 31)) { bad = true; break; }
-      put(p.x_ffn + u, tag, res + S.rowacc[u - r.x], skip);
+      const int k = u - r.x;
+      const float res = layer == 0 ? __half2float(p.tok_emb[(size_t)tok * p.d + u]) : sm_res_attn(p)[k];
+      const float v = res + sm_rowacc(p)[k];
+      sm_res_ffn(p)[k] = v;
+      put(p.x_ffn + u, tag, v, skip);
     }
-    return !dev::consumer_sync_or(bad);
+    return true;
   }
 
   // RMSNorm + gate/up GEMV + SwiGLU -> h.
@@ -754,12 +1109,12 @@ struct Consumer {
     if (r.y <= r.x) return true;
     float ss;
     if (!load_vec(p.x_ffn, tag, nullptr, p.d, w.ffn_norm, ss, 40)) return false;
-    if (!gemv(ST_GU, w, r.x, r.y)) return false;
+    if (!gemv(ST_GU, r.x, r.y)) return false;
     const float rs = 1.0f / sqrtf(ss / (float)p.d + p.eps);
     const bool skip = fault_here(ST_GU);
     for (int u = r.x + tid; u < r.y; u += kConsumerThreads) {
       const int k = u - r.x;
-      const float g = S.rowacc[2 * k] * rs, up = S.rowacc[2 * k + 1] * rs;
+      const float g = sm_rowacc(p)[2 * k] * rs, up = sm_rowacc(p)[2 * k + 1] * rs;
       const float sg = g / (1.0f + expf(-g));
       put(p.hbuf + u, tag, sg * up, skip);
     }
@@ -773,15 +1128,15 @@ struct Consumer {
     if (r.y <= r.x) return true;
     float ss;
     if (!load_vec(p.hbuf, tag, nullptr, p.F, nullptr, ss, 50)) return false;
-    if (!gemv(ST_DOWN, w, r.x, r.y)) return false;
+    if (!gemv(ST_DOWN, r.x, r.y)) return false;
     const bool skip = fault_here(ST_DOWN);
-    bool bad = false;
     for (int u = r.x + tid; u < r.y; u += kConsumerThreads) {
-      float res;
-      if (!wait_f(p.x_ffn + u, tag, res, 51)) { bad = true; break; }
-      put(p.x_attn + u, tag_next, res + S.rowacc[u - r.x], skip);
+      const int k = u - r.x;
+      const float v = sm_res_ffn(p)[k] + sm_rowacc(p)[k];
+      sm_res_attn(p)[k] = v;
+      put(p.x_attn + u, tag_next, v, skip);
     }
-    return !dev::consumer_sync_or(bad);
+    return true;
   }
 
   __device__ __forceinline__ static bool better(float v, int i, float bv, int bi) {
@@ -802,7 +1157,7 @@ struct Consumer {
   // Final RMSNorm + LM head + argmax; or, on steps that pick no id, only
   // the per-step fenced publish.  Returns false on abort; *tok_out gets the
   // greedy id (uniform across the grid).
-  __device__ bool stage_lm(bool pick, int step_row, unsigned tag, int* tok_out) {
+  __device__ __noinline__ bool stage_lm(bool pick, int step_row, unsigned tag, int* tok_out) {
     stage = ST_LM;
     float best = -INFINITY;
     int bi = INT_MAX;
@@ -810,13 +1165,14 @@ struct Consumer {
     if (pick && r.y > r.x) {
       float ss;
       if (!load_vec(p.x_attn, tag, nullptr, p.d, p.final_norm, ss, 60)) return false;
-      if (!gemv(ST_LM, p.layers[0], r.x, r.y)) return false;
+      if (!gemv(ST_LM, r.x, r.y)) return false;
+      trace(2);
       const float rs = 1.0f / sqrtf(ss / (float)p.d + p.eps);
       float* cap = (p.capture && step_row < p.capture_rows)
                        ? p.capture + (size_t)step_row * p.V
                        : nullptr;
       for (int u = r.x + tid; u < r.y; u += kConsumerThreads) {
-        const float v = S.rowacc[u - r.x] * rs;
+        const float v = sm_rowacc(p)[u - r.x] * rs;
         if (cap) cap[u] = v;
         if (better(v, u, best, bi)) {
           best = v;
@@ -826,18 +1182,18 @@ struct Consumer {
     }
     warp_argmax(best, bi);
     if (lane == 0) {
-      S.red[warp] = best;
-      S.redi[warp] = bi;
+      sm_red(p)[warp] = best;
+      sm_redi(p)[warp] = bi;
     }
     dev::consumer_sync();
     const bool skip = fault_here(ST_LM);
     if (tid == 0) {
-      float b = S.red[0];
-      int ib = S.redi[0];
+      float b = sm_red(p)[0];
+      int ib = sm_redi(p)[0];
       for (int w = 1; w < kConsumerWarps; ++w)
-        if (better(S.red[w], S.redi[w], b, ib)) {
-          b = S.red[w];
-          ib = S.redi[w];
+        if (better(sm_red(p)[w], sm_redi(p)[w], b, ib)) {
+          b = sm_red(p)[w];
+          ib = sm_redi(p)[w];
         }
       // release: every plain store this CTA made in this step (KV cache,
       // logits) happens-before any CTA that reads these slots.
@@ -854,11 +1210,13 @@ struct Consumer {
     float gb = -INFINITY;
     int gi = INT_MAX;
     for (int c = tid; c < p.grid; c += kConsumerThreads) {
-      unsigned vb, ib;
-      if (!wait_tag(p.slots + 2 * c, tag, vb, 61) || !wait_tag(p.slots + 2 * c + 1, tag, ib, 62)) {
+      ulonglong2 w2[1];
+      const int k2[1] = {c};
+      if (!poll_pairs<1>(p.slots, k2, p.grid, tag, w2, 61)) {
         bad = true;
         break;
       }
+      const unsigned vb = (unsigned)w2[0].x, ib = (unsigned)w2[0].y;
       if (better(__uint_as_float(vb), (int)ib, gb, gi)) {
         gb = __uint_as_float(vb);
         gi = (int)ib;
@@ -868,20 +1226,65 @@ struct Consumer {
     dev::fence_acq_rel_gpu();
     warp_argmax(gb, gi);
     if (lane == 0) {
-      S.red2[warp] = gb;
-      S.redi2[warp] = gi;
+      sm_red2(p)[warp] = gb;
+      sm_redi2(p)[warp] = gi;
     }
     if (dev::consumer_sync_or(bad)) return false;
-    float b = S.red2[0];
-    int ib = S.redi2[0];
+    float b = sm_red2(p)[0];
+    int ib = sm_redi2(p)[0];
     for (int w = 1; w < kConsumerWarps; ++w)
-      if (better(S.red2[w], S.redi2[w], b, ib)) {
-        b = S.red2[w];
-        ib = S.redi2[w];
+      if (better(sm_red2(p)[w], sm_redi2(p)[w], b, ib)) {
+        b = sm_red2(p)[w];
+        ib = sm_redi2(p)[w];
       }
     *tok_out = ib;
-    if (tid == 0) t_sync += clock64() - c0;
+    if (tid == 0) {
+      t_sync += clock64() - c0;
+      // this step's KV writes of every CTA are now visible to this CTA:
+      // the producer may copy them for the next step
+      dev::st_release_cta(sm_flags(p) + F_KVSTEP, step + 1);
+    }
     return true;
+  }
+
+  // Walks a stage's chunk sequence without computing (stream-only timing).
+  __device__ __noinline__ bool skip_stage(int st, int ub, int ue) {
+    const int R = range_rows(p, st, ub, ue);
+    const int kp = stage_k(p, st) / kPieceElems;
+    bool bad = false;
+    for (int g0 = 0; g0 < R; g0 += kGroupRows) {
+      const int rg = min(kGroupRows, R - g0);
+      const Chunking ch = chunking(rg, kp, p.chunk_bytes);
+      for (int kc = 0; kc < ch.nk; ++kc) {
+        uint32_t off;
+        if (!wait_chunk((uint32_t)(rg * ch.count(kc) * kPieceBytes), off)) bad = true;
+        release_chunk();
+      }
+    }
+    return !dev::consumer_sync_or(bad);
+  }
+
+  // Standalone GEMV engine run: y = W x over the LM-head stage's rows,
+  // `iters` times (mode 0: stream the weights only, mode 1: full GEMV).
+  __device__ void gemv_bench(int mode, const float* x, float* y, int iters) {
+    const int2 r = p.ranges[ST_LM * p.grid + blockIdx.x];
+    const int K = p.d;
+    float acc = 0.f;
+    for (int k2 = tid; k2 < K / 2; k2 += kConsumerThreads) {
+      const float2 v = reinterpret_cast<const float2*>(x)[k2];
+      store_pair(k2, v.x, v.y, K, nullptr, acc);
+    }
+    dev::consumer_sync();
+    bool ok = true;
+    for (int it = 0; it < iters && ok; ++it)
+      ok = mode == 0 ? skip_stage(ST_LM, r.x, r.y) : gemv(ST_LM, r.x, r.y);
+    if (ok && mode == 1)
+      for (int u = r.x + tid; u < r.y; u += kConsumerThreads) y[u] = sm_rowacc(p)[u - r.x];
+    if (tid == 0) {
+      sm_flags(p)[F_STOP] = 1;
+      u64* st = p.cta_stats + kStatsPerCta * blockIdx.x;
+      st[2] = (u64)t_stream;
+    }
   }
 
   template <int HD>
@@ -897,14 +1300,26 @@ struct Consumer {
         layer = l;
         const LayerW& w = p.layers[l];
         const unsigned tag = epoch_of(p, i, l);
-        ok = stage_qkv(w, tok, pos, tag) && stage_attn<HD>(pos, tag) && stage_o(w, tok, tag) &&
-             stage_gu(w, tag) && stage_down(w, tag, tag + 1u);
+        trace(0);
+        ok = stage_qkv(w, tok, pos, tag);
+        trace(2);
+        ok = ok && stage_attn<HD>(pos, tag);
+        trace(3);
+        ok = ok && stage_o(w, tok, tag);
+        trace(5);
+        ok = ok && stage_gu(w, tag);
+        trace(7);
+        ok = ok && stage_down(w, tag, tag + 1u);
+        trace(9);
       }
       if (!ok) break;
       layer = p.L;
       const bool pick = i >= p.lm_from;
       int next = 0;
-      if (!stage_lm(pick, i - p.lm_from, epoch_of(p, i, p.L), &next)) {
+      trace(0);
+      const bool lm_ok = stage_lm(pick, i - p.lm_from, epoch_of(p, i, p.L), &next);
+      trace(3);
+      if (!lm_ok) {
         ok = false;
         break;
       }
@@ -914,14 +1329,14 @@ struct Consumer {
       if (p.forced && i + 1 < p.n_steps) tok = p.forced[i + 1];
       else tok = next;
     }
-    if (tid == 0) S.flags[F_STOP] = 1;
+    if (tid == 0) sm_flags(p)[F_STOP] = 1;
     if (blockIdx.x == 0 && tid == 0) p.status->n_done = done;
     if (tid == 0) {
-      u64* st = p.cta_stats + 4 * blockIdx.x;
+      u64* st = p.cta_stats + kStatsPerCta * blockIdx.x;
       st[0] = (u64)(clock64() - c_begin);
       st[1] = (u64)t_sync;
       st[2] = (u64)t_stream;
-      st[3] = (u64)done;
+      st[4] = (u64)done;
     }
   }
 };
@@ -930,28 +1345,88 @@ struct Consumer {
 
 template <int HD>
 __global__ void __launch_bounds__(kThreads, 1) kie_monokernel(const __grid_constant__ MonoParams p) {
-  extern __shared__ __align__(128) unsigned char smem[];
-  const Smem S = carve(p, smem);
   if (threadIdx.x == 0) {
-    for (int s = 0; s < p.ring_slots; ++s) {
-      dev::mbar_init(S.full_s + 8 * s, 1);
-      dev::mbar_init(S.empty_s + 8 * s, kConsumerWarps);
+    for (int s = 0; s < kRingBars; ++s) {
+      dev::mbar_init(sm_full_s(p) + 8 * s, 1);
+      dev::mbar_init(sm_empty_s(p) + 8 * s, kConsumerWarps);
     }
-    S.flags[F_ABORT] = 0;
-    S.flags[F_STOP] = 0;
-    S.flags[F_LAST] = 0;
+    sm_flags(p)[F_ABORT] = 0;
+    sm_flags(p)[F_STOP] = 0;
+    sm_flags(p)[F_LAST] = 0;
+    sm_flags(p)[F_KVSTEP] = 0;
     dev::mbar_fence_init();
   }
   __syncthreads();
   if (threadIdx.x >= kConsumerThreads) {
     if (threadIdx.x == kConsumerThreads) {
-      Producer prod(p, S);
+      Producer prod(p);
       prod.run();
     }
     return;
   }
-  Consumer c(p, S);
+  Consumer c(p);
   c.run<HD>();
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    kie_gemv_kernel(const __grid_constant__ MonoParams p, int mode, const float* x, float* y,
+                    int iters) {
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kRingBars; ++s) {
+      dev::mbar_init(sm_full_s(p) + 8 * s, 1);
+      dev::mbar_init(sm_empty_s(p) + 8 * s, kConsumerWarps);
+    }
+    sm_flags(p)[F_ABORT] = 0;
+    sm_flags(p)[F_STOP] = 0;
+    sm_flags(p)[F_LAST] = 0;
+    sm_flags(p)[F_KVSTEP] = 0;
+    dev::mbar_fence_init();
+  }
+  __syncthreads();
+  if (threadIdx.x >= kConsumerThreads) {
+    if (threadIdx.x == kConsumerThreads) {
+      Producer prod(p);
+      bool ok = true;
+      for (int it = 0; it < iters && ok; ++it) {
+        const unsigned char* src = p.packed + p.packed_off[blockIdx.x];
+        ok = prod.stage(ST_LM, src);
+      }
+      prod.drain();
+      p.cta_stats[kStatsPerCta * blockIdx.x + 3] = (unsigned long long)prod.t_wait;
+    }
+    return;
+  }
+  Consumer c(p);
+  c.gemv_bench(mode, x, y, iters);
+}
+
+__global__ void __launch_bounds__(256) kie_repack_kernel(const __grid_constant__ MonoParams p,
+                                                         unsigned char* packed) {
+  unsigned char* dst = packed + p.packed_off[blockIdx.x];
+  for (int l = 0; l < p.L; ++l) {
+    const LayerW& w = p.layers[l];
+    repack_stage(p, ST_QKV, w, dst);
+    repack_stage(p, ST_O, w, dst);
+    repack_stage(p, ST_GU, w, dst);
+    repack_stage(p, ST_DOWN, w, dst);
+  }
+  repack_stage(p, ST_LM, p.layers[0], dst);
+}
+
+cudaError_t repack_launch(const MonoParams& p, unsigned char* packed, cudaStream_t s) {
+  kie_repack_kernel<<<p.grid, 256, 0, s>>>(p, packed);
+  return cudaGetLastError();
+}
+
+cudaError_t gemv_configure(int smem_bytes) {
+  return cudaFuncSetAttribute((const void*)kie_gemv_kernel,
+                              cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes);
+}
+
+cudaError_t gemv_launch(const MonoParams& p, int mode, const float* x, float* y, int iters,
+                        int grid, int smem_bytes, cudaStream_t s) {
+  kie_gemv_kernel<<<grid, kThreads, smem_bytes, s>>>(p, mode, x, y, iters);
+  return cudaGetLastError();
 }
 
 cudaError_t mono_configure(int hd, int smem_bytes, int* blocks_per_sm) {

@@ -14,4 +14,14 @@ cudaError_t mono_configure(int hd, int smem_bytes, int* blocks_per_sm);
 // Cooperative launch (all CTAs co-resident) of `grid` persistent CTAs.
 cudaError_t mono_launch(const MonoParams& p, int hd, int grid, int smem_bytes, cudaStream_t s);
 
+// Copies the weight matrices into `packed`, each CTA's one-token stream at
+// p.packed_off[cta], in the order the decode kernel streams them.
+cudaError_t repack_launch(const MonoParams& p, unsigned char* packed, cudaStream_t s);
+
+// Standalone weight-stream GEMV (the LM-head stage over an arbitrary
+// matrix): y = W x, `iters` times; mode 0 streams without computing.
+cudaError_t gemv_configure(int smem_bytes);
+cudaError_t gemv_launch(const MonoParams& p, int mode, const float* x, float* y, int iters,
+                        int grid, int smem_bytes, cudaStream_t s);
+
 }  // namespace kie

@@ -14,11 +14,19 @@ enum Stage : int { ST_QKV = 0, ST_O = 1, ST_GU = 2, ST_DOWN = 3, ST_LM = 4, N_ST
 constexpr int kConsumerWarps = 8;            // warps that compute
 constexpr int kThreads = (kConsumerWarps + 1) * 32;  // + one producer warp
 constexpr int kConsumerThreads = kConsumerWarps * 32;
+constexpr int kGroupRows = 16;              // rows streamed together (two per warp)
 constexpr int kPieceElems = 256;             // one warp pass: 32 lanes x 8 fp16
 constexpr int kPieceBytes = kPieceElems * 2;
-constexpr int kMaxSlots = 16;
+constexpr int kRingBars = 16;                // mbarrier pairs of the byte ring (power of 2)
 constexpr int kMaxGroup = 8;                 // heads per KV head handled by one CTA
 constexpr int kAttnBlock = 256;              // positions per attention block
+constexpr int kMaxSplitCombine = 96;
+constexpr int kPollBackoffNs = 128;          // sleep between re-polls of tagged words         // attention splits one combine handles
+// per-CTA counters: loop cycles, sync-wait cycles, stream-wait cycles,
+// producer slot-wait cycles, steps done, spare
+constexpr int kStatsPerCta = 8;
+// stage-trace stamps per layer (the LM head adds 4 per step)
+constexpr int kTracePerLayer = 16;
 
 // Device status word block (library scratch, zeroed before each launch).
 struct DevStatus {
@@ -36,7 +44,7 @@ struct LayerW {
 // Shared-memory carve-up of one CTA (byte offsets from the dynamic base).
 struct SmemLayout {
   int ring_off, bar_off, xs_off, rowacc_off, misc_off, total;
-  int xs_bytes, rowacc_rows;
+  int xs_bytes, rowacc_rows, resid_rows;
 };
 
 struct MonoParams {
@@ -54,7 +62,9 @@ struct MonoParams {
   // plan
   const int2* ranges;      // [N_STAGES][grid] unit range per CTA
   int grid;
-  int ring_slots, slot_bytes;
+  int ring_bytes, chunk_bytes;   // byte ring size; largest chunk (one bulk copy)
+  const unsigned char* packed;   // library copy of the weight matrices in stream order
+  const unsigned long long* packed_off;  // [grid] byte offset of each CTA's stream
   int max_split, min_split_len;
   SmemLayout sm;
   // scratch (tagged 64-bit words: high 32 bits = epoch tag, low = fp32 bits)
@@ -70,8 +80,12 @@ struct MonoParams {
   int capture_rows;
   int* out_ids;
   DevStatus* status;
-  unsigned long long* cta_stats;  // [grid][4]: loop, sync wait, stream wait, spare
+  unsigned long long* cta_stats;  // [grid][kStatsPerCta]
   long long timeout_ns;
+  unsigned poll_ns;        // sleep between re-polls of tagged words
+  unsigned long long* trace;  // stage timestamps of CTA trace_cta, or null
+  int trace_cta, trace_steps;
+  int trace_clock;         // 1: stamps are SM cycles (clock64), 0: %globaltimer ns
   int fault_cta, fault_step, fault_layer, fault_stage;
 };
 

@@ -68,7 +68,10 @@ std::vector<int2> partition(const Shape& s, int grid, int stage) {
     bound[v] = unit_at_rows(s, stage, target);
   }
   bound[grid] = stage_units(s, stage);
-  const int rot = (stage * 41) % grid;
+  // O and down share one partition: the CTA that owns residual row r in the
+  // O stage owns it in the down stage too, so the residual stream of its
+  // rows never leaves the CTA.
+  const int rot = ((stage == ST_DOWN ? ST_O : stage) * 41) % grid;
   std::vector<int2> r(grid);
   for (int c = 0; c < grid; ++c) {
     const int v = (c + rot) % grid;
@@ -78,22 +81,19 @@ std::vector<int2> partition(const Shape& s, int grid, int stage) {
 }
 
 int attn_smem_bytes(int G, int hd) {
-  const int ngrp = kConsumerThreads / (hd / 2);
   int b = 0;
-  b += G * hd * 4;              // q (scaled)
-  b += G * kAttnBlock * 4;      // scores / probabilities of one block
-  b += 2 * hd * 4;              // current position's k and v
-  b += ngrp * G * hd * 4;       // V-phase partial sums per position group
-  b += G * hd * 4;              // running output
-  b += 4 * kMaxGroup * 4;       // running max, sum, rescale, spare
+  b += (hd / 8) * (G * 8 + 4) * 4;   // q, chunk-major with padded rows
+  b += std::max(G * kAttnBlock, 3 * kMaxSplitCombine * kMaxGroup) * 4;  // scores / combine
+  b += 2 * hd * 4;                   // current position's k and v
+  b += G * hd * 4;                   // running output
+  b += 4 * kMaxGroup * 4;            // running max, sum, rescale, spare
   return b;
 }
 
 static int align_up(int x, int a) { return (x + a - 1) / a * a; }
 
-bool plan_smem(const Shape& s, int grid, int slot_bytes, int smem_limit,
-               const std::vector<std::vector<int2>>& ranges, SmemLayout* out,
-               int* ring_slots) {
+bool plan_smem(const Shape& s, int grid, int chunk_bytes, int smem_limit,
+               const std::vector<std::vector<int2>>& ranges, SmemLayout* out, int* ring_bytes) {
   const int G = s.H / s.KV;
   const int kmax = std::max(std::max(s.d, s.H * s.hd), s.F);
   SmemLayout L{};
@@ -103,22 +103,33 @@ bool plan_smem(const Shape& s, int grid, int slot_bytes, int smem_limit,
     for (int c = 0; c < grid; ++c)
       maxrows = std::max(maxrows, rows_in_range(s, st, ranges[st][c].x, ranges[st][c].y));
   L.rowacc_rows = maxrows;
-  const int bars = 2 * kMaxSlots * 8;
-  const int misc = 1024;
+  int maxres = 0;
+  for (int c = 0; c < grid; ++c)
+    maxres = std::max(maxres, rows_in_range(s, ST_O, ranges[ST_O][c].x, ranges[ST_O][c].y));
+  L.resid_rows = maxres;
+  const int bars = 2 * kRingBars * 8;
+  const int misc = align_up(64 * 4 + 2 * maxres * 4, 128);
   const int fixed = align_up(bars, 128) + L.xs_bytes + align_up(maxrows * 4, 128) + misc;
-  const int avail = smem_limit - fixed;
-  int slots = avail / slot_bytes;
-  if (slots > kMaxSlots) slots = kMaxSlots;
-  if (slots < 2) return false;
+  const int ring = (smem_limit - fixed) / 512 * 512;
+  if (ring < 2 * chunk_bytes) return false;
   L.ring_off = 0;
-  L.bar_off = slots * slot_bytes;
+  L.bar_off = ring;
   L.xs_off = L.bar_off + align_up(bars, 128);
   L.rowacc_off = L.xs_off + L.xs_bytes;
   L.misc_off = L.rowacc_off + align_up(maxrows * 4, 128);
   L.total = L.misc_off + misc;
   *out = L;
-  *ring_slots = slots;
+  *ring_bytes = ring;
   return L.total <= smem_limit;
+}
+
+size_t stream_bytes(const Shape& s, const std::vector<std::vector<int2>>& ranges, int cta) {
+  size_t layer = 0;
+  for (int st = ST_QKV; st <= ST_DOWN; ++st)
+    layer += (size_t)rows_in_range(s, st, ranges[st][cta].x, ranges[st][cta].y) * stage_k(s, st) * 2;
+  const size_t lm =
+      (size_t)rows_in_range(s, ST_LM, ranges[ST_LM][cta].x, ranges[ST_LM][cta].y) * s.d * 2;
+  return (size_t)s.L * layer + lm;
 }
 
 }  // namespace kie

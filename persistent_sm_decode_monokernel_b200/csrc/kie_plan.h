@@ -32,9 +32,13 @@ std::vector<int2> partition(const Shape& s, int grid, int stage);
 // Attention shared-memory bytes for group size G and head_dim hd.
 int attn_smem_bytes(int G, int hd);
 
-// Shared memory carve-up; returns false if it does not fit `smem_limit`.
-bool plan_smem(const Shape& s, int grid, int slot_bytes, int smem_limit,
-               const std::vector<std::vector<int2>>& ranges, SmemLayout* out,
-               int* ring_slots);
+// Shared memory carve-up: fixed regions first, the rest (rounded down to
+// 512 B) is the weight ring.  Returns false if the ring would be smaller
+// than two chunks of `chunk_bytes`.
+bool plan_smem(const Shape& s, int grid, int chunk_bytes, int smem_limit,
+               const std::vector<std::vector<int2>>& ranges, SmemLayout* out, int* ring_bytes);
+
+// Bytes of CTA `cta`'s one-token weight stream (all layers + LM head).
+size_t stream_bytes(const Shape& s, const std::vector<std::vector<int2>>& ranges, int cta);
 
 }  // namespace kie

@@ -107,9 +107,12 @@ def test_partition_covers_and_balances(lib, name):
                              2: 2 * s.ffn_dim, 3: s.d_model, 4: s.vocab}[st]
         unit_rows = 2 if st in (0, 2) else 1
         assert max(rows) - min(rows) <= 2 * unit_rows - 1 + (st == 0), (st, max(rows), min(rows))
-    # the CTAs that carry an extra unit differ between stages
+    # O and down share one partition (each CTA keeps its residual rows)
+    for c in range(grid):
+        assert _kie.kie_plan_units(d, grid, 1, c) == _kie.kie_plan_units(d, grid, 3, c)
+    # elsewhere the CTAs that carry an extra unit differ between stages
     big = []
-    for st in (1, 3):
+    for st in (1, 4):
         rows = [_rows(s, st, *_kie.kie_plan_units(d, grid, st, c)) for c in range(grid)]
         big.append({c for c in range(grid) if rows[c] == max(rows)})
     assert big[0] != big[1] or len(big[0]) == grid
