@@ -151,6 +151,19 @@ __device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
   return *reinterpret_cast<float2*>(&d);
 }
 
+// a0 += w.lo * x.lo, a1 += w.hi * x.hi: fp16 x fp16 products accumulated in
+// fp32 (sm_100 mixed-precision FMA), one instruction per element and no
+// separate conversion.
+__device__ __forceinline__ void fma_f16x2_f32(float& a0, float& a1, uint32_t w, uint32_t x) {
+  asm("{\n\t.reg .f16 wl, wh, xl, xh;\n\t"
+      "mov.b32 {wl, wh}, %2;\n\t"
+      "mov.b32 {xl, xh}, %3;\n\t"
+      "fma.rn.f32.f16 %0, wl, xl, %0;\n\t"
+      "fma.rn.f32.f16 %1, wh, xh, %1;\n\t}"
+      : "+f"(a0), "+f"(a1)
+      : "r"(w), "r"(x));
+}
+
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);

@@ -488,14 +488,6 @@ struct Consumer {
     ++crel;
   }
 
-  // ---- permuted activation layout: element k of a K-vector sits where
-  // lane (k%256)/8 of piece k/256 reads it with two conflict-free 16-byte
-  // loads (elements 0-3 of the lane's 8 in the low half, 4-7 in the high).
-  __device__ __forceinline__ int perm(int k, int K) const {
-    const int piece = k >> 8, w = k & 255, ln = w >> 3, e = w & 7;
-    return (e < 4 ? 0 : (K >> 1)) + ((piece * 32 + ln) << 2) + (e & 3);
-  }
-
   // Polls NB pairs of tagged words (pair b at src + 2*k2[b], used when
   // k2[b] < n2) until every word carries `tag`.  All pending pairs are
   // re-read together, so a round costs one L2 round trip; rounds after the
@@ -549,9 +541,15 @@ struct Consumer {
     }
   }
 
-  // Stores elements 2*k2 and 2*k2+1 of a K-vector into xs (times the gain
-  // when given); adds their squares to acc.
-  __device__ __forceinline__ void store_pair(int k2, float a, float b, int K, const __half* gain,
+  // ---- GEMV input vector in shared memory: fp16, natural order (lane l of
+  // piece q reads elements 256q + 8l .. +8 with one 16-byte load).
+  __device__ __forceinline__ __half2* xs16() const {
+    return reinterpret_cast<__half2*>(kie_smem + p.sm.xs_off);
+  }
+
+  // Stores elements 2*k2 and 2*k2+1 of a K-vector into xs as fp16 (times
+  // the gain when given); adds the squares of the raw values to acc.
+  __device__ __forceinline__ void store_pair(int k2, float a, float b, const __half* gain,
                                              float& acc) {
     acc = fmaf(a, a, acc);
     acc = fmaf(b, b, acc);
@@ -560,7 +558,7 @@ struct Consumer {
       a *= g.x;
       b *= g.y;
     }
-    *reinterpret_cast<float2*>(sm_xs(p) + perm(2 * k2, K)) = make_float2(a, b);
+    xs16()[k2] = __floats2half2_rn(a, b);
   }
 
   // Loads a K-vector into xs (times `gain` if given) and returns in `ss` the
@@ -579,7 +577,7 @@ struct Consumer {
       const __half2* e2 = reinterpret_cast<const __half2*>(emb);
       for (int k2 = tid; k2 < K2; k2 += kConsumerThreads) {
         const float2 v = __half22float2(e2[k2]);
-        store_pair(k2, v.x, v.y, K, gain, acc);
+        store_pair(k2, v.x, v.y, gain, acc);
       }
     } else {
       for (int base = tid; base < K2 && !bad; base += kConsumerThreads * NB) {
@@ -595,7 +593,7 @@ struct Consumer {
         for (int b = 0; b < NB; ++b)
           if (k2[b] < K2)
             store_pair(k2[b], __uint_as_float((unsigned)v[b].x), __uint_as_float((unsigned)v[b].y),
-                       K, gain, acc);
+                       gain, acc);
       }
     }
     acc = dev::warp_sum(acc);
@@ -637,19 +635,14 @@ struct Consumer {
   // at most 8 rows gives each row 8/rg (power of two) warps that split its
   // pieces and are summed in a fixed order, so results do not depend on
   // timing.
-  __device__ __forceinline__ static void dot_piece(const uint4& w, const float4& a,
-                                                   const float4& b, float2 (&c)[4]) {
-    c[0] = dev::ffma2(__half22float2(*reinterpret_cast<const __half2*>(&w.x)),
-                      make_float2(a.x, a.y), c[0]);
-    c[1] = dev::ffma2(__half22float2(*reinterpret_cast<const __half2*>(&w.y)),
-                      make_float2(a.z, a.w), c[1]);
-    c[2] = dev::ffma2(__half22float2(*reinterpret_cast<const __half2*>(&w.z)),
-                      make_float2(b.x, b.y), c[2]);
-    c[3] = dev::ffma2(__half22float2(*reinterpret_cast<const __half2*>(&w.w)),
-                      make_float2(b.z, b.w), c[3]);
+  __device__ __forceinline__ static void dot_piece(const uint4& w, const uint4& x, float (&c)[8]) {
+    dev::fma_f16x2_f32(c[0], c[1], w.x, x.x);
+    dev::fma_f16x2_f32(c[2], c[3], w.y, x.y);
+    dev::fma_f16x2_f32(c[4], c[5], w.z, x.z);
+    dev::fma_f16x2_f32(c[6], c[7], w.w, x.w);
   }
-  __device__ __forceinline__ static float sum4(const float2 (&c)[4]) {
-    return ((c[0].x + c[0].y) + (c[1].x + c[1].y)) + ((c[2].x + c[2].y) + (c[3].x + c[3].y));
+  __device__ __forceinline__ static float sum8(const float (&c)[8]) {
+    return ((c[0] + c[1]) + (c[2] + c[3])) + ((c[4] + c[5]) + (c[6] + c[7]));
   }
 
   __device__ __noinline__ bool gemv(int st, int ub, int ue) {
@@ -657,8 +650,7 @@ struct Consumer {
     const int K = stage_k(p, st);
     const int kp = K / kPieceElems;
     const unsigned char* ring = sm_ring(p);
-    const float4* xlo = reinterpret_cast<const float4*>(kie_smem + p.sm.xs_off) + lane;
-    const float4* xhi = xlo + (K >> 3);   // + K/2 floats
+    const uint4* xv = reinterpret_cast<const uint4*>(kie_smem + p.sm.xs_off) + lane;
     float* rowacc = sm_rowacc(p);
     const Chunking chf = chunking(kGroupRows, kp, p.chunk_bytes);
     bool bad = false;
@@ -668,9 +660,9 @@ struct Consumer {
       if (rg > kConsumerWarps) {
         // two rows per warp: w and w+8 (the second may be missing)
         const bool two = warp + kConsumerWarps < rg;
-        float2 c0[4], c1[4];
+        float c0[8], c1[8];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) c0[i] = c1[i] = make_float2(0.f, 0.f);
+        for (int i = 0; i < 8; ++i) c0[i] = c1[i] = 0.f;
         for (int kc = 0; kc < ch.nk; ++kc) {
           const int n = ch.count(kc), p0 = ch.first(kc);
           uint32_t off;
@@ -679,25 +671,23 @@ struct Consumer {
             const uint4* w0 =
                 reinterpret_cast<const uint4*>(ring + off + (size_t)warp * n * kPieceBytes) + lane;
             const uint4* w1 = w0 + (size_t)kConsumerWarps * n * 32;
-            const float4* xl = xlo + (size_t)p0 * 32;
-            const float4* xh = xhi + (size_t)p0 * 32;
+            const uint4* x = xv + (size_t)p0 * 32;
             if (two) {
 #pragma unroll 4
               for (int q = 0; q < n; ++q) {
-                const float4 a = xl[q * 32], b = xh[q * 32];
-                const uint4 u0 = w0[q * 32], u1 = w1[q * 32];
-                dot_piece(u0, a, b, c0);
-                dot_piece(u1, a, b, c1);
+                const uint4 a = x[q * 32];
+                dot_piece(w0[q * 32], a, c0);
+                dot_piece(w1[q * 32], a, c1);
               }
             } else {
-#pragma unroll 2
-              for (int q = 0; q < n; ++q) dot_piece(w0[q * 32], xl[q * 32], xh[q * 32], c0);
+#pragma unroll 4
+              for (int q = 0; q < n; ++q) dot_piece(w0[q * 32], x[q * 32], c0);
             }
           }
           release_chunk();
         }
-        const float s0 = dev::warp_sum(sum4(c0));
-        const float s1 = dev::warp_sum(sum4(c1));
+        const float s0 = dev::warp_sum(sum8(c0));
+        const float s1 = dev::warp_sum(sum8(c1));
         if (lane == 0) {
           rowacc[g0 + warp] = s0;
           if (two) rowacc[g0 + warp + kConsumerWarps] = s1;
@@ -706,9 +696,9 @@ struct Consumer {
         const int lw = rg == 1 ? 3 : rg == 2 ? 2 : rg <= 4 ? 1 : 0;   // log2(warps per row)
         const int r = warp >> lw, part = warp & ((1 << lw) - 1);
         const bool active = r < rg;
-        float2 c0[4];
+        float c0[8];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) c0[i] = make_float2(0.f, 0.f);
+        for (int i = 0; i < 8; ++i) c0[i] = 0.f;
         for (int kc = 0; kc < ch.nk; ++kc) {
           const int n = ch.count(kc), p0 = ch.first(kc);
           uint32_t off;
@@ -717,15 +707,14 @@ struct Consumer {
             const int pa = (part * n) >> lw, pb = ((part + 1) * n) >> lw;
             const uint4* wr =
                 reinterpret_cast<const uint4*>(ring + off + (size_t)r * n * kPieceBytes) + lane;
-            const float4* xl = xlo + (size_t)p0 * 32;
-            const float4* xh = xhi + (size_t)p0 * 32;
-#pragma unroll 2
-            for (int q = pa; q < pb; ++q) dot_piece(wr[q * 32], xl[q * 32], xh[q * 32], c0);
+            const uint4* x = xv + (size_t)p0 * 32;
+#pragma unroll 4
+            for (int q = pa; q < pb; ++q) dot_piece(wr[q * 32], x[q * 32], c0);
           }
           release_chunk();
         }
         if (active) {
-          const float s = dev::warp_sum(sum4(c0));
+          const float s = dev::warp_sum(sum8(c0));
           if (lane == 0) {
             if (lw == 0) rowacc[g0 + r] = s;
             else sm_part(p)[warp] = s;
@@ -1272,7 +1261,7 @@ struct Consumer {
     float acc = 0.f;
     for (int k2 = tid; k2 < K / 2; k2 += kConsumerThreads) {
       const float2 v = reinterpret_cast<const float2*>(x)[k2];
-      store_pair(k2, v.x, v.y, K, nullptr, acc);
+      store_pair(k2, v.x, v.y, nullptr, acc);
     }
     dev::consumer_sync();
     bool ok = true;
