@@ -1067,6 +1067,10 @@ struct Consumer {
         put(p.obuf + ((size_t)j * G + g) * HD + dd, tag, O, skip);
       }
       if (tid == 0) p.att_ctr[layer * p.KV + j] = 0u;
+      // the combine weights live in the activation buffer, which the next
+      // stage's input load overwrites: no thread may start that load while
+      // another still reads them
+      dev::consumer_sync();
       trace(13);
     }
     return true;
