@@ -53,6 +53,41 @@ def _peaks():
         return FALLBACK_HBM_GBS, "fallback"
 
 
+KERNEL_SOURCES = ["kie_kernel.cu", "kie_device.cuh", "kie_params.h"]
+
+
+def kernel_sha() -> str:
+    import hashlib
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, "persistent_sm_decode_monokernel_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(w: synth.Workload, n_steps: int):
+    """DRAM bytes per launch from the committed ncu summary of this workload
+    (bytes per decode step x steps), or None when the summary is missing or
+    was taken on a different kernel source."""
+    path = os.path.join(ROOT, "profiles", f"monokernel_{w.name}_traffic.md")
+    try:
+        text = open(path).read()
+    except OSError:
+        return None, "no profile summary"
+    vals = {}
+    for line in text.splitlines():
+        if ":" in line and line.strip().startswith("- "):
+            k, v = line.strip()[2:].split(":", 1)
+            vals[k.strip()] = v.strip().split()[0] if v.strip() else ""
+    if vals.get("kernel_source_sha256") != kernel_sha():
+        return None, "kernel changed since the ncu capture"
+    try:
+        per_step = float(vals["dram_bytes_per_step"])
+    except (KeyError, ValueError):
+        return None, "summary lacks dram_bytes_per_step"
+    return per_step * n_steps, path
+
+
 def decode_bytes(w: synth.Workload, pos0: int, n_steps: int) -> float:
     """Algorithmic HBM bytes of n_steps decode steps starting at position
     pos0: every weight matrix, the norm gains and one embedding row per
@@ -311,6 +346,9 @@ def run_gpu(args, w, dist, rank, world):
     avg_launch_s = (sum(launch_ms) / len(launch_ms)) / 1000.0
     bytes_launch = decode_bytes(w, P, S)
     achieved = bytes_launch / avg_launch_s / 1e9
+    traffic, traffic_src = profiled_traffic(w, S)
+    if args.traffic is not None:
+        traffic, traffic_src = args.traffic, "command line"
     line = {
         "metric": METRIC, "value": value, "unit": "tok/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup,
@@ -320,7 +358,7 @@ def run_gpu(args, w, dist, rank, world):
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "peak_source": peak_kind,
                      "frac_vs_nominal_8tbs": achieved / NOMINAL_HBM_GBS,
-                     "traffic": args.traffic,
+                     "traffic": traffic, "traffic_source": traffic_src,
                      "algorithmic_bytes_per_launch": bytes_launch,
                      "avg_launch_ms": avg_launch_s * 1000.0},
         "e2e": {"value": e2e_tok / e2e_max, "unit": "tok/s",
@@ -349,14 +387,20 @@ def main(argv=None):
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=5)
     ap.add_argument("--warmup", type=int, default=3)
-    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD,
+                    choices=sorted(synth.WORKLOADS) + sorted(synth.PROFILE_WORKLOADS))
+    ap.add_argument("--decode-steps", type=int, default=None,
+                    help="decode steps per launch (default: the workload's); for profiler runs")
     ap.add_argument("--impl", default="kie", choices=["kie", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ref-tokens-per-step", type=int, default=4)
     ap.add_argument("--traffic", type=float, default=None,
                     help="DRAM bytes per launch from an ncu capture of the same kernel")
     args = ap.parse_args(argv)
-    w = synth.WORKLOADS[args.workload]
+    w = synth.workload(args.workload)
+    if args.decode_steps is not None:
+        import dataclasses
+        w = dataclasses.replace(w, decode_steps=args.decode_steps)
     if args.impl == "reference":
         rank = int(os.environ.get("RANK", "0"))
         world = int(os.environ.get("WORLD_SIZE", str(args.gpus)))

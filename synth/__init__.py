@@ -32,7 +32,8 @@ import numpy as np
 
 __all__ = [
     "ModelShape", "Workload", "WORKLOADS", "SynthModel", "make_model",
-    "make_prompt", "make_forced_ids", "tensor_names", "WEIGHT_STD",
+    "make_prompt", "make_forced_ids", "tensor_names", "WEIGHT_STD", "PROFILE_WORKLOADS",
+    "workload",
 ]
 
 WEIGHT_STD = 0.02
@@ -110,6 +111,18 @@ WORKLOADS: Dict[str, Workload] = {w.name: w for w in [
     Workload("l32-d4096", ModelShape(32, 4096, 32, 8, 128, 14336, 128256,
                                      rope_base=500000.0), 1024, 512),
 ]}
+
+
+# Smaller cases with the 2.2B model's per-layer shapes, for profiler captures
+# (an ncu capture replays each launch dozens of times; these keep the device
+# footprint to a couple of GB).
+PROFILE_WORKLOADS: Dict[str, Workload] = {w.name: w for w in [
+    Workload("l4-d2560", ModelShape(4, 2560, 20, 4, 128, 6912, 50304), 512, 8),
+]}
+
+
+def workload(name: str) -> Workload:
+    return WORKLOADS[name] if name in WORKLOADS else PROFILE_WORKLOADS[name]
 
 
 def tensor_names(n_layers: int) -> List[str]:
