@@ -82,7 +82,8 @@ typedef enum {
   KIE_ERR_CAPACITY = 4,     /* the call would write past max_seq positions */
   KIE_ERR_STATE = 5,        /* decode before prefill, or the context is failed */
   KIE_ERR_TIMEOUT = 6,      /* a device-side wait gave up (bounded spin) */
-  KIE_ERR_PROTOCOL = 7      /* a device-side consistency check failed */
+  KIE_ERR_PROTOCOL = 7,     /* a device-side consistency check failed */
+  KIE_ERR_TOO_LARGE = 8     /* larger than the fixed scratch of kie_gemv_f16_noalloc */
 } kie_status;
 
 /* Model shape.  Supported: head_dim 64 or 128; n_heads a multiple of
@@ -233,6 +234,36 @@ KIE_API kie_status kie_destroy(kie_ctx *ctx);
 KIE_API kie_status kie_gemv_f16(const void *W, const float *x, float *y, int32_t N, int32_t K,
                                 int32_t iters, int32_t mode, int32_t chunk_bytes,
                                 void *cuda_stream, float *ms_out, double *stats_out);
+
+/* Largest fp16 weight matrix (N*K*2 bytes) kie_gemv_f16_noalloc takes. */
+#define KIE_NOALLOC_MAX_WEIGHT_BYTES (16u * 1024u * 1024u)
+
+/* The GEMV of kie_gemv_f16 (mode 1, one pass, 32 KB chunks) for callers
+ * that cannot allocate device memory: a process that reserved all of the
+ * GPU's memory for its own pool at start-up, where cudaMalloc would fail or
+ * eat into that pool, or a latency-bound loop, where cudaMalloc and
+ * cudaFree synchronise the device.  The pages describe no such entry point;
+ * it exists for these callers only.
+ *
+ * y[N] = W[N][K] x[K]: W fp16 row-major, x and y fp32, all device pointers
+ * (W and x 16-byte aligned), K a multiple of 256, N >= 1, and
+ * N*K*2 <= KIE_NOALLOC_MAX_WEIGHT_BYTES, else KIE_ERR_TOO_LARGE.  The caller
+ * owns W, x and y.  All device scratch (the streamed copy of W, the row
+ * split, the status word) lives in one fixed array compiled into the
+ * library, of KIE_NOALLOC_MAX_WEIGHT_BYTES plus under 64 KB; every GPU that
+ * loads the library holds it until the process exits.  The call allocates
+ * no device memory.
+ *
+ * The first call on a device looks up the array's address on that device
+ * (cudaGetSymbolAddress, which may load the library's device code there);
+ * make that first call before any stream capture.  Every call clears the
+ * parts of the array that must start at zero; all calls on a device share
+ * the array, so calls that overlap on the GPU (two streams, two host
+ * threads) race and give wrong results: serialise them.  Synchronous on
+ * `cuda_stream`.  Errors: KIE_ERR_INVALID_ARG, KIE_ERR_TOO_LARGE,
+ * KIE_ERR_CUDA, KIE_ERR_TIMEOUT (a bounded device wait gave up). */
+KIE_API kie_status kie_gemv_f16_noalloc(const void *W, const float *x, float *y, int32_t N,
+                                        int32_t K, void *cuda_stream);
 
 /* Host-only planning query (no CUDA call): the unit range [begin, end) that
  * CTA `cta` of a `grid`-CTA launch owns in GEMV stage `stage` (0 QKV, 1 O,

@@ -25,6 +25,9 @@ KIE_ERR_CAPACITY = 4
 KIE_ERR_STATE = 5
 KIE_ERR_TIMEOUT = 6
 KIE_ERR_PROTOCOL = 7
+KIE_ERR_TOO_LARGE = 8
+
+KIE_NOALLOC_MAX_WEIGHT_BYTES = 16 * 1024 * 1024
 
 KIE_OPT_TIMEOUT_NS = 1
 KIE_OPT_CHUNK_BYTES = 2
@@ -94,6 +97,7 @@ SIGNATURES = {
     "kie_gemv_f16": (ctypes.c_int, [_P, _P, _P, _I32, _I32, _I32, _I32, _I32, _P,
                                     ctypes.POINTER(ctypes.c_float),
                                     ctypes.POINTER(ctypes.c_double)]),
+    "kie_gemv_f16_noalloc": (ctypes.c_int, [_P, _P, _P, _I32, _I32, _P]),
 }
 
 _lib: Optional[ctypes.CDLL] = None
@@ -253,6 +257,15 @@ def kie_gemv_f16(W, x, y, iters: int = 1, mode: int = 1, chunk_bytes: int = 3276
            "kie_gemv_f16")
     return ms.value, {"stream_wait_cycles": st[0], "producer_wait_cycles": st[1],
                       "grid": int(st[2]), "ring_bytes": int(st[3])}
+
+
+def kie_gemv_f16_noalloc(W, x, y, stream=None) -> None:
+    """y = W x through the entry point that allocates no device memory (its
+    scratch is a fixed array inside the library; see kie.h)."""
+    N, K = W.shape
+    _check(load_library().kie_gemv_f16_noalloc(_ptr(W), _ptr(x), _ptr(y), N, K,
+                                               ctypes.c_void_p(stream or 0)),
+           "kie_gemv_f16_noalloc")
 
 
 def kie_destroy(ctx) -> None:

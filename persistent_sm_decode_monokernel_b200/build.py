@@ -18,7 +18,7 @@ CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(HERE, "libkie.so")
 
-SOURCES = ["kie_host.cu", "kie_kernel.cu", "kie_plan.cpp"]
+SOURCES = ["kie_host.cu", "kie_kernel.cu", "kie_plan.cpp", "kie_noalloc.cu"]
 HEADERS = ["kie_params.h", "kie_plan.h", "kie_kernel.h", "kie_device.cuh"]
 
 NVCC_FLAGS = [

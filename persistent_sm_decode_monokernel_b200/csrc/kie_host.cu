@@ -741,6 +741,7 @@ const char* kie_status_str(kie_status s) {
     case KIE_ERR_STATE: return "invalid state";
     case KIE_ERR_TIMEOUT: return "device wait timed out";
     case KIE_ERR_PROTOCOL: return "device protocol violation";
+    case KIE_ERR_TOO_LARGE: return "size exceeds the fixed scratch of the no-allocation entry point";
   }
   return "unknown status";
 }

@@ -128,6 +128,6 @@ def test_plan_units_rejects_bad_args(lib):
 
 
 def test_status_strings(lib):
-    for s in range(8):
+    for s in range(9):
         assert lib.kie_status_str(s)
     assert lib.kie_status_str(99) == b"unknown status"
