@@ -140,7 +140,8 @@ typedef struct {
 typedef enum {
   KIE_OPT_TIMEOUT_NS = 1,     /* bound of every device-side wait (default 2e9) */
   KIE_OPT_CHUNK_BYTES = 2,    /* largest weight chunk in bytes (>= 8192, multiple of 512;
-                                 default 32768); re-plans the ring and rebuilds the packed
+                                 default 65536, or 32768 where two 64 KB chunks do not
+                                 fit the ring); re-plans the ring and rebuilds the packed
                                  weight copy, so the caller's matrices must still be valid */
   KIE_OPT_MIN_SPLIT_LEN = 3,  /* minimum positions per attention split (default 64) */
   KIE_OPT_FAULT_CTA = 4,      /* test hook: CTA that withholds one publication (-1 off) */
@@ -148,7 +149,10 @@ typedef enum {
   KIE_OPT_FAULT_LAYER = 6,    /* test hook: layer of the withheld publication */
   KIE_OPT_FAULT_STAGE = 7,    /* test hook: 0 QKV, 1 O, 2 gate/up, 3 down, 4 LM */
   KIE_OPT_POLL_BACKOFF_NS = 8, /* sleep between re-polls of another CTA's data (default 128) */
-  KIE_OPT_TRACE_CLOCK = 9      /* stage trace in SM cycles (1) instead of ns (0, default) */
+  KIE_OPT_TRACE_CLOCK = 9,     /* stage trace in SM cycles (1) instead of ns (0, default) */
+  KIE_OPT_L2_PREFETCH_BYTES = 10 /* per CTA, weight-stream bytes requested into L2 ahead of
+                                    the shared-memory ring (multiple of 512, <= 16 MiB;
+                                    0 = off, the default) */
 } kie_option;
 
 /* Bytes of the caller-provided KV cache: 2*n_layers*n_kv_heads*max_seq*head_dim*2.
@@ -203,7 +207,9 @@ KIE_API kie_status kie_set_logits_capture(kie_ctx *ctx, float *dev_logits,
 
 /* Stage trace (measurement): while set, CTA `cta` of every launch writes
  * %globaltimer stamps (ns) to dev_buf, a device buffer of `capacity` u64
- * owned by the caller.  Per step it writes n_layers*16 + 4 slots: for each
+ * owned by the caller; cta = -1 traces every CTA, laid out
+ * [step][cta][slot] (grid CTAs per step, see kie_get_stats).  Per step and
+ * CTA it writes n_layers*16 + 4 slots: for each
  * layer QKV begin, QKV input ready, QKV done, attention done, O input
  * ready, O done, gate/up input ready, gate/up done, down input ready, down
  * done, and (CTAs with attention work) q ready, attention math done,

@@ -83,11 +83,13 @@ class Session:
 
     def trace(self, steps: int, cta: int = 0):
         """Turns the stage trace on for `steps` steps of CTA `cta`; returns the
-        [steps, n_layers*16 + 4] int64 device buffer it fills."""
+        [steps, n_layers*16 + 4] int64 device buffer it fills.  cta=-1 traces
+        every CTA into a [steps, grid, n_layers*16 + 4] buffer."""
         import torch
         per = self.shape.n_layers * 16 + 4
-        self._trace = torch.zeros((steps, per), dtype=torch.int64, device="cuda")
-        kie_set_trace(self.ctx, self._trace, steps * per, cta)
+        shape = (steps, per) if cta >= 0 else (steps, self.stats()["grid"], per)
+        self._trace = torch.zeros(shape, dtype=torch.int64, device="cuda")
+        kie_set_trace(self.ctx, self._trace, self._trace.numel(), cta)
         return self._trace
 
     def trace_off(self) -> None:

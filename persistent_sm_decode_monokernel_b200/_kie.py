@@ -38,6 +38,7 @@ KIE_OPT_FAULT_LAYER = 6
 KIE_OPT_FAULT_STAGE = 7
 KIE_OPT_POLL_BACKOFF_NS = 8
 KIE_OPT_TRACE_CLOCK = 9
+KIE_OPT_L2_PREFETCH_BYTES = 10
 
 STAGE_QKV, STAGE_O, STAGE_GU, STAGE_DOWN, STAGE_LM = range(5)
 

@@ -48,7 +48,7 @@ struct kie_ctx {
 
   // plan
   std::vector<std::vector<int2>> hranges;
-  int grid = 0, ring_bytes = 0, chunk_bytes = 32768, smem = 0, max_split = 1, min_split_len = 64;
+  int grid = 0, ring_bytes = 0, chunk_bytes = 65536, smem = 0, max_split = 1, min_split_len = 64;
   unsigned char* packed = nullptr;            // weight matrices in per-CTA stream order
   unsigned long long* packed_off = nullptr;   // [grid]
   size_t packed_bytes = 0;
@@ -65,6 +65,7 @@ struct kie_ctx {
   // options and capture
   long long timeout_ns = 2000000000LL;
   unsigned poll_ns = 128;
+  long long l2_prefetch = 0;
   int fault_cta = -1, fault_step = -1, fault_layer = -1, fault_stage = -1;
   float* capture = nullptr;
   int capture_rows = 0;
@@ -186,6 +187,7 @@ kie_status launch(kie_ctx* c, int n_steps, int pos0, const int32_t* host_ids, bo
   p.cta_stats = c->cta_stats;
   p.timeout_ns = c->timeout_ns;
   p.poll_ns = c->poll_ns;
+  p.l2_prefetch = c->l2_prefetch;
   p.trace = c->trace;
   p.trace_cta = c->trace_cta;
   p.trace_steps = c->trace_steps;
@@ -360,9 +362,15 @@ kie_status kie_create(const kie_model_desc* d, const kie_weights* w, void* kv_ca
   c->grid = grid;
   c->hranges.resize(kie::N_STAGES);
   for (int st = 0; st < kie::N_STAGES; ++st) c->hranges[st] = kie::partition(c->shape, grid, st);
-  if (!kie::plan_smem(c->shape, grid, c->chunk_bytes, smem_optin, c->hranges, &c->sm,
-                      &c->ring_bytes))
-    return fail(KIE_ERR_UNSUPPORTED);
+  // largest chunk that leaves room for two in the ring: 64 KB, else 32 KB
+  bool planned = false;
+  for (int cb : {65536, 32768}) {
+    c->chunk_bytes = cb;
+    if ((planned = kie::plan_smem(c->shape, grid, cb, smem_optin, c->hranges, &c->sm,
+                                  &c->ring_bytes)))
+      break;
+  }
+  if (!planned) return fail(KIE_ERR_UNSUPPORTED);
   c->smem = c->sm.total;
   int per_sm = 0;
   if (cuda_bad(kie::mono_configure(d->head_dim, c->smem, &per_sm))) return fail(KIE_ERR_CUDA);
@@ -387,7 +395,7 @@ kie_status kie_create(const kie_model_desc* d, const kie_weights* w, void* kv_ca
       cuda_bad(cudaMalloc(&c->rope, sizeof(float2) * rope.size())) ||
       cuda_bad(cudaMalloc(&c->ranges, sizeof(int2) * flat.size())) ||
       cuda_bad(cudaMalloc(&c->tagged, 8 * c->tagged_words)) ||
-      cuda_bad(cudaMalloc(&c->partials, sizeof(float) * (size_t)grid * G * (d->head_dim + 2))) ||
+      cuda_bad(cudaMalloc(&c->partials, sizeof(float) * (size_t)grid * G * (d->head_dim + 4))) ||
       cuda_bad(cudaMalloc(&c->att_ctr, sizeof(unsigned) * d->n_layers * d->n_kv_heads)) ||
       cuda_bad(cudaMalloc(&c->d_ids, sizeof(int32_t) * d->max_seq)) ||
       cuda_bad(cudaMalloc(&c->d_io, kStatusBytes + sizeof(int32_t) * d->max_seq)) ||
@@ -646,12 +654,12 @@ kie_status kie_gemv_f16(const void* W, const float* x, float* y, int32_t N, int3
 
 kie_status kie_set_trace(kie_ctx* c, uint64_t* dev_buf, int32_t capacity, int32_t cta) {
   if (!c) return KIE_ERR_INVALID_ARG;
-  if (dev_buf && (capacity < 1 || cta < 0 || cta >= c->grid))
+  if (dev_buf && (capacity < 1 || cta < -1 || cta >= c->grid))
     return set_err(c, KIE_ERR_INVALID_ARG, "bad trace buffer or CTA");
   const int per = c->desc.n_layers * kie::kTracePerLayer + 4;
   c->trace = reinterpret_cast<unsigned long long*>(dev_buf);
   c->trace_cta = cta;
-  c->trace_steps = dev_buf ? capacity / per : 0;
+  c->trace_steps = dev_buf ? capacity / (per * (cta < 0 ? c->grid : 1)) : 0;
   return KIE_OK;
 }
 
@@ -695,6 +703,10 @@ kie_status kie_set_option(kie_ctx* c, kie_option opt, int64_t v) {
     case KIE_OPT_POLL_BACKOFF_NS:
       if (v < 0 || v > 100000) return KIE_ERR_INVALID_ARG;
       c->poll_ns = (unsigned)v;
+      return KIE_OK;
+    case KIE_OPT_L2_PREFETCH_BYTES:
+      if (v < 0 || v % 512 || v > (16 << 20)) return KIE_ERR_INVALID_ARG;
+      c->l2_prefetch = v;
       return KIE_OK;
     case KIE_OPT_FAULT_CTA: c->fault_cta = (int)v; return KIE_OK;
     case KIE_OPT_FAULT_STEP: c->fault_step = (int)v; return KIE_OK;

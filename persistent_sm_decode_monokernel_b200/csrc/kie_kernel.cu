@@ -234,9 +234,41 @@ struct Producer {
   uint32_t wend;   // ring write position
   uint32_t live_off[kRingBars], live_end[kRingBars];
   long long t_wait;  // cycles spent waiting for ring space
+  // L2 prefetch of the weight stream (p.l2_prefetch > 0): the bytes from
+  // the copy cursor to p.l2_prefetch beyond it are kept requested into L2,
+  // across stage and step boundaries, so HBM keeps streaming while the ring
+  // is full and later copies hit L2.
+  const unsigned char* wbase;
+  long long len_layers, len_lm;  // bytes of the CTA's per-step stream
+  long long pf_ahead;            // bytes requested beyond the copy cursor
+  long long pf_off;              // prefetch cursor: offset within step pf_step
+  int pf_step;
 
   __device__ explicit Producer(const MonoParams& pp)
-      : p(pp), pol(dev::policy_evict_first()), idx(0), cons(0), wend(0), t_wait(0) {}
+      : p(pp), pol(dev::policy_evict_first()), idx(0), cons(0), wend(0), t_wait(0),
+        wbase(nullptr), len_layers(0), len_lm(0), pf_ahead(0), pf_off(0), pf_step(0) {}
+
+  __device__ long long stage_len(int st) const {
+    const int2 r = p.ranges[st * p.grid + blockIdx.x];
+    return (long long)range_rows(p, st, r.x, r.y) * stage_k(p, st) * 2;
+  }
+
+  // Tops the prefetch up to `next` + p.l2_prefetch bytes beyond the copy cursor.
+  __device__ void prefetch(uint32_t next) {
+    const long long want = (long long)next + p.l2_prefetch;
+    while (pf_ahead < want && pf_step < p.n_steps) {
+      const long long rem = len_layers + (pf_step >= p.lm_from ? len_lm : 0) - pf_off;
+      if (rem <= 0) {
+        ++pf_step;
+        pf_off = 0;
+        continue;
+      }
+      const long long g = min(min(rem, 65536ll), want - pf_ahead);
+      dev::bulk_prefetch_l2(wbase + pf_off, (uint32_t)g);
+      pf_off += g;
+      pf_ahead += g;
+    }
+  }
 
   // Waits until chunk i has been consumed; false = stop.
   __device__ bool wait_consumed(uint32_t i) {
@@ -304,8 +336,12 @@ struct Producer {
     for (int g0 = 0; g0 < R; g0 += kGroupRows) {
       const int rg = min(kGroupRows, R - g0);
       const Chunking ch = chunking(rg, kp, p.chunk_bytes);
-      for (int kc = 0; kc < ch.nk; ++kc)
-        if (!chunk(src, (uint32_t)(rg * ch.count(kc) * kPieceBytes))) return false;
+      for (int kc = 0; kc < ch.nk; ++kc) {
+        const uint32_t sz = (uint32_t)(rg * ch.count(kc) * kPieceBytes);
+        if (p.l2_prefetch > 0) prefetch(sz);
+        if (!chunk(src, sz)) return false;
+        pf_ahead -= sz;
+      }
     }
     return true;
   }
@@ -372,6 +408,9 @@ struct Producer {
   __device__ void run() {
     bool ok = true;
     const unsigned char* base = p.packed + p.packed_off[blockIdx.x];
+    wbase = base;
+    len_layers = p.L * (stage_len(ST_QKV) + stage_len(ST_O) + stage_len(ST_GU) + stage_len(ST_DOWN));
+    len_lm = stage_len(ST_LM);
     for (int i = 0; i < p.n_steps && ok; ++i) {
       const unsigned char* src = base;
       for (int l = 0; l < p.L && ok; ++l)
@@ -431,9 +470,11 @@ struct Consumer {
   // 10 per layer (QKV begin/loaded/done, attention done, O loaded/done,
   // gate-up loaded/done, down loaded/done) + 4 for the LM head.
   __device__ __forceinline__ void trace(int ev) const {
-    if (p.trace && tid == 0 && (int)blockIdx.x == p.trace_cta && step < p.trace_steps) {
+    if (p.trace && tid == 0 && (p.trace_cta < 0 || (int)blockIdx.x == p.trace_cta) &&
+        step < p.trace_steps) {
       const int per = p.L * kTracePerLayer + 4;
-      const int idx = step * per + (layer < p.L ? layer * kTracePerLayer : p.L * kTracePerLayer) + ev;
+      const int row = p.trace_cta < 0 ? step * p.grid + (int)blockIdx.x : step;
+      const int idx = row * per + (layer < p.L ? layer * kTracePerLayer : p.L * kTracePerLayer) + ev;
       p.trace[idx] = p.trace_clock ? (unsigned long long)clock64()
                                    : (unsigned long long)dev::globaltimer();
     }
@@ -563,12 +604,12 @@ struct Consumer {
 
   // Loads a K-vector into xs (times `gain` if given) and returns in `ss` the
   // sum of squares of the raw values.  Source: tagged words, or an fp16
-  // embedding row.  The polls of one thread are issued in batches of 16-byte
-  // loads so that their L2 round trips overlap.  Returns false (uniformly)
-  // on abort.
+  // embedding row.  The polls of one thread are issued in batches of up to
+  // 16 16-byte loads (one batch for K <= 8192) so that their L2 round trips
+  // overlap.  Returns false (uniformly) on abort.
   __device__ __noinline__ bool load_vec(const u64* src, unsigned tag, const __half* emb, int K,
                            const __half* gain, float& ss, int where) {
-    constexpr int NB = 4;
+    constexpr int NB = 8;
     const long long c0 = clock64();
     float acc = 0.f;
     bool bad = false;
@@ -792,6 +833,84 @@ struct Consumer {
     return true;
   }
 
+  // The last item of KV head j combines all nsplit partials:
+  // weights w_q = exp(m_q - M) / sum_q exp(m_q - M) l_q per head.
+  // Warp g reads head g's (m, l) of every split at once (lane = split);
+  // then each thread owns 4 output dims of one head and issues the loads of
+  // 8 splits before using any, so a combine costs a few L2 round trips.
+  template <int HD>
+  __device__ __noinline__ void attn_combine(int j, int nsplit, unsigned tag) {
+    constexpr int PST = HD + 4;
+    const int G = p.G;
+    float* wq = sm_xs(p) + (HD / 8) * (G * 8 + 4);     // the scores area: [nsplit][G]
+    dev::fence_acq_rel_gpu();
+    const float* base = p.partials + (size_t)(j * nsplit) * G * PST;
+    if (warp < G) {
+      constexpr int QPL = (kMaxSplitCombine + 31) / 32;
+      float mv[QPL], lv[QPL];
+      float M = -INFINITY;
+#pragma unroll
+      for (int k = 0; k < QPL; ++k) {
+        const int q = lane + 32 * k;
+        mv[k] = -INFINITY;
+        lv[k] = 0.f;
+        if (q < nsplit) {
+          const float2 ml = *reinterpret_cast<const float2*>(base + ((size_t)q * G + warp) * PST);
+          mv[k] = ml.x;
+          lv[k] = ml.y;
+        }
+      }
+#pragma unroll
+      for (int k = 0; k < QPL; ++k) M = fmaxf(M, mv[k]);
+      M = dev::warp_max(M);
+      float f[QPL], Ls = 0.f;
+#pragma unroll
+      for (int k = 0; k < QPL; ++k) {
+        f[k] = lane + 32 * k < nsplit ? expf(mv[k] - M) : 0.f;
+        Ls = fmaf(f[k], lv[k], Ls);
+      }
+      const float inv = 1.0f / dev::warp_sum(Ls);
+#pragma unroll
+      for (int k = 0; k < QPL; ++k)
+        if (lane + 32 * k < nsplit) wq[(lane + 32 * k) * G + warp] = f[k] * inv;
+    }
+    dev::consumer_sync();
+    const bool skip = fault_here(1);
+    for (int e = tid; e < G * HD / 4; e += kConsumerThreads) {
+      const int g = e / (HD / 4), d4 = e - g * (HD / 4);
+      const float* src = base + (size_t)g * PST + 4 + 4 * d4;
+      float4 O = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int q0 = 0; q0 < nsplit; q0 += 8) {
+        float4 v[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+          if (q0 + u < nsplit)
+            v[u] = *reinterpret_cast<const float4*>(src + (size_t)(q0 + u) * G * PST);
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          if (q0 + u < nsplit) {
+            const float wv = wq[(q0 + u) * G + g];
+            O.x = fmaf(wv, v[u].x, O.x);
+            O.y = fmaf(wv, v[u].y, O.y);
+            O.z = fmaf(wv, v[u].z, O.z);
+            O.w = fmaf(wv, v[u].w, O.w);
+          }
+        }
+      }
+      u64* dst = p.obuf + ((size_t)j * G + g) * HD + 4 * d4;
+      put(dst, tag, O.x, skip);
+      put(dst + 1, tag, O.y, skip);
+      put(dst + 2, tag, O.z, skip);
+      put(dst + 3, tag, O.w, skip);
+    }
+    if (tid == 0) p.att_ctr[layer * p.KV + j] = 0u;
+    // the combine weights live in the activation buffer, which the next
+    // stage's input load overwrites: no thread may start that load while
+    // another still reads them
+    dev::consumer_sync();
+    trace(13);
+  }
+
   // Split-K attention over positions 0..pos for the G query heads of one
   // KV head; the last item of a KV head combines the partials.  K and V
   // blocks arrive through the ring (issued by the producer before q is
@@ -1011,16 +1130,16 @@ struct Consumer {
       }
     }
     trace(11);
-    // publish this item's partial (m, l, unnormalised o)
-    float* part = p.partials + (size_t)blockIdx.x * G * (HD + 2);
-    for (int e = tid; e < G * HD; e += kConsumerThreads) {
-      const int g = e / HD, dd = e - g * HD;
-      part[g * (HD + 2) + 2 + dd] = orun[e];
+    // publish this item's partial: per head a row [m, l, -, -, o[HD]] of
+    // HD + 4 floats (16-byte aligned rows; o unnormalised)
+    constexpr int PST = HD + 4;
+    float* part = p.partials + (size_t)blockIdx.x * G * PST;
+    for (int e = tid; e < G * HD / 4; e += kConsumerThreads) {
+      const int g = e / (HD / 4), d4 = e - g * (HD / 4);
+      *reinterpret_cast<float4*>(part + g * PST + 4 + 4 * d4) =
+          *reinterpret_cast<const float4*>(orun + g * HD + 4 * d4);
     }
-    if (tid < G) {
-      part[tid * (HD + 2)] = mrun[tid];
-      part[tid * (HD + 2) + 1] = lrun[tid];
-    }
+    if (tid < G) *reinterpret_cast<float2*>(part + tid * PST) = make_float2(mrun[tid], lrun[tid]);
     dev::consumer_sync();
     const int nsplit = it.nsplit;
     if (tid == 0) {
@@ -1030,49 +1149,7 @@ struct Consumer {
     }
     dev::consumer_sync();
     trace(12);
-    if (sm_flags(p)[F_LAST]) {
-      dev::fence_acq_rel_gpu();
-      // the last item of KV head j combines all nsplit partials:
-      // weights w_q = exp(m_q - M) / sum_q exp(m_q - M) l_q per head
-      const float* base = p.partials + (size_t)(j * nsplit) * G * (HD + 2);
-      float* wq = sc;                                   // [nsplit][G]
-      float* mq = sc + kMaxSplitCombine * kMaxGroup;    // [nsplit][G] m, then l
-      for (int e = tid; e < nsplit * G; e += kConsumerThreads) {
-        const int q = e / G, g = e - (e / G) * G;
-        const float2 ml = *reinterpret_cast<const float2*>(base + ((size_t)q * G + g) * (HD + 2));
-        mq[2 * e] = ml.x;
-        mq[2 * e + 1] = ml.y;
-      }
-      dev::consumer_sync();
-      if (tid < G) {
-        float M = -INFINITY;
-        for (int q = 0; q < nsplit; ++q) M = fmaxf(M, mq[2 * (q * G + tid)]);
-        float Lsum = 0.f;
-        for (int q = 0; q < nsplit; ++q) {
-          const float f = expf(mq[2 * (q * G + tid)] - M);
-          wq[q * G + tid] = f;
-          Lsum = fmaf(f, mq[2 * (q * G + tid) + 1], Lsum);
-        }
-        const float inv = 1.0f / Lsum;
-        for (int q = 0; q < nsplit; ++q) wq[q * G + tid] *= inv;
-      }
-      dev::consumer_sync();
-      const bool skip = fault_here(1);
-      for (int e = tid; e < G * HD; e += kConsumerThreads) {
-        const int g = e / HD, dd = e - g * HD;
-        float O = 0.f;
-#pragma unroll 4
-        for (int q = 0; q < nsplit; ++q)
-          O = fmaf(wq[q * G + g], base[((size_t)q * G + g) * (HD + 2) + 2 + dd], O);
-        put(p.obuf + ((size_t)j * G + g) * HD + dd, tag, O, skip);
-      }
-      if (tid == 0) p.att_ctr[layer * p.KV + j] = 0u;
-      // the combine weights live in the activation buffer, which the next
-      // stage's input load overwrites: no thread may start that load while
-      // another still reads them
-      dev::consumer_sync();
-      trace(13);
-    }
+    if (sm_flags(p)[F_LAST]) attn_combine<HD>(j, nsplit, tag);
     return true;
   }
 

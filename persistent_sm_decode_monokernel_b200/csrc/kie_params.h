@@ -69,7 +69,7 @@ struct MonoParams {
   SmemLayout sm;
   // scratch (tagged 64-bit words: high 32 bits = epoch tag, low = fp32 bits)
   unsigned long long *x_attn, *x_ffn, *hbuf, *qbuf, *kvnew, *obuf, *slots;
-  float* partials;         // [grid][G][hd + 2]
+  float* partials;         // [grid][G][hd + 4]: m, l, 2 unused, o[hd]
   unsigned int* att_ctr;   // [L][KV] last-arriver counters
   // run
   int n_steps, pos0, first_tok;
@@ -83,6 +83,7 @@ struct MonoParams {
   unsigned long long* cta_stats;  // [grid][kStatsPerCta]
   long long timeout_ns;
   unsigned poll_ns;        // sleep between re-polls of tagged words
+  long long l2_prefetch;   // weight-stream bytes kept requested into L2 ahead of the copies
   unsigned long long* trace;  // stage timestamps of CTA trace_cta, or null
   int trace_cta, trace_steps;
   int trace_clock;         // 1: stamps are SM cycles (clock64), 0: %globaltimer ns
