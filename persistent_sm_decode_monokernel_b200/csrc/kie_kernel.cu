@@ -83,6 +83,11 @@ __device__ __forceinline__ float* sm_res_ffn(const MonoParams& p) {
 __device__ __forceinline__ const unsigned char* sm_ring(const MonoParams& p) {
   return kie_smem + p.sm.ring_off;
 }
+// Writable view of the ring, for the consumers' fills of attention tiles
+// they own (after the tile's copies have landed).
+__device__ __forceinline__ unsigned char* sm_ring_w(const MonoParams& p) {
+  return kie_smem + p.sm.ring_off;
+}
 __device__ __forceinline__ uint32_t sm_ring_s(const MonoParams& p) {
   return dev::smem_u32(kie_smem + p.sm.ring_off);
 }
@@ -197,9 +202,14 @@ __device__ __forceinline__ AttnItem attn_item(const MonoParams& p, int pos) {
   a.t1 = (int)(((long long)(s + 1) * n_pos) / nsplit);
   return a;
 }
-// Positions per attention block (one K chunk and one V chunk in the ring).
+// Attention K/V tiles in the ring: rows of hd fp16 at a stride of hd + 8
+// elements, so that the 8 rows an mma fragment load touches fall in 8
+// different bank groups.
+__device__ __forceinline__ int attn_row_stride(const MonoParams& p) { return (p.hd + 8) * 2; }
+// Positions per attention block (one K tile and one V tile in the ring), a
+// multiple of 16.
 __device__ __forceinline__ int attn_block(const MonoParams& p) {
-  return min(kAttnBlock, p.chunk_bytes / (p.hd * 2));
+  return max(16, min(kAttnBlock, p.chunk_bytes / attn_row_stride(p)) & ~15);
 }
 __device__ __forceinline__ const __half* kv_rows(const MonoParams& p, int layer, int kv, int j) {
   return p.kv + (((size_t)layer * 2 + kv) * p.KV + j) * (size_t)p.max_seq * p.hd;
@@ -329,6 +339,26 @@ struct Producer {
     return true;
   }
 
+  // One attention tile: `alloc` ring bytes, of which rows [0, n) are copied
+  // from `src` (row_bytes each, contiguous) at a ring stride of `stride`;
+  // the consumers fill the remaining rows.
+  __device__ bool tile(const unsigned char* src, int n, uint32_t row_bytes, uint32_t stride,
+                       uint32_t alloc) {
+    if (sm_flags(p)[F_STOP]) return false;
+    const uint32_t off = ring_place(wend, alloc, (uint32_t)p.ring_bytes);
+    if (!acquire(off, off + alloc)) return false;
+    const uint32_t b = idx & (kRingBars - 1);
+    const uint32_t full = sm_full_s(p) + 8 * b;
+    dev::mbar_arrive_expect_tx(full, (uint32_t)n * row_bytes);
+    for (int r = 0; r < n; ++r)
+      dev::bulk_g2s(sm_ring_s(p) + off + r * stride, src + (size_t)r * row_bytes, row_bytes, full,
+                    pol);
+    live_off[b] = off;
+    live_end[b] = off + alloc;
+    ++idx;
+    return true;
+  }
+
   __device__ bool stage(int st, const unsigned char*& src) {
     const int2 r = p.ranges[st * p.grid + blockIdx.x];
     const int R = range_rows(p, st, r.x, r.y);
@@ -375,13 +405,14 @@ struct Producer {
     const int tb = attn_block(p);
     const unsigned char* K = reinterpret_cast<const unsigned char*>(kv_rows(p, l, 0, it.j));
     const unsigned char* V = reinterpret_cast<const unsigned char*>(kv_rows(p, l, 1, it.j));
-    const size_t row = (size_t)p.hd * 2;
+    const uint32_t row = (uint32_t)p.hd * 2, stride = (uint32_t)attn_row_stride(p);
     for (int b0 = it.t0; b0 < it.t1; b0 += tb) {
-      const int nc = min(min(it.t1, b0 + tb), pos) - b0;
-      if (nc <= 0) continue;
-      const unsigned char* k = K + b0 * row;
-      const unsigned char* v = V + b0 * row;
-      if (!chunk(k, (uint32_t)(nc * row)) || !chunk(v, (uint32_t)(nc * row))) return false;
+      const int nb = min(it.t1, b0 + tb) - b0;
+      const int nc = max(0, min(b0 + nb, pos) - b0);   // rows already in the cache
+      const uint32_t alloc = (uint32_t)((nb + 15) & ~15) * stride;
+      if (!tile(K + (size_t)b0 * row, nc, row, stride, alloc) ||
+          !tile(V + (size_t)b0 * row, nc, row, stride, alloc))
+        return false;
     }
     return true;
   }
@@ -449,6 +480,34 @@ __device__ void repack_stage(const MonoParams& p, int st, const LayerW& w, unsig
 }
 
 // ----------------------------------------------------------------- consumer
+
+// Attention scratch in the activation area of shared memory: q as fp16 hi
+// and lo tiles [16][HD + 8], P tile [16][kAttnBlock + 8] fp16, scores
+// [G][kAttnBlock] fp32 (the combine reuses them), the current position's k
+// and v, the running output [G][HD] and per-head running max, sum and
+// rescale factor.
+template <int HD>
+struct AttnSmem {
+  __half *qhi, *qlo, *ps;
+  float *sc, *kn, *vn, *orun, *mrun, *lrun, *alpha;
+  __device__ explicit AttnSmem(const MonoParams& p) {
+    unsigned char* b = reinterpret_cast<unsigned char*>(sm_xs(p));
+    qhi = reinterpret_cast<__half*>(b);
+    b += 16 * (HD + 8) * 2;
+    qlo = reinterpret_cast<__half*>(b);
+    b += 16 * (HD + 8) * 2;
+    ps = reinterpret_cast<__half*>(b);
+    b += 16 * (kAttnBlock + 8) * 2;
+    sc = reinterpret_cast<float*>(b);
+    b += max(p.G * kAttnBlock, 3 * kMaxSplitCombine * kMaxGroup) * 4;
+    kn = reinterpret_cast<float*>(b);
+    vn = kn + HD;
+    orun = vn + HD;
+    mrun = orun + p.G * HD;
+    lrun = mrun + kMaxGroup;
+    alpha = lrun + kMaxGroup;
+  }
+};
 
 struct Consumer {
   const MonoParams& p;
@@ -842,7 +901,7 @@ struct Consumer {
   __device__ __noinline__ void attn_combine(int j, int nsplit, unsigned tag) {
     constexpr int PST = HD + 4;
     const int G = p.G;
-    float* wq = sm_xs(p) + (HD / 8) * (G * 8 + 4);     // the scores area: [nsplit][G]
+    float* wq = AttnSmem<HD>(p).sc;                   // the scores area: [nsplit][G]
     dev::fence_acq_rel_gpu();
     const float* base = p.partials + (size_t)(j * nsplit) * G * PST;
     if (warp < G) {
@@ -913,39 +972,40 @@ struct Consumer {
 
   // Split-K attention over positions 0..pos for the G query heads of one
   // KV head; the last item of a KV head combines the partials.  K and V
-  // blocks arrive through the ring (issued by the producer before q is
-  // ready); the current position's k and v come from the tagged words.
-  //   scores: P = 1, 2 or 4 threads per position split the HD/8 16-byte
-  //           chunks of the K row: part p of position t reads chunk
-  //           (p + P*(i + t)) mod HD/8 at step i, so the 8 lanes of a load
-  //           phase read chunks with 8 different residues mod 8 (8 bank
-  //           groups); q sits chunk-major with an odd multiple of 4 floats
-  //           per chunk row, so the same rotated reads of q are
-  //           conflict-free too;
-  //   P.V:    thread (head g, 4 dims) runs over the block's positions with
-  //           four independent accumulators.
+  // tiles arrive through the ring (issued by the producer before q is
+  // ready, rows at a padded stride); the current position's k and v come
+  // from the tagged words and are written into the tiles here.  Both
+  // contractions run on warp-level mma (m16n8k16, fp16 in, fp32 out):
+  //   scores: S^T[head][t] = Q K^T, A = q (heads padded to 16 rows) split
+  //           into fp16 hi + lo parts so that S keeps fp32 accuracy, B = the
+  //           K tile; warps take 8-position column tiles in turn;
+  //   softmax: warp g owns head g (online over the item's blocks); P is
+  //           rounded to fp16 and its row sums use the rounded values;
+  //   P.V:    O[head][dims] += P V, B fragments by transposed ldmatrix from
+  //           the V tile; warp w owns HD/8 dims.
   template <int HD>
   __device__ __noinline__ bool stage_attn(int pos, unsigned tag) {
     stage = 5;
     const AttnItem it = attn_item(p, pos);
     if (!it.valid) return true;
-    constexpr int NCH = HD / 8;        // 16-byte K chunks per row
-    constexpr int DQ = HD / 4;         // dim quads per head
+    constexpr int QS = HD + 8;                  // halfs per Q tile row
+    constexpr int PSW = kAttnBlock + 8;         // halfs per P tile row
+    constexpr int KT = HD / 16;                 // k-steps of the score mma
+    constexpr int DTW = HD / 8 / kConsumerWarps;  // 8-dim output tiles per warp
     const int G = p.G;
-    const int QST = G * 8 + 4;         // floats per q chunk row (padded)
     const int j = it.j;
-    float* qc = sm_xs(p);              // [NCH][QST]: q chunk c of head g at c*QST + g*8
-    float* sc = qc + NCH * QST;        // [G][kAttnBlock]
-    float* kn = sc + G * kAttnBlock;
-    float* vn = kn + HD;
-    float* orun = vn + HD;
-    float* mrun = orun + G * HD;
-    float* lrun = mrun + kMaxGroup;
-    float* alpha = lrun + kMaxGroup;
+    const AttnSmem<HD> a(p);
     const float scale = 1.0f / sqrtf((float)HD);
     const long long c0 = clock64();
-    // q (tagged), scaled, stored chunk-major
     bool bad = false;
+    // Q rows >= G and the whole P tile start at zero (those rows stay zero)
+    for (int e = tid; e < (16 - G) * QS; e += kConsumerThreads) {
+      a.qhi[G * QS + e] = __float2half_rn(0.f);
+      a.qlo[G * QS + e] = __float2half_rn(0.f);
+    }
+    for (int e = tid; e < 16 * PSW / 2; e += kConsumerThreads)
+      reinterpret_cast<uint32_t*>(a.ps)[e] = 0u;
+    // q (tagged), scaled, as fp16 hi + lo
     {
       const u64* src = p.qbuf + (size_t)j * G * HD;
       const int n2 = G * HD / 2;
@@ -963,172 +1023,150 @@ struct Consumer {
         for (int b = 0; b < NB; ++b) {
           if (k2[b] < n2) {
             const int e = 2 * k2[b], g = e / HD, d = e - g * HD;
-            qc[(d >> 3) * QST + g * 8 + (d & 7)] = __uint_as_float((unsigned)v[b].x) * scale;
-            qc[(d >> 3) * QST + g * 8 + (d & 7) + 1] = __uint_as_float((unsigned)v[b].y) * scale;
+            const float x0 = __uint_as_float((unsigned)v[b].x) * scale;
+            const float x1 = __uint_as_float((unsigned)v[b].y) * scale;
+            const __half h0 = __float2half_rn(x0), h1 = __float2half_rn(x1);
+            *reinterpret_cast<__half2*>(a.qhi + g * QS + d) = __halves2half2(h0, h1);
+            *reinterpret_cast<__half2*>(a.qlo + g * QS + d) = __halves2half2(
+                __float2half_rn(x0 - __half2float(h0)), __float2half_rn(x1 - __half2float(h1)));
           }
         }
       }
     }
     if (it.t1 > pos && !bad) {
-      bad = !load_pairs(p.kvnew + j * HD, tag, HD / 2, kn, 1.0f, 21) ||
-            !load_pairs(p.kvnew + p.KV * HD + j * HD, tag, HD / 2, vn, 1.0f, 22);
+      bad = !load_pairs(p.kvnew + j * HD, tag, HD / 2, a.kn, 1.0f, 21) ||
+            !load_pairs(p.kvnew + p.KV * HD + j * HD, tag, HD / 2, a.vn, 1.0f, 22);
     }
-    for (int e = tid; e < G * HD; e += kConsumerThreads) orun[e] = 0.f;
     if (tid < kMaxGroup) {
-      mrun[tid] = -INFINITY;
-      lrun[tid] = 0.f;
+      a.mrun[tid] = -INFINITY;
+      a.lrun[tid] = 0.f;
     }
     if (dev::consumer_sync_or(bad)) return false;
     if (tid == 0) t_sync += clock64() - c0;
     trace(10);
 
+    const int gid = lane >> 2, tig = lane & 3;
+    // A fragments of q come from the hi / lo tiles (rows gid are heads,
+    // rows gid + 8 zero padding)
+    const __half* qh = a.qhi + gid * QS + tig * 2;
+    const __half* ql = a.qlo + gid * QS + tig * 2;
+    float oacc[DTW][4];
+#pragma unroll
+    for (int dt = 0; dt < DTW; ++dt) oacc[dt][0] = oacc[dt][1] = oacc[dt][2] = oacc[dt][3] = 0.f;
+
     const unsigned char* ring = sm_ring(p);
+    const int RS = attn_row_stride(p);
+    const int RSH = RS / 2;
     const int tb = attn_block(p);
-    const int g_pv = tid / DQ, dq = tid - (tid / DQ) * DQ;   // P.V thread role
     for (int b0 = it.t0; b0 < it.t1; b0 += tb) {
       const int nb = min(it.t1, b0 + tb) - b0;
-      const int nc = min(b0 + nb, pos) - b0;    // rows that came through the ring
+      const int nc = max(0, min(b0 + nb, pos) - b0);   // rows that came through the ring
+      const int nbp = (nb + 15) & ~15;
+      const uint32_t sz = (uint32_t)(nbp * RS);
       uint32_t offk = 0, offv = 0;
-      bool badc = false;
-      if (nc > 0) {
-        const uint32_t sz = (uint32_t)(nc * HD * 2);
-        if (!wait_chunk(sz, offk)) badc = true;
-        if (!wait_chunk(sz, offv)) badc = true;
-      }
+      bool badc = !wait_chunk(sz, offk);
+      badc = !wait_chunk(sz, offv) || badc;
       if (b0 == it.t0) trace(14);
+      __half* Kt = reinterpret_cast<__half*>(sm_ring_w(p) + offk);
+      __half* Vt = reinterpret_cast<__half*>(sm_ring_w(p) + offv);
       if (!badc) {
-        // threads per position: 4, 2 or 1
-        const int lp = nb <= kConsumerThreads / 4 ? 2 : nb <= kConsumerThreads / 2 ? 1 : 0;
-        const int P = 1 << lp;
-        const int cper = NCH >> lp;                    // chunks per thread
-        const uint4* Krows = reinterpret_cast<const uint4*>(ring + offk);
-        for (int base = 0; base < nb * P; base += kConsumerThreads) {
-          const int e = base + tid;
-          const int t = e >> lp, part = e & (P - 1);
-          float sg[kMaxGroup];
-#pragma unroll
-          for (int g = 0; g < kMaxGroup; ++g) sg[g] = 0.f;
-          if (t < nb) {
-            const bool cur = t >= nc;
-            for (int i = 0; i < cper; ++i) {
-              const int c = (part + P * (i + t)) & (NCH - 1);
-              float kf[8];
-              if (!cur) {
-                const uint4 kv = Krows[(size_t)t * NCH + c];
-                const float2 a = __half22float2(*reinterpret_cast<const __half2*>(&kv.x));
-                const float2 b = __half22float2(*reinterpret_cast<const __half2*>(&kv.y));
-                const float2 cc = __half22float2(*reinterpret_cast<const __half2*>(&kv.z));
-                const float2 d = __half22float2(*reinterpret_cast<const __half2*>(&kv.w));
-                kf[0] = a.x; kf[1] = a.y; kf[2] = b.x; kf[3] = b.y;
-                kf[4] = cc.x; kf[5] = cc.y; kf[6] = d.x; kf[7] = d.y;
-              } else {
-#pragma unroll
-                for (int q = 0; q < 8; ++q) kf[q] = kn[c * 8 + q];
-              }
-              const float* qrow = qc + c * QST;
-#pragma unroll
-              for (int g = 0; g < kMaxGroup; ++g) {
-                if (g < G) {
-                  const float4 qa = *reinterpret_cast<const float4*>(qrow + g * 8);
-                  const float4 qb = *reinterpret_cast<const float4*>(qrow + g * 8 + 4);
-                  float s2 = sg[g];
-                  s2 = fmaf(qa.x, kf[0], s2); s2 = fmaf(qa.y, kf[1], s2);
-                  s2 = fmaf(qa.z, kf[2], s2); s2 = fmaf(qa.w, kf[3], s2);
-                  s2 = fmaf(qb.x, kf[4], s2); s2 = fmaf(qb.y, kf[5], s2);
-                  s2 = fmaf(qb.z, kf[6], s2); s2 = fmaf(qb.w, kf[7], s2);
-                  sg[g] = s2;
-                }
-              }
-            }
-          }
-          // sum the P parts of a position (adjacent lanes)
-#pragma unroll
-          for (int g = 0; g < kMaxGroup; ++g) {
-            if (g < G) {
-              float v = sg[g];
-              if (lp >= 2) v += __shfl_xor_sync(0xffffffffu, v, 2);
-              if (lp >= 1) v += __shfl_xor_sync(0xffffffffu, v, 1);
-              if (t < nb && part == 0) sc[g * kAttnBlock + t] = v;
-            }
-          }
+        // row nc: the current position (when in this block); rows up to nbp: zero
+        for (int e = tid; e < (nbp - nc) * HD; e += kConsumerThreads) {
+          const int r = nc + e / HD, d = e - (e / HD) * HD;
+          const bool cur = r < nb;
+          Kt[r * RSH + d] = __float2half_rn(cur ? a.kn[d] : 0.f);
+          Vt[r * RSH + d] = __float2half_rn(cur ? a.vn[d] : 0.f);
         }
       }
       if (dev::consumer_sync_or(badc)) return false;
+      // scores
+      for (int nt = warp; nt < nbp / 8; nt += kConsumerWarps) {
+        float c[4] = {0.f, 0.f, 0.f, 0.f};
+        const unsigned char* krow = ring + offk + (nt * 8 + gid) * RS + tig * 4;
+#pragma unroll
+        for (int ks = 0; ks < KT; ++ks) {
+          const uint32_t kb0 = *reinterpret_cast<const uint32_t*>(krow + ks * 32);
+          const uint32_t kb1 = *reinterpret_cast<const uint32_t*>(krow + ks * 32 + 16);
+          dev::mma_16816(c, *reinterpret_cast<const uint32_t*>(qh + ks * 16), 0u,
+                         *reinterpret_cast<const uint32_t*>(qh + ks * 16 + 8), 0u, kb0, kb1);
+          dev::mma_16816(c, *reinterpret_cast<const uint32_t*>(ql + ks * 16), 0u,
+                         *reinterpret_cast<const uint32_t*>(ql + ks * 16 + 8), 0u, kb0, kb1);
+        }
+        if (gid < G) {
+          const int t = nt * 8 + 2 * tig;
+          a.sc[gid * kAttnBlock + t] = t < nb ? c[0] : -INFINITY;
+          a.sc[gid * kAttnBlock + t + 1] = t + 1 < nb ? c[1] : -INFINITY;
+        }
+      }
+      dev::consumer_sync();
       // online softmax over the block: warp g owns head g
       if (warp < G) {
-        float* row = sc + warp * kAttnBlock;
+        const float* row = a.sc + warp * kAttnBlock;
+        __half* prow = a.ps + warp * PSW;
         float mx = -INFINITY;
-        for (int t = lane; t < nb; t += 32) mx = fmaxf(mx, row[t]);
+        for (int t = lane; t < nbp; t += 32) mx = fmaxf(mx, row[t]);
         mx = dev::warp_max(mx);
-        const float mold = mrun[warp];
+        const float mold = a.mrun[warp];
         const float mnew = fmaxf(mold, mx);
         float sum = 0.f;
-        for (int t = lane; t < nb; t += 32) {
-          const float e = expf(row[t] - mnew);
-          row[t] = e;
-          sum += e;
+        for (int t = lane; t < nbp; t += 32) {
+          const __half e = __float2half_rn(expf(row[t] - mnew));
+          prow[t] = e;
+          sum += __half2float(e);
         }
         sum = dev::warp_sum(sum);
         if (lane == 0) {
-          const float a = expf(mold - mnew);
-          alpha[warp] = a;
-          lrun[warp] = lrun[warp] * a + sum;
-          mrun[warp] = mnew;
+          const float al = expf(mold - mnew);
+          a.alpha[warp] = al;
+          a.lrun[warp] = a.lrun[warp] * al + sum;
+          a.mrun[warp] = mnew;
         }
       }
       dev::consumer_sync();
       if (b0 == it.t0) trace(15);
-      if (g_pv < G) {
-        const uint2* Vrows = reinterpret_cast<const uint2*>(ring + offv);
-        const float* pr = sc + g_pv * kAttnBlock;
-        float4 acc[4];
+      // P.V into the running output (rows gid < G are heads)
+      {
+        const float al = gid < G ? a.alpha[gid] : 0.f;
 #pragma unroll
-        for (int u = 0; u < 4; ++u) acc[u] = make_float4(0.f, 0.f, 0.f, 0.f);
-        int t = 0;
-        for (; t + 4 <= nc; t += 4) {
-#pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const uint2 raw = Vrows[(size_t)(t + u) * DQ + dq];
-            const float2 a = __half22float2(*reinterpret_cast<const __half2*>(&raw.x));
-            const float2 b = __half22float2(*reinterpret_cast<const __half2*>(&raw.y));
-            const float w = pr[t + u];
-            acc[u].x = fmaf(w, a.x, acc[u].x);
-            acc[u].y = fmaf(w, a.y, acc[u].y);
-            acc[u].z = fmaf(w, b.x, acc[u].z);
-            acc[u].w = fmaf(w, b.y, acc[u].w);
-          }
+        for (int dt = 0; dt < DTW; ++dt) {
+          oacc[dt][0] *= al;
+          oacc[dt][1] *= al;
         }
-        for (; t < nb; ++t) {
-          float4 v;
-          if (t < nc) {
-            const uint2 raw = Vrows[(size_t)t * DQ + dq];
-            const float2 a = __half22float2(*reinterpret_cast<const __half2*>(&raw.x));
-            const float2 b = __half22float2(*reinterpret_cast<const __half2*>(&raw.y));
-            v = make_float4(a.x, a.y, b.x, b.y);
+        const int d0 = warp * 8 * DTW;
+        const int m = lane >> 3, r8 = lane & 7;
+        const uint32_t vrow = sm_ring_s(p) + offv + (uint32_t)(((m & 1) * 8 + r8) * RS) +
+                              (uint32_t)((d0 + (m >> 1) * 8) * 2);
+        for (int kk = 0; kk < nbp / 16; ++kk) {
+          const __half* pr = a.ps + gid * PSW + kk * 16 + tig * 2;
+          const uint32_t pa0 = *reinterpret_cast<const uint32_t*>(pr);
+          const uint32_t pa2 = *reinterpret_cast<const uint32_t*>(pr + 8);
+          const uint32_t va = vrow + (uint32_t)(kk * 16 * RS);
+          if constexpr (DTW == 2) {
+            uint32_t v0, v1, v2, v3;
+            dev::ldmatrix_x4_trans(va, v0, v1, v2, v3);
+            dev::mma_16816(oacc[0], pa0, 0u, pa2, 0u, v0, v1);
+            dev::mma_16816(oacc[DTW - 1], pa0, 0u, pa2, 0u, v2, v3);
           } else {
-            v = *reinterpret_cast<const float4*>(vn + dq * 4);
+            uint32_t v0, v1;
+            dev::ldmatrix_x2_trans(va, v0, v1);
+            dev::mma_16816(oacc[0], pa0, 0u, pa2, 0u, v0, v1);
           }
-          const float w = pr[t];
-          acc[0].x = fmaf(w, v.x, acc[0].x);
-          acc[0].y = fmaf(w, v.y, acc[0].y);
-          acc[0].z = fmaf(w, v.z, acc[0].z);
-          acc[0].w = fmaf(w, v.w, acc[0].w);
         }
-        float4* o = reinterpret_cast<float4*>(orun + g_pv * HD + dq * 4);
-        const float a = alpha[g_pv];
-        float4 cur = *o;
-        cur.x = fmaf(cur.x, a, (acc[0].x + acc[1].x) + (acc[2].x + acc[3].x));
-        cur.y = fmaf(cur.y, a, (acc[0].y + acc[1].y) + (acc[2].y + acc[3].y));
-        cur.z = fmaf(cur.z, a, (acc[0].z + acc[1].z) + (acc[2].z + acc[3].z));
-        cur.w = fmaf(cur.w, a, (acc[0].w + acc[1].w) + (acc[2].w + acc[3].w));
-        *o = cur;
       }
       dev::consumer_sync();
-      if (nc > 0) {
-        release_chunk();
-        release_chunk();
+      release_chunk();
+      release_chunk();
+    }
+    // running output of heads gid < G to shared memory
+    if (gid < G) {
+#pragma unroll
+      for (int dt = 0; dt < DTW; ++dt) {
+        const int d = warp * 8 * DTW + dt * 8 + 2 * tig;
+        a.orun[gid * HD + d] = oacc[dt][0];
+        a.orun[gid * HD + d + 1] = oacc[dt][1];
       }
     }
+    dev::consumer_sync();
     trace(11);
     // publish this item's partial: per head a row [m, l, -, -, o[HD]] of
     // HD + 4 floats (16-byte aligned rows; o unnormalised)
@@ -1137,9 +1175,10 @@ struct Consumer {
     for (int e = tid; e < G * HD / 4; e += kConsumerThreads) {
       const int g = e / (HD / 4), d4 = e - g * (HD / 4);
       *reinterpret_cast<float4*>(part + g * PST + 4 + 4 * d4) =
-          *reinterpret_cast<const float4*>(orun + g * HD + 4 * d4);
+          *reinterpret_cast<const float4*>(a.orun + g * HD + 4 * d4);
     }
-    if (tid < G) *reinterpret_cast<float2*>(part + tid * PST) = make_float2(mrun[tid], lrun[tid]);
+    if (tid < G)
+      *reinterpret_cast<float2*>(part + tid * PST) = make_float2(a.mrun[tid], a.lrun[tid]);
     dev::consumer_sync();
     const int nsplit = it.nsplit;
     if (tid == 0) {

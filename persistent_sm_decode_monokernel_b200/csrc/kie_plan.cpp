@@ -82,7 +82,8 @@ std::vector<int2> partition(const Shape& s, int grid, int stage) {
 
 int attn_smem_bytes(int G, int hd) {
   int b = 0;
-  b += (hd / 8) * (G * 8 + 4) * 4;   // q, chunk-major with padded rows
+  b += 2 * 16 * (hd + 8) * 2;        // q as fp16 hi and lo tiles (16 padded rows)
+  b += 16 * (kAttnBlock + 8) * 2;    // P tile, fp16
   b += std::max(G * kAttnBlock, 3 * kMaxSplitCombine * kMaxGroup) * 4;  // scores / combine
   b += 2 * hd * 4;                   // current position's k and v
   b += G * hd * 4;                   // running output
