@@ -209,12 +209,15 @@ KIE_API kie_status kie_set_logits_capture(kie_ctx *ctx, float *dev_logits,
  * %globaltimer stamps (ns) to dev_buf, a device buffer of `capacity` u64
  * owned by the caller; cta = -1 traces every CTA, laid out
  * [step][cta][slot] (grid CTAs per step, see kie_get_stats).  Per step and
- * CTA it writes n_layers*16 + 4 slots: for each
+ * CTA it writes n_layers*24 + 4 slots: for each
  * layer QKV begin, QKV input ready, QKV done, attention done, O input
  * ready, O done, gate/up input ready, gate/up done, down input ready, down
  * done, and (CTAs with attention work) q ready, attention math done,
- * partial published, combine done (slots 10-13; 14-15 unused); then
- * LM-head begin, input ready, GEMV done, pick known.  Steps beyond the
+ * partial published, combine done, first K/V tile landed, first block's
+ * softmax done (slots 10-15); slots 16-19 and 21: ns the first consumer
+ * warp waited for streamed chunks in QKV, O, gate/up, down and attention
+ * (durations, not stamps); then LM-head begin, input ready, GEMV done,
+ * pick known.  Steps beyond the
  * capacity are not traced.  NULL turns tracing off. */
 KIE_API kie_status kie_set_trace(kie_ctx *ctx, uint64_t *dev_buf, int32_t capacity, int32_t cta);
 

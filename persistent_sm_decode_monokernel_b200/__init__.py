@@ -17,7 +17,9 @@ from ._kie import (KieError, kie_check_desc, kie_create, kie_decode, kie_decode_
                    kie_plan_units, kie_prefill, kie_rewind, kie_set_logits_capture,
                    kie_set_option, kie_set_trace, load_library, make_desc)
 
-__all__ = ["Session", "KieError", "load_library", "make_desc", "upload_weights"]
+TRACE_PER_LAYER = 24   # trace slots per layer (kie.h, kie_set_trace)
+
+__all__ = ["TRACE_PER_LAYER", "Session", "KieError", "load_library", "make_desc", "upload_weights"]
 
 
 def upload_weights(host: Mapping[str, np.ndarray], device="cuda"):
@@ -83,10 +85,10 @@ class Session:
 
     def trace(self, steps: int, cta: int = 0):
         """Turns the stage trace on for `steps` steps of CTA `cta`; returns the
-        [steps, n_layers*16 + 4] int64 device buffer it fills.  cta=-1 traces
-        every CTA into a [steps, grid, n_layers*16 + 4] buffer."""
+        [steps, n_layers*24 + 4] int64 device buffer it fills.  cta=-1 traces
+        every CTA into a [steps, grid, n_layers*24 + 4] buffer."""
         import torch
-        per = self.shape.n_layers * 16 + 4
+        per = self.shape.n_layers * TRACE_PER_LAYER + 4
         shape = (steps, per) if cta >= 0 else (steps, self.stats()["grid"], per)
         self._trace = torch.zeros(shape, dtype=torch.int64, device="cuda")
         kie_set_trace(self.ctx, self._trace, self._trace.numel(), cta)

@@ -516,10 +516,12 @@ struct Consumer {
   uint32_t crel;   // next chunk to release (chunks are released in order)
   uint32_t cend;   // ring read position (mirrors the producer's placement)
   long long t_sync, t_stream;
+  long long w_stage;       // ns warp 0 waited for streamed chunks in the current stage (trace)
   int step, layer, stage;  // for error reports
 
   __device__ explicit Consumer(const MonoParams& pp)
-      : p(pp), cidx(0), crel(0), cend(0), t_sync(0), t_stream(0), step(0), layer(0), stage(0) {
+      : p(pp), cidx(0), crel(0), cend(0), t_sync(0), t_stream(0), w_stage(0), step(0), layer(0),
+        stage(0) {
     tid = threadIdx.x;
     warp = tid >> 5;
     lane = tid & 31;
@@ -528,15 +530,24 @@ struct Consumer {
   // Stage-boundary timestamps of one CTA (measurement): per step
   // 10 per layer (QKV begin/loaded/done, attention done, O loaded/done,
   // gate-up loaded/done, down loaded/done) + 4 for the LM head.
-  __device__ __forceinline__ void trace(int ev) const {
+  __device__ __forceinline__ void trace_put(int ev, unsigned long long v) const {
     if (p.trace && tid == 0 && (p.trace_cta < 0 || (int)blockIdx.x == p.trace_cta) &&
         step < p.trace_steps) {
       const int per = p.L * kTracePerLayer + 4;
       const int row = p.trace_cta < 0 ? step * p.grid + (int)blockIdx.x : step;
       const int idx = row * per + (layer < p.L ? layer * kTracePerLayer : p.L * kTracePerLayer) + ev;
-      p.trace[idx] = p.trace_clock ? (unsigned long long)clock64()
-                                   : (unsigned long long)dev::globaltimer();
+      p.trace[idx] = v;
     }
+  }
+  __device__ __forceinline__ void trace(int ev) const {
+    if (p.trace)
+      trace_put(ev, p.trace_clock ? (unsigned long long)clock64()
+                                  : (unsigned long long)dev::globaltimer());
+  }
+  // Stream wait of the stage just finished (slots 16 + stage), then reset.
+  __device__ __forceinline__ void trace_stream_wait(int st) {
+    if (p.trace) trace_put(16 + st, (unsigned long long)w_stage);
+    w_stage = 0;
   }
   __device__ __forceinline__ void trace_loaded() const {
     switch (stage) {
@@ -578,7 +589,10 @@ struct Consumer {
         }
       }
     }
-    if (tid == 0) t_stream += clock64() - c0;
+    if (tid == 0) {
+      t_stream += clock64() - c0;
+      if (p.trace) w_stage += dev::globaltimer() - t0;
+    }
     return ok;
   }
   // Releases the oldest chunk this warp waited for and has not released.
@@ -1412,14 +1426,19 @@ struct Consumer {
         trace(0);
         ok = stage_qkv(w, tok, pos, tag);
         trace(2);
+        trace_stream_wait(ST_QKV);
         ok = ok && stage_attn<HD>(pos, tag);
         trace(3);
+        trace_stream_wait(5);
         ok = ok && stage_o(w, tok, tag);
         trace(5);
+        trace_stream_wait(ST_O);
         ok = ok && stage_gu(w, tag);
         trace(7);
+        trace_stream_wait(ST_GU);
         ok = ok && stage_down(w, tag, tag + 1u);
         trace(9);
+        trace_stream_wait(ST_DOWN);
       }
       if (!ok) break;
       layer = p.L;
@@ -1428,6 +1447,7 @@ struct Consumer {
       trace(0);
       const bool lm_ok = stage_lm(pick, i - p.lm_from, epoch_of(p, i, p.L), &next);
       trace(3);
+      w_stage = 0;
       if (!lm_ok) {
         ok = false;
         break;
@@ -1467,12 +1487,14 @@ __global__ void __launch_bounds__(kThreads, 1) kie_monokernel(const __grid_const
   }
   __syncthreads();
   if (threadIdx.x >= kConsumerThreads) {
+    dev::regs_dec<kRegsProducer>();
     if (threadIdx.x == kConsumerThreads) {
       Producer prod(p);
       prod.run();
     }
     return;
   }
+  dev::regs_inc<kRegsConsumer>();
   Consumer c(p);
   c.run<HD>();
 }
@@ -1493,6 +1515,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   __syncthreads();
   if (threadIdx.x >= kConsumerThreads) {
+    dev::regs_dec<kRegsProducer>();
     if (threadIdx.x == kConsumerThreads) {
       Producer prod(p);
       bool ok = true;
@@ -1505,6 +1528,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     return;
   }
+  dev::regs_inc<kRegsConsumer>();
   Consumer c(p);
   c.gemv_bench(mode, x, y, iters);
 }

@@ -12,7 +12,17 @@ namespace kie {
 enum Stage : int { ST_QKV = 0, ST_O = 1, ST_GU = 2, ST_DOWN = 3, ST_LM = 4, N_STAGES = 5 };
 
 constexpr int kConsumerWarps = 8;            // warps that compute
-constexpr int kThreads = (kConsumerWarps + 1) * 32;  // + one producer warp
+// + one producer warpgroup (only its first lane works): warpgroup-granular
+// register split, see kRegsConsumer / kRegsProducer
+constexpr int kThreads = (kConsumerWarps + 4) * 32;
+// Registers per thread after the split: the launch gives every thread 168
+// (12 warps fit one SM); the producer warpgroup gives up to kRegsProducer
+// and the consumer warpgroups take kRegsConsumer:
+// 8 * kRegsConsumer + 4 * kRegsProducer <= 12 * 168.
+constexpr int kRegsLaunch = 168;
+constexpr int kRegsConsumer = 224;
+constexpr int kRegsProducer = 40;
+static_assert(8 * kRegsConsumer + 4 * kRegsProducer <= 12 * kRegsLaunch, "register split");
 constexpr int kConsumerThreads = kConsumerWarps * 32;
 constexpr int kGroupRows = 16;              // rows streamed together (two per warp)
 constexpr int kPieceElems = 256;             // one warp pass: 32 lanes x 8 fp16
@@ -26,7 +36,7 @@ constexpr int kPollBackoffNs = 128;          // sleep between re-polls of tagged
 // producer slot-wait cycles, steps done, spare
 constexpr int kStatsPerCta = 8;
 // stage-trace stamps per layer (the LM head adds 4 per step)
-constexpr int kTracePerLayer = 16;
+constexpr int kTracePerLayer = 24;
 
 // Device status word block (library scratch, zeroed before each launch).
 struct DevStatus {
