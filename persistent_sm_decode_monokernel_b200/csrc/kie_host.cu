@@ -555,7 +555,7 @@ kie_status kie_gemv_f16(const void* W, const float* x, float* y, int32_t N, int3
   L.xs_bytes = (K * 4 + 127) / 128 * 128;
   L.rowacc_rows = maxrows;
   L.resid_rows = 0;
-  const int fixed = 256 + L.xs_bytes + (maxrows * 4 + 127) / 128 * 128 + 256;
+  const int fixed = 256 + L.xs_bytes + (maxrows * 4 + 127) / 128 * 128 + kie::kEngineMisc;
   const int ring = (smem_optin - fixed) / 512 * 512;
   if (ring < 2 * chunk_bytes) return KIE_ERR_UNSUPPORTED;
   L.ring_off = 0;
@@ -563,7 +563,7 @@ kie_status kie_gemv_f16(const void* W, const float* x, float* y, int32_t N, int3
   L.xs_off = L.bar_off + 256;
   L.rowacc_off = L.xs_off + L.xs_bytes;
   L.misc_off = L.rowacc_off + (maxrows * 4 + 127) / 128 * 128;
-  L.total = L.misc_off + 256;
+  L.total = L.misc_off + kie::kEngineMisc;
 
   int2* d_ranges = nullptr;
   DevStatus* d_status = nullptr;

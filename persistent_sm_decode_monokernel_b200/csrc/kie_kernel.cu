@@ -80,6 +80,20 @@ __device__ __forceinline__ float* sm_res_attn(const MonoParams& p) { return sm_m
 __device__ __forceinline__ float* sm_res_ffn(const MonoParams& p) {
   return sm_misc(p) + 64 + p.sm.resid_rows;
 }
+
+// This CTA's GEMV work in one stage, computed once per launch: kGroupRows
+// row groups and the k-chunking of a full group and of the last group.
+struct StagePlan {
+  int rows, kp;          // rows of the CTA in the stage, 512-byte pieces per row
+  int nfull, tail;       // full groups; rows of the last, partial group (0: none)
+  int f_nk, f_base, f_rem;  // chunking of a full group (see Chunking)
+  int t_nk, t_base, t_rem;  // chunking of the partial group
+  int t_lw;              // partial group of <= kConsumerWarps rows: log2 warps per row
+  int pad[5];
+};
+__device__ __forceinline__ StagePlan* sm_plan(const MonoParams& p) {
+  return reinterpret_cast<StagePlan*>(sm_misc(p) + 64 + 2 * p.sm.resid_rows);
+}
 __device__ __forceinline__ const unsigned char* sm_ring(const MonoParams& p) {
   return kie_smem + p.sm.ring_off;
 }
@@ -564,6 +578,33 @@ struct Consumer {
            p.fault_stage == st;
   }
 
+  // Slow path of a chunk wait: bounded spin on the full barrier.
+  __device__ __noinline__ bool wait_slow(uint32_t bar, uint32_t par) {
+    const long long c0 = clock64();
+    const long long t0 = dev::globaltimer();
+    bool ok = true;
+    for (unsigned it = 1;; ++it) {
+      if (dev::mbar_try_wait(bar, par)) break;
+      if ((it & 15u) == 0u) {
+        if (sm_flags(p)[F_ABORT]) {
+          ok = false;
+          break;
+        }
+        if (dev::globaltimer() - t0 > p.timeout_ns) {
+          raise_error(p, DEV_TIMEOUT, step, layer, stage, 3);
+          sm_flags(p)[F_ABORT] = 1;
+          ok = false;
+          break;
+        }
+      }
+    }
+    if (tid == 0) {
+      t_stream += clock64() - c0;
+      if (p.trace) w_stage += dev::globaltimer() - t0;
+    }
+    return ok;
+  }
+
   // ---- ring: waits for the next chunk (sz bytes) and returns its offset
   __device__ __forceinline__ bool wait_chunk(uint32_t sz, uint32_t& off) {
     off = ring_place(cend, sz, (uint32_t)p.ring_bytes);
@@ -742,13 +783,8 @@ struct Consumer {
     return true;
   }
 
-  // ---- GEMV of this CTA's rows of a stage into rowacc (raw dot products).
-  // A group of up to 16 rows streams as k-chunks.  In a full group warp w
-  // owns rows w and w+8 for all of the group's chunks (one activation load
-  // serves two rows) and keeps its partial sums in registers.  A group of
-  // at most 8 rows gives each row 8/rg (power of two) warps that split its
-  // pieces and are summed in a fixed order, so results do not depend on
-  // timing.
+  // ---- GEMV arithmetic: lane l of a 512-byte piece multiplies 8 fp16
+  // weights by the 8 fp16 activations it shares with the other row.
   __device__ __forceinline__ static void dot_piece(const uint4& w, const uint4& x, float (&c)[8]) {
     dev::fma_f16x2_f32(c[0], c[1], w.x, x.x);
     dev::fma_f16x2_f32(c[2], c[3], w.y, x.y);
@@ -759,92 +795,149 @@ struct Consumer {
     return ((c[0] + c[1]) + (c[2] + c[3])) + ((c[4] + c[5]) + (c[6] + c[7]));
   }
 
-  __device__ __noinline__ bool gemv(int st, int ub, int ue) {
-    const int R = range_rows(p, st, ub, ue);
-    const int K = stage_k(p, st);
-    const int kp = K / kPieceElems;
+  // Fills the stage plans (threads 0..N_STAGES-1; the caller synchronises).
+  __device__ void make_plans() {
+    if (tid < N_STAGES) {
+      const int st = tid;
+      const int2 r = p.ranges[st * p.grid + blockIdx.x];
+      StagePlan pl{};
+      pl.rows = range_rows(p, st, r.x, r.y);
+      pl.kp = stage_k(p, st) / kPieceElems;
+      pl.nfull = pl.rows / kGroupRows;
+      pl.tail = pl.rows - pl.nfull * kGroupRows;
+      const Chunking f = chunking(kGroupRows, pl.kp, p.chunk_bytes);
+      pl.f_nk = f.nk;
+      pl.f_base = f.base;
+      pl.f_rem = f.rem;
+      if (pl.tail > 0) {
+        const Chunking t = chunking(pl.tail, pl.kp, p.chunk_bytes);
+        pl.t_nk = t.nk;
+        pl.t_base = t.base;
+        pl.t_rem = t.rem;
+        pl.t_lw = pl.tail == 1 ? 3 : pl.tail == 2 ? 2 : pl.tail <= 4 ? 1 : 0;
+      }
+      sm_plan(p)[st] = pl;
+    }
+  }
+
+  // GEMV of this CTA's rows of stage st: raw dot products, read back with
+  // row_result.  A group of up to 16 rows streams as k-chunks.  In a group
+  // of more than 8 rows warp w owns rows w and w+8 for all of the group's
+  // chunks (one activation load serves two rows) and keeps its partial sums
+  // in registers.  A last group of at most 8 rows gives each row 8/rg
+  // (power of two) warps that split its pieces; their partial sums are
+  // added in a fixed order by row_result, so results do not depend on
+  // timing.  Ring positions and the parameter block are held in registers
+  // for the whole stage; one barrier at the end.
+  __device__ __noinline__ bool gemv(int st) {
+    const MonoParams& p = this->p;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const StagePlan pl = sm_plan(p)[st];
     const unsigned char* ring = sm_ring(p);
     const uint4* xv = reinterpret_cast<const uint4*>(kie_smem + p.sm.xs_off) + lane;
     float* rowacc = sm_rowacc(p);
-    const Chunking chf = chunking(kGroupRows, kp, p.chunk_bytes);
+    const uint32_t ring_bytes = (uint32_t)p.ring_bytes;
+    const uint32_t full_s = sm_full_s(p), empty_s = sm_empty_s(p);
+    uint32_t ci = cidx, cr = crel, ce = cend;
     bool bad = false;
-    for (int g0 = 0; g0 < R; g0 += kGroupRows) {
-      const int rg = min(kGroupRows, R - g0);
-      const Chunking ch = rg == kGroupRows ? chf : chunking(rg, kp, p.chunk_bytes);
-      if (rg > kConsumerWarps) {
-        // two rows per warp: w and w+8 (the second may be missing)
-        const bool two = warp + kConsumerWarps < rg;
-        float c0[8], c1[8];
+    auto wait = [&](uint32_t sz, uint32_t& off) -> bool {
+      off = ring_place(ce, sz, ring_bytes);
+      const uint32_t bar = full_s + 8 * (ci & (kRingBars - 1));
+      const uint32_t par = (ci / kRingBars) & 1u;
+      ++ci;
+      if (dev::mbar_test_wait(bar, par)) return true;
+      return wait_slow(bar, par);
+    };
+    auto release = [&]() {
+      __syncwarp();
+      if (lane == 0) dev::mbar_arrive(empty_s + 8 * (cr & (kRingBars - 1)));
+      ++cr;
+    };
+    // groups with two rows per warp (w and w+8; the second may be missing)
+    auto group2 = [&](int g0, int rg, int nk, int base, int rem) {
+      const bool two = warp + kConsumerWarps < rg;
+      float c0[8], c1[8];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) c0[i] = c1[i] = 0.f;
-        for (int kc = 0; kc < ch.nk; ++kc) {
-          const int n = ch.count(kc), p0 = ch.first(kc);
-          uint32_t off;
-          if (!wait_chunk((uint32_t)(rg * n * kPieceBytes), off) && !bad) bad = true;
-          if (!bad) {
-            const uint4* w0 =
-                reinterpret_cast<const uint4*>(ring + off + (size_t)warp * n * kPieceBytes) + lane;
-            const uint4* w1 = w0 + (size_t)kConsumerWarps * n * 32;
-            const uint4* x = xv + (size_t)p0 * 32;
-            if (two) {
+      for (int i = 0; i < 8; ++i) c0[i] = c1[i] = 0.f;
+      for (int kc = 0; kc < nk; ++kc) {
+        const int n = base + (kc < rem ? 1 : 0), p0 = kc * base + min(kc, rem);
+        uint32_t off;
+        if (!wait((uint32_t)(rg * n * kPieceBytes), off)) bad = true;
+        if (!bad) {
+          const uint4* w0 =
+              reinterpret_cast<const uint4*>(ring + off + (size_t)warp * n * kPieceBytes) + lane;
+          const uint4* w1 = w0 + (size_t)kConsumerWarps * n * 32;
+          const uint4* x = xv + (size_t)p0 * 32;
+          if (two) {
 #pragma unroll 4
-              for (int q = 0; q < n; ++q) {
-                const uint4 a = x[q * 32];
-                dot_piece(w0[q * 32], a, c0);
-                dot_piece(w1[q * 32], a, c1);
-              }
-            } else {
-#pragma unroll 4
-              for (int q = 0; q < n; ++q) dot_piece(w0[q * 32], x[q * 32], c0);
+            for (int q = 0; q < n; ++q) {
+              const uint4 a = x[q * 32];
+              dot_piece(w0[q * 32], a, c0);
+              dot_piece(w1[q * 32], a, c1);
             }
-          }
-          release_chunk();
-        }
-        const float s0 = dev::warp_sum(sum8(c0));
-        const float s1 = dev::warp_sum(sum8(c1));
-        if (lane == 0) {
-          rowacc[g0 + warp] = s0;
-          if (two) rowacc[g0 + warp + kConsumerWarps] = s1;
-        }
-      } else {
-        const int lw = rg == 1 ? 3 : rg == 2 ? 2 : rg <= 4 ? 1 : 0;   // log2(warps per row)
-        const int r = warp >> lw, part = warp & ((1 << lw) - 1);
-        const bool active = r < rg;
-        float c0[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) c0[i] = 0.f;
-        for (int kc = 0; kc < ch.nk; ++kc) {
-          const int n = ch.count(kc), p0 = ch.first(kc);
-          uint32_t off;
-          if (!wait_chunk((uint32_t)(rg * n * kPieceBytes), off) && !bad) bad = true;
-          if (active && !bad) {
-            const int pa = (part * n) >> lw, pb = ((part + 1) * n) >> lw;
-            const uint4* wr =
-                reinterpret_cast<const uint4*>(ring + off + (size_t)r * n * kPieceBytes) + lane;
-            const uint4* x = xv + (size_t)p0 * 32;
+          } else {
 #pragma unroll 4
-            for (int q = pa; q < pb; ++q) dot_piece(wr[q * 32], x[q * 32], c0);
-          }
-          release_chunk();
-        }
-        if (active) {
-          const float s = dev::warp_sum(sum8(c0));
-          if (lane == 0) {
-            if (lw == 0) rowacc[g0 + r] = s;
-            else sm_part(p)[warp] = s;
+            for (int q = 0; q < n; ++q) dot_piece(w0[q * 32], x[q * 32], c0);
           }
         }
-        if (lw > 0) {
-          dev::consumer_sync();
-          if (tid < rg) {
-            float s = 0.f;
-            for (int q = 0; q < (1 << lw); ++q) s += sm_part(p)[(tid << lw) + q];
-            rowacc[g0 + tid] = s;
-          }
+        release();
+      }
+      const float s0 = dev::warp_sum(sum8(c0));
+      const float s1 = dev::warp_sum(sum8(c1));
+      if (lane == 0) {
+        rowacc[g0 + warp] = s0;
+        if (two) rowacc[g0 + warp + kConsumerWarps] = s1;
+      }
+    };
+    for (int g = 0; g < pl.nfull; ++g) group2(g * kGroupRows, kGroupRows, pl.f_nk, pl.f_base, pl.f_rem);
+    const int tb = pl.nfull * kGroupRows;
+    if (pl.tail > kConsumerWarps) {
+      group2(tb, pl.tail, pl.t_nk, pl.t_base, pl.t_rem);
+    } else if (pl.tail > 0) {
+      const int lw = pl.t_lw, rg = pl.tail;
+      const int r = warp >> lw, part = warp & ((1 << lw) - 1);
+      const bool active = r < rg;
+      float c0[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) c0[i] = 0.f;
+      for (int kc = 0; kc < pl.t_nk; ++kc) {
+        const int n = pl.t_base + (kc < pl.t_rem ? 1 : 0), p0 = kc * pl.t_base + min(kc, pl.t_rem);
+        uint32_t off;
+        if (!wait((uint32_t)(rg * n * kPieceBytes), off)) bad = true;
+        if (active && !bad) {
+          const int pa = (part * n) >> lw, pb = ((part + 1) * n) >> lw;
+          const uint4* wr =
+              reinterpret_cast<const uint4*>(ring + off + (size_t)r * n * kPieceBytes) + lane;
+          const uint4* x = xv + (size_t)p0 * 32;
+#pragma unroll 4
+          for (int q = pa; q < pb; ++q) dot_piece(wr[q * 32], x[q * 32], c0);
+        }
+        release();
+      }
+      if (active) {
+        const float s = dev::warp_sum(sum8(c0));
+        if (lane == 0) {
+          if (lw == 0) rowacc[tb + r] = s;
+          else sm_part(p)[warp] = s;
         }
       }
     }
+    cidx = ci;
+    crel = cr;
+    cend = ce;
     return !dev::consumer_sync_or(bad);
+  }
+
+  // Raw dot product of row k (0-based within the CTA's rows) of the last gemv.
+  __device__ __forceinline__ float row_result(const StagePlan& pl, int k) const {
+    const int tb = pl.nfull * kGroupRows;
+    if (pl.tail > 0 && pl.t_lw > 0 && k >= tb) {
+      const int base = (k - tb) << pl.t_lw;
+      float s = 0.f;
+      for (int q = 0; q < (1 << pl.t_lw); ++q) s += sm_part(p)[base + q];
+      return s;
+    }
+    return sm_rowacc(p)[k];
   }
 
   __device__ __forceinline__ void put(u64* dst, unsigned tag, float v, bool skip) {
@@ -861,10 +954,11 @@ struct Consumer {
     const __half* emb = layer == 0 ? p.tok_emb + (size_t)tok * p.d : nullptr;
     if (r.y > r.x) {
       if (!load_vec(p.x_attn, tag, emb, p.d, w.attn_norm, ss, 10)) return false;
-      if (!gemv(ST_QKV, r.x, r.y)) return false;
+      if (!gemv(ST_QKV)) return false;
     } else {
       return true;
     }
+    const StagePlan pl = sm_plan(p)[ST_QKV];
     const float rs = 1.0f / sqrtf(ss / (float)p.d + p.eps);
     const int half = p.hd >> 1;
     const int nqp = p.H * half, np_all = qkv_pair_units(p);
@@ -876,7 +970,7 @@ struct Consumer {
     for (int u = r.x + tid; u < r.y; u += kConsumerThreads) {
       const int k = u - r.x;
       if (u < np_all) {
-        const float a = sm_rowacc(p)[2 * k] * rs, b = sm_rowacc(p)[2 * k + 1] * rs;
+        const float a = row_result(pl, 2 * k) * rs, b = row_result(pl, 2 * k + 1) * rs;
         const bool isq = u < nqp;
         const int uu = isq ? u : u - nqp;
         const int h = uu / half, i = uu - h * half;
@@ -897,7 +991,7 @@ struct Consumer {
       } else {
         const int vr = u - np_all;
         const int lr = 2 * np + (k - np);
-        const __half vh = __float2half_rn(sm_rowacc(p)[lr] * rs);
+        const __half vh = __float2half_rn(row_result(pl, lr) * rs);
         const int h = vr / p.hd, e = vr - h * p.hd;
         vbase[((size_t)h * p.max_seq + pos) * p.hd + e] = vh;
         put(p.kvnew + p.KV * p.hd + vr, tag, __half2float(vh), skip);
@@ -1213,12 +1307,13 @@ struct Consumer {
     if (r.y <= r.x) return true;
     float ss;
     if (!load_vec(p.obuf, tag, nullptr, p.H * p.hd, nullptr, ss, 30)) return false;
-    if (!gemv(ST_O, r.x, r.y)) return false;
+    if (!gemv(ST_O)) return false;
+    const StagePlan pl = sm_plan(p)[ST_O];
     const bool skip = fault_here(ST_O);
     for (int u = r.x + tid; u < r.y; u += kConsumerThreads) {
       const int k = u - r.x;
       const float res = layer == 0 ? __half2float(p.tok_emb[(size_t)tok * p.d + u]) : sm_res_attn(p)[k];
-      const float v = res + sm_rowacc(p)[k];
+      const float v = res + row_result(pl, k);
       sm_res_ffn(p)[k] = v;
       put(p.x_ffn + u, tag, v, skip);
     }
@@ -1232,12 +1327,13 @@ struct Consumer {
     if (r.y <= r.x) return true;
     float ss;
     if (!load_vec(p.x_ffn, tag, nullptr, p.d, w.ffn_norm, ss, 40)) return false;
-    if (!gemv(ST_GU, r.x, r.y)) return false;
+    if (!gemv(ST_GU)) return false;
+    const StagePlan pl = sm_plan(p)[ST_GU];
     const float rs = 1.0f / sqrtf(ss / (float)p.d + p.eps);
     const bool skip = fault_here(ST_GU);
     for (int u = r.x + tid; u < r.y; u += kConsumerThreads) {
       const int k = u - r.x;
-      const float g = sm_rowacc(p)[2 * k] * rs, up = sm_rowacc(p)[2 * k + 1] * rs;
+      const float g = row_result(pl, 2 * k) * rs, up = row_result(pl, 2 * k + 1) * rs;
       const float sg = g / (1.0f + expf(-g));
       put(p.hbuf + u, tag, sg * up, skip);
     }
@@ -1251,11 +1347,12 @@ struct Consumer {
     if (r.y <= r.x) return true;
     float ss;
     if (!load_vec(p.hbuf, tag, nullptr, p.F, nullptr, ss, 50)) return false;
-    if (!gemv(ST_DOWN, r.x, r.y)) return false;
+    if (!gemv(ST_DOWN)) return false;
+    const StagePlan pl = sm_plan(p)[ST_DOWN];
     const bool skip = fault_here(ST_DOWN);
     for (int u = r.x + tid; u < r.y; u += kConsumerThreads) {
       const int k = u - r.x;
-      const float v = sm_res_ffn(p)[k] + sm_rowacc(p)[k];
+      const float v = sm_res_ffn(p)[k] + row_result(pl, k);
       sm_res_attn(p)[k] = v;
       put(p.x_attn + u, tag_next, v, skip);
     }
@@ -1288,14 +1385,15 @@ struct Consumer {
     if (pick && r.y > r.x) {
       float ss;
       if (!load_vec(p.x_attn, tag, nullptr, p.d, p.final_norm, ss, 60)) return false;
-      if (!gemv(ST_LM, r.x, r.y)) return false;
+      if (!gemv(ST_LM)) return false;
+      const StagePlan pl = sm_plan(p)[ST_LM];
       trace(2);
       const float rs = 1.0f / sqrtf(ss / (float)p.d + p.eps);
       float* cap = (p.capture && step_row < p.capture_rows)
                        ? p.capture + (size_t)step_row * p.V
                        : nullptr;
       for (int u = r.x + tid; u < r.y; u += kConsumerThreads) {
-        const float v = sm_rowacc(p)[u - r.x] * rs;
+        const float v = row_result(pl, u - r.x) * rs;
         if (cap) cap[u] = v;
         if (better(v, u, best, bi)) {
           best = v;
@@ -1390,6 +1488,7 @@ struct Consumer {
   // Standalone GEMV engine run: y = W x over the LM-head stage's rows,
   // `iters` times (mode 0: stream the weights only, mode 1: full GEMV).
   __device__ void gemv_bench(int mode, const float* x, float* y, int iters) {
+    make_plans();
     const int2 r = p.ranges[ST_LM * p.grid + blockIdx.x];
     const int K = p.d;
     float acc = 0.f;
@@ -1400,9 +1499,9 @@ struct Consumer {
     dev::consumer_sync();
     bool ok = true;
     for (int it = 0; it < iters && ok; ++it)
-      ok = mode == 0 ? skip_stage(ST_LM, r.x, r.y) : gemv(ST_LM, r.x, r.y);
+      ok = mode == 0 ? skip_stage(ST_LM, r.x, r.y) : gemv(ST_LM);
     if (ok && mode == 1)
-      for (int u = r.x + tid; u < r.y; u += kConsumerThreads) y[u] = sm_rowacc(p)[u - r.x];
+      for (int u = r.x + tid; u < r.y; u += kConsumerThreads) y[u] = row_result(sm_plan(p)[ST_LM], u - r.x);
     if (tid == 0) {
       sm_flags(p)[F_STOP] = 1;
       u64* st = p.cta_stats + kStatsPerCta * blockIdx.x;
@@ -1412,6 +1511,8 @@ struct Consumer {
 
   template <int HD>
   __device__ void run() {
+    make_plans();
+    dev::consumer_sync();
     const long long c_begin = clock64();
     int tok = p.forced ? p.forced[0] : p.first_tok;
     int done = 0;

@@ -120,7 +120,7 @@ kie_status kie_gemv_f16_noalloc(const void* W, const float* x, float* y, int32_t
   L.rowacc_rows = maxrows;
   L.resid_rows = 0;
   const int rowacc_bytes = (maxrows * 4 + 127) / 128 * 128;
-  const int fixed = 256 + L.xs_bytes + rowacc_bytes + 256;
+  const int fixed = 256 + L.xs_bytes + rowacc_bytes + kie::kEngineMisc;
   const int ring = (smem_optin - fixed) / 512 * 512;
   if (ring < 2 * kChunkBytes) return KIE_ERR_UNSUPPORTED;
   L.ring_off = 0;
@@ -128,7 +128,7 @@ kie_status kie_gemv_f16_noalloc(const void* W, const float* x, float* y, int32_t
   L.xs_off = L.bar_off + 256;
   L.rowacc_off = L.xs_off + L.xs_bytes;
   L.misc_off = L.rowacc_off + rowacc_bytes;
-  L.total = L.misc_off + 256;
+  L.total = L.misc_off + kie::kEngineMisc;
 
   auto* d_status = reinterpret_cast<DevStatus*>(scratch + kOffStatus);
   auto* d_layer = reinterpret_cast<LayerW*>(scratch + kOffLayer);

@@ -37,6 +37,9 @@ constexpr int kPollBackoffNs = 128;          // sleep between re-polls of tagged
 constexpr int kStatsPerCta = 8;
 // stage-trace stamps per layer (the LM head adds 4 per step)
 constexpr int kTracePerLayer = 24;
+// Scratch words (reductions, flags) and the per-stage GEMV plans of the
+// standalone GEMV engine's shared memory (no residual rows there).
+constexpr int kEngineMisc = 640;
 
 // Device status word block (library scratch, zeroed before each launch).
 struct DevStatus {
