@@ -1004,7 +1004,7 @@ struct Consumer {
   // weights w_q = exp(m_q - M) / sum_q exp(m_q - M) l_q per head.
   // Warp g reads head g's (m, l) of every split at once (lane = split);
   // then each thread owns 4 output dims of one head and issues the loads of
-  // 8 splits before using any, so a combine costs a few L2 round trips.
+  // 16 splits before using any, so a combine costs a few L2 round trips.
   template <int HD>
   __device__ __noinline__ void attn_combine(int j, int nsplit, unsigned tag) {
     constexpr int PST = HD + 4;
@@ -1047,14 +1047,14 @@ struct Consumer {
       const int g = e / (HD / 4), d4 = e - g * (HD / 4);
       const float* src = base + (size_t)g * PST + 4 + 4 * d4;
       float4 O = make_float4(0.f, 0.f, 0.f, 0.f);
-      for (int q0 = 0; q0 < nsplit; q0 += 8) {
-        float4 v[8];
+      for (int q0 = 0; q0 < nsplit; q0 += 16) {
+        float4 v[16];
 #pragma unroll
-        for (int u = 0; u < 8; ++u)
+        for (int u = 0; u < 16; ++u)
           if (q0 + u < nsplit)
             v[u] = *reinterpret_cast<const float4*>(src + (size_t)(q0 + u) * G * PST);
 #pragma unroll
-        for (int u = 0; u < 8; ++u) {
+        for (int u = 0; u < 16; ++u) {
           if (q0 + u < nsplit) {
             const float wv = wq[(q0 + u) * G + g];
             O.x = fmaf(wv, v[u].x, O.x);
