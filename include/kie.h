@@ -34,8 +34,10 @@
  *       w_gate, w_up [ffn_dim][d_model]; w_down [d_model][ffn_dim].
  *     Every pointer must be device memory, 16-byte aligned.
  *   - The KV cache is one device buffer of kie_kv_cache_bytes() bytes,
- *     16-byte aligned, laid out fp16 [n_layers][2][n_kv_heads][max_seq][hd]
- *     (index 0 = K after RoPE, 1 = V).
+ *     16-byte aligned, laid out fp16 [n_layers][2][n_kv_heads][max_seq][hd + 8]
+ *     (index 0 = K after RoPE, 1 = V; the last 8 elements of each position's
+ *     row are padding, never read, so that consecutive rows copied into
+ *     shared memory fall in different banks).
  *   - The CALLER owns the weights and the KV cache.  kie_create copies the
  *     weight matrices (wq..w_down, lm_head) into a library-owned buffer laid
  *     out in the order each CTA streams them, so that every streamed chunk
@@ -155,7 +157,7 @@ typedef enum {
                                     0 = off, the default) */
 } kie_option;
 
-/* Bytes of the caller-provided KV cache: 2*n_layers*n_kv_heads*max_seq*head_dim*2.
+/* Bytes of the caller-provided KV cache: 2*n_layers*n_kv_heads*max_seq*(head_dim+8)*2.
  * Returns 0 for a NULL or invalid desc.  Host only. */
 KIE_API size_t kie_kv_cache_bytes(const kie_model_desc *desc);
 

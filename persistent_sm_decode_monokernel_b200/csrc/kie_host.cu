@@ -272,7 +272,8 @@ extern "C" {
 
 size_t kie_kv_cache_bytes(const kie_model_desc* d) {
   if (!d || kie_check_desc(d) != KIE_OK) return 0;
-  return (size_t)2 * d->n_layers * d->n_kv_heads * (size_t)d->max_seq * d->head_dim * 2;
+  return (size_t)2 * d->n_layers * d->n_kv_heads * (size_t)d->max_seq * (d->head_dim + kie::kKvPad) *
+         2;
 }
 
 kie_status kie_check_desc(const kie_model_desc* d) {

@@ -216,17 +216,17 @@ __device__ __forceinline__ AttnItem attn_item(const MonoParams& p, int pos) {
   a.t1 = (int)(((long long)(s + 1) * n_pos) / nsplit);
   return a;
 }
-// Attention K/V tiles in the ring: rows of hd fp16 at a stride of hd + 8
-// elements, so that the 8 rows an mma fragment load touches fall in 8
-// different bank groups.
-__device__ __forceinline__ int attn_row_stride(const MonoParams& p) { return (p.hd + 8) * 2; }
+// Attention K/V tiles in the ring: rows of hd fp16 at the cache's padded
+// stride of hd + kKvPad elements, so that the 8 rows an mma fragment load
+// touches fall in 8 different bank groups.
+__device__ __forceinline__ int attn_row_stride(const MonoParams& p) { return (p.hd + kKvPad) * 2; }
 // Positions per attention block (one K tile and one V tile in the ring), a
 // multiple of 16.
 __device__ __forceinline__ int attn_block(const MonoParams& p) {
   return max(16, min(kAttnBlock, p.chunk_bytes / attn_row_stride(p)) & ~15);
 }
 __device__ __forceinline__ const __half* kv_rows(const MonoParams& p, int layer, int kv, int j) {
-  return p.kv + (((size_t)layer * 2 + kv) * p.KV + j) * (size_t)p.max_seq * p.hd;
+  return p.kv + (((size_t)layer * 2 + kv) * p.KV + j) * (size_t)p.max_seq * (p.hd + kKvPad);
 }
 
 __device__ __forceinline__ unsigned epoch_of(const MonoParams& p, int step, int layer) {
@@ -353,20 +353,17 @@ struct Producer {
     return true;
   }
 
-  // One attention tile: `alloc` ring bytes, of which rows [0, n) are copied
-  // from `src` (row_bytes each, contiguous) at a ring stride of `stride`;
-  // the consumers fill the remaining rows.
-  __device__ bool tile(const unsigned char* src, int n, uint32_t row_bytes, uint32_t stride,
-                       uint32_t alloc) {
+  // One attention tile: `alloc` ring bytes, of which the first `bytes`
+  // (whole padded cache rows) are copied from `src` in one bulk copy; the
+  // consumers fill the remaining rows.
+  __device__ bool tile(const unsigned char* src, uint32_t bytes, uint32_t alloc) {
     if (sm_flags(p)[F_STOP]) return false;
     const uint32_t off = ring_place(wend, alloc, (uint32_t)p.ring_bytes);
     if (!acquire(off, off + alloc)) return false;
     const uint32_t b = idx & (kRingBars - 1);
     const uint32_t full = sm_full_s(p) + 8 * b;
-    dev::mbar_arrive_expect_tx(full, (uint32_t)n * row_bytes);
-    for (int r = 0; r < n; ++r)
-      dev::bulk_g2s(sm_ring_s(p) + off + r * stride, src + (size_t)r * row_bytes, row_bytes, full,
-                    pol);
+    dev::mbar_arrive_expect_tx(full, bytes);
+    if (bytes > 0) dev::bulk_g2s(sm_ring_s(p) + off, src, bytes, full, pol);
     live_off[b] = off;
     live_end[b] = off + alloc;
     ++idx;
@@ -419,13 +416,13 @@ struct Producer {
     const int tb = attn_block(p);
     const unsigned char* K = reinterpret_cast<const unsigned char*>(kv_rows(p, l, 0, it.j));
     const unsigned char* V = reinterpret_cast<const unsigned char*>(kv_rows(p, l, 1, it.j));
-    const uint32_t row = (uint32_t)p.hd * 2, stride = (uint32_t)attn_row_stride(p);
+    const uint32_t stride = (uint32_t)attn_row_stride(p);
     for (int b0 = it.t0; b0 < it.t1; b0 += tb) {
       const int nb = min(it.t1, b0 + tb) - b0;
       const int nc = max(0, min(b0 + nb, pos) - b0);   // rows already in the cache
       const uint32_t alloc = (uint32_t)((nb + 15) & ~15) * stride;
-      if (!tile(K + (size_t)b0 * row, nc, row, stride, alloc) ||
-          !tile(V + (size_t)b0 * row, nc, row, stride, alloc))
+      if (!tile(K + (size_t)b0 * stride, (uint32_t)nc * stride, alloc) ||
+          !tile(V + (size_t)b0 * stride, (uint32_t)nc * stride, alloc))
         return false;
     }
     return true;
@@ -965,8 +962,9 @@ struct Consumer {
     const int np = qkv_pairs_in(p, r.x, r.y);
     const float2* cs = p.rope + (size_t)pos * half;
     const bool skip = fault_here(ST_QKV);
-    __half* kbase = p.kv + (size_t)layer * 2 * p.KV * p.max_seq * p.hd;
-    __half* vbase = kbase + (size_t)p.KV * p.max_seq * p.hd;
+    const int kvs = p.hd + kKvPad;                    // padded cache row
+    __half* kbase = p.kv + (size_t)layer * 2 * p.KV * p.max_seq * kvs;
+    __half* vbase = kbase + (size_t)p.KV * p.max_seq * kvs;
     for (int u = r.x + tid; u < r.y; u += kConsumerThreads) {
       const int k = u - r.x;
       if (u < np_all) {
@@ -982,7 +980,7 @@ struct Consumer {
           put(p.qbuf + h * p.hd + i + half, tag, hi, skip);
         } else {
           const __half klo = __float2half_rn(lo), khi = __float2half_rn(hi);
-          __half* kd = kbase + ((size_t)h * p.max_seq + pos) * p.hd;
+          __half* kd = kbase + ((size_t)h * p.max_seq + pos) * kvs;
           kd[i] = klo;
           kd[i + half] = khi;
           put(p.kvnew + h * p.hd + i, tag, __half2float(klo), skip);
@@ -993,7 +991,7 @@ struct Consumer {
         const int lr = 2 * np + (k - np);
         const __half vh = __float2half_rn(row_result(pl, lr) * rs);
         const int h = vr / p.hd, e = vr - h * p.hd;
-        vbase[((size_t)h * p.max_seq + pos) * p.hd + e] = vh;
+        vbase[((size_t)h * p.max_seq + pos) * kvs + e] = vh;
         put(p.kvnew + p.KV * p.hd + vr, tag, __half2float(vh), skip);
       }
     }

@@ -37,6 +37,10 @@ constexpr int kPollBackoffNs = 128;          // sleep between re-polls of tagged
 constexpr int kStatsPerCta = 8;
 // stage-trace stamps per layer (the LM head adds 4 per step)
 constexpr int kTracePerLayer = 24;
+// KV cache rows carry kKvPad unused fp16 elements after the hd values, so a
+// run of rows lands in shared memory (one bulk copy) at a stride whose 8
+// consecutive rows fall in 8 different bank groups.
+constexpr int kKvPad = 8;
 // Scratch words (reductions, flags) and the per-stage GEMV plans of the
 // standalone GEMV engine's shared memory (no residual rows there).
 constexpr int kEngineMisc = 640;

@@ -70,7 +70,7 @@ def test_check_desc_rejects_bad_eos_and_capacity(lib):
 def test_kv_cache_bytes(lib):
     for w in synth.WORKLOADS.values():
         s = w.shape
-        want = 2 * s.n_layers * s.n_kv_heads * w.max_seq * s.head_dim * 2
+        want = 2 * s.n_layers * s.n_kv_heads * w.max_seq * (s.head_dim + 8) * 2   # padded rows
         assert _kie.kie_kv_cache_bytes(_desc(s, w.max_seq)) == want
     bad = _desc(synth.WORKLOADS["tiny-l2-d256"].shape, 0)
     assert _kie.kie_kv_cache_bytes(bad) == 0
