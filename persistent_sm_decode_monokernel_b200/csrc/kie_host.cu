@@ -38,8 +38,7 @@ struct kie_ctx {
   size_t tagged_words = 0;
   unsigned long long *x_attn = nullptr, *x_ffn = nullptr, *hbuf = nullptr, *qbuf = nullptr,
                      *kvnew = nullptr, *obuf = nullptr, *slots = nullptr;
-  float* partials = nullptr;
-  unsigned int* att_ctr = nullptr;
+  unsigned long long* partials = nullptr;
   int* d_ids = nullptr;               // fed ids of a launch [max_seq]
   unsigned char* d_io = nullptr;      // DevStatus + out ids [max_seq]
   unsigned long long* cta_stats = nullptr;
@@ -80,6 +79,12 @@ namespace {
 
 constexpr size_t kStatusBytes = sizeof(DevStatus);
 
+// Attention partials: per CTA, G rows of 2 + head_dim/2 tagged words.
+size_t partial_bytes(const kie_ctx* c) {
+  const size_t G = c->desc.n_heads / c->desc.n_kv_heads;
+  return sizeof(unsigned long long) * (size_t)c->grid * G * (c->desc.head_dim / 2 + 2);
+}
+
 kie_status set_err(kie_ctx* c, kie_status s, const std::string& msg) {
   if (c) c->err = msg;
   return s;
@@ -110,7 +115,6 @@ void free_all(kie_ctx* c) {
   cudaFree(c->ranges);
   cudaFree(c->tagged);
   cudaFree(c->partials);
-  cudaFree(c->att_ctr);
   cudaFree(c->d_ids);
   cudaFree(c->d_io);
   cudaFree(c->cta_stats);
@@ -130,6 +134,7 @@ kie_status launch(kie_ctx* c, int n_steps, int pos0, const int32_t* host_ids, bo
   const unsigned need = (unsigned)n_steps * (unsigned)(d.n_layers + 1) + 2u;
   if ((unsigned long long)c->epoch + need >= 0xFFFFFF00ull) {
     KIE_CUDA(c, cudaMemsetAsync(c->tagged, 0, c->tagged_words * 8, c->stream));
+    KIE_CUDA(c, cudaMemsetAsync(c->partials, 0, partial_bytes(c), c->stream));
     c->epoch = 0;
   }
   if (forced) {
@@ -173,7 +178,6 @@ kie_status launch(kie_ctx* c, int n_steps, int pos0, const int32_t* host_ids, bo
   p.obuf = c->obuf;
   p.slots = c->slots;
   p.partials = c->partials;
-  p.att_ctr = c->att_ctr;
   p.n_steps = n_steps;
   p.pos0 = pos0;
   p.first_tok = first_tok;
@@ -396,8 +400,7 @@ kie_status kie_create(const kie_model_desc* d, const kie_weights* w, void* kv_ca
       cuda_bad(cudaMalloc(&c->rope, sizeof(float2) * rope.size())) ||
       cuda_bad(cudaMalloc(&c->ranges, sizeof(int2) * flat.size())) ||
       cuda_bad(cudaMalloc(&c->tagged, 8 * c->tagged_words)) ||
-      cuda_bad(cudaMalloc(&c->partials, sizeof(float) * (size_t)grid * G * (d->head_dim + 4))) ||
-      cuda_bad(cudaMalloc(&c->att_ctr, sizeof(unsigned) * d->n_layers * d->n_kv_heads)) ||
+      cuda_bad(cudaMalloc(&c->partials, partial_bytes(c))) ||
       cuda_bad(cudaMalloc(&c->d_ids, sizeof(int32_t) * d->max_seq)) ||
       cuda_bad(cudaMalloc(&c->d_io, kStatusBytes + sizeof(int32_t) * d->max_seq)) ||
       cuda_bad(cudaMalloc(&c->cta_stats, sizeof(unsigned long long) * kie::kStatsPerCta * grid)) ||
@@ -419,8 +422,7 @@ kie_status kie_create(const kie_model_desc* d, const kie_weights* w, void* kv_ca
       cuda_bad(cudaMemcpyAsync(c->ranges, flat.data(), sizeof(int2) * flat.size(),
                                cudaMemcpyHostToDevice, c->stream)) ||
       cuda_bad(cudaMemsetAsync(c->tagged, 0, 8 * c->tagged_words, c->stream)) ||
-      cuda_bad(cudaMemsetAsync(c->att_ctr, 0, sizeof(unsigned) * d->n_layers * d->n_kv_heads,
-                               c->stream)) ||
+      cuda_bad(cudaMemsetAsync(c->partials, 0, partial_bytes(c), c->stream)) ||
       cuda_bad(cudaMemsetAsync(c->cta_stats, 0, sizeof(unsigned long long) * kie::kStatsPerCta * grid,
                                c->stream)) ||
       cuda_bad(cudaStreamSynchronize(c->stream)))

@@ -46,7 +46,7 @@ using u64 = unsigned long long;
 
 namespace {
 
-enum : int { F_ABORT = 0, F_STOP = 1, F_LAST = 2, F_KVSTEP = 3 };
+enum : int { F_ABORT = 0, F_STOP = 1, F_KVSTEP = 3 };
 
 // The dynamic shared-memory block.  Pointers derived from it directly keep
 // their address space, so the compiler emits shared-memory loads for them.
@@ -199,7 +199,7 @@ __device__ __forceinline__ uint32_t ring_place(uint32_t& wend, uint32_t sz, uint
 // This CTA's attention work item at position pos: KV head j, positions
 // [t0, t1) of 0..pos.  Items are (KV head, split) pairs, item = CTA index.
 struct AttnItem {
-  int j, t0, t1, nsplit;
+  int j, s, t0, t1, nsplit;   // KV head, split index, positions [t0, t1), splits of head j
   bool valid;
 };
 __device__ __forceinline__ AttnItem attn_item(const MonoParams& p, int pos) {
@@ -212,6 +212,7 @@ __device__ __forceinline__ AttnItem attn_item(const MonoParams& p, int pos) {
   a.valid = it < p.KV * nsplit;
   a.j = it / nsplit;
   const int s = it - a.j * nsplit;
+  a.s = s;
   a.t0 = (int)(((long long)s * n_pos) / nsplit);
   a.t1 = (int)(((long long)(s + 1) * n_pos) / nsplit);
   return a;
@@ -998,86 +999,92 @@ struct Consumer {
     return true;
   }
 
-  // The last item of KV head j combines all nsplit partials:
-  // weights w_q = exp(m_q - M) / sum_q exp(m_q - M) l_q per head.
-  // Warp g reads head g's (m, l) of every split at once (lane = split);
-  // then each thread owns 4 output dims of one head and issues the loads of
-  // 16 splits before using any, so a combine costs a few L2 round trips.
+  // Combine of a KV head's partials, spread over the head's items: item s
+  // owns output dims [d0, d1) (a multiple of 4 wide) of every one of the G
+  // heads.  A partial row of (item, head) is [m, l, o/l as fp16 pairs] in
+  // tagged words, so completeness is read from the tags: no fence and no
+  // counter.  The item polls the (m, l) of every split and its dims of
+  // every split's o/l in one batch, then with
+  // w_s = exp(m_s - M) l_s / sum_s exp(m_s - M) l_s writes
+  // o = sum_s w_s (o_s / l_s) for its dims.  Returns false (uniformly) on
+  // abort.
   template <int HD>
-  __device__ __noinline__ void attn_combine(int j, int nsplit, unsigned tag) {
-    constexpr int PST = HD + 4;
-    const int G = p.G;
-    float* wq = AttnSmem<HD>(p).sc;                   // the scores area: [nsplit][G]
-    dev::fence_acq_rel_gpu();
-    const float* base = p.partials + (size_t)(j * nsplit) * G * PST;
-    if (warp < G) {
-      constexpr int QPL = (kMaxSplitCombine + 31) / 32;
-      float mv[QPL], lv[QPL];
-      float M = -INFINITY;
+  __device__ __noinline__ bool attn_combine(const AttnItem& it, unsigned tag) {
+    constexpr int ROW = 2 + HD / 2;          // tagged words per (item, head) row
+    const int G = p.G, nsplit = it.nsplit, j = it.j;
+    const int W = (((HD + nsplit - 1) / nsplit) + 3) & ~3;
+    const int d0 = it.s * W, d1 = min(HD, d0 + W);
+    if (d0 >= d1) return true;
+    const int nd4 = (d1 - d0) / 4;           // o word pairs per row in this slice
+    const u64* base = p.partials + (size_t)(j * nsplit) * G * ROW;
+    const int n2 = nsplit * G * ROW / 2;     // pairs of the head's partial block
+    const int nml = nsplit * G, ntot = nml + nml * nd4;
+    // polled values go where q, P and the scores lived (free once the
+    // blocks are done): (m, l) [nsplit * G], then o/l [nsplit * G][4 * nd4]
+    // at a 16-byte boundary; with nsplit <= 96 and G <= 8 at most 18,432
+    // bytes, within the q, P and score tiles (>= 22,272 bytes)
+    float2* ml = reinterpret_cast<float2*>(AttnSmem<HD>(p).qhi);
+    float* os = reinterpret_cast<float*>(ml + ((nml + 1) & ~1));
+    constexpr int NB = 4;
+    bool bad = false;
+    for (int q0 = tid; q0 < ntot && !bad; q0 += kConsumerThreads * NB) {
+      int k2[NB];
+      ulonglong2 v[NB];
 #pragma unroll
-      for (int k = 0; k < QPL; ++k) {
-        const int q = lane + 32 * k;
-        mv[k] = -INFINITY;
-        lv[k] = 0.f;
-        if (q < nsplit) {
-          const float2 ml = *reinterpret_cast<const float2*>(base + ((size_t)q * G + warp) * PST);
-          mv[k] = ml.x;
-          lv[k] = ml.y;
+      for (int b = 0; b < NB; ++b) {
+        const int q = q0 + b * kConsumerThreads;
+        if (q < nml) {
+          k2[b] = q * (ROW / 2);
+        } else if (q < ntot) {
+          const int r = (q - nml) / nd4, d4 = (q - nml) - r * nd4;
+          k2[b] = (r * ROW + 2 + d0 / 2 + 2 * d4) / 2;
+        } else {
+          k2[b] = n2;
         }
       }
-#pragma unroll
-      for (int k = 0; k < QPL; ++k) M = fmaxf(M, mv[k]);
-      M = dev::warp_max(M);
-      float f[QPL], Ls = 0.f;
-#pragma unroll
-      for (int k = 0; k < QPL; ++k) {
-        f[k] = lane + 32 * k < nsplit ? expf(mv[k] - M) : 0.f;
-        Ls = fmaf(f[k], lv[k], Ls);
+      if (!poll_pairs<NB>(base, k2, n2, tag, v, 23)) {
+        bad = true;
+        break;
       }
-      const float inv = 1.0f / dev::warp_sum(Ls);
 #pragma unroll
-      for (int k = 0; k < QPL; ++k)
-        if (lane + 32 * k < nsplit) wq[(lane + 32 * k) * G + warp] = f[k] * inv;
+      for (int b = 0; b < NB; ++b) {
+        const int q = q0 + b * kConsumerThreads;
+        if (q < nml) {
+          ml[q] = make_float2(__uint_as_float((unsigned)v[b].x), __uint_as_float((unsigned)v[b].y));
+        } else if (q < ntot) {
+          const int r = (q - nml) / nd4, d4 = (q - nml) - r * nd4;
+          const unsigned lo = (unsigned)v[b].x, hi = (unsigned)v[b].y;
+          const float2 x0 = __half22float2(*reinterpret_cast<const __half2*>(&lo));
+          const float2 x1 = __half22float2(*reinterpret_cast<const __half2*>(&hi));
+          *reinterpret_cast<float4*>(os + r * 4 * nd4 + 4 * d4) = make_float4(x0.x, x0.y, x1.x, x1.y);
+        }
+      }
     }
-    dev::consumer_sync();
+    if (dev::consumer_sync_or(bad)) return false;
     const bool skip = fault_here(1);
-    for (int e = tid; e < G * HD / 4; e += kConsumerThreads) {
-      const int g = e / (HD / 4), d4 = e - g * (HD / 4);
-      const float* src = base + (size_t)g * PST + 4 + 4 * d4;
-      float4 O = make_float4(0.f, 0.f, 0.f, 0.f);
-      for (int q0 = 0; q0 < nsplit; q0 += 16) {
-        float4 v[16];
-#pragma unroll
-        for (int u = 0; u < 16; ++u)
-          if (q0 + u < nsplit)
-            v[u] = *reinterpret_cast<const float4*>(src + (size_t)(q0 + u) * G * PST);
-#pragma unroll
-        for (int u = 0; u < 16; ++u) {
-          if (q0 + u < nsplit) {
-            const float wv = wq[(q0 + u) * G + g];
-            O.x = fmaf(wv, v[u].x, O.x);
-            O.y = fmaf(wv, v[u].y, O.y);
-            O.z = fmaf(wv, v[u].z, O.z);
-            O.w = fmaf(wv, v[u].w, O.w);
-          }
-        }
+    const int wd = d1 - d0;
+    for (int e = tid; e < G * wd; e += kConsumerThreads) {
+      const int g = e / wd, dd = e - g * wd;
+      float M = -INFINITY;
+      for (int q = 0; q < nsplit; ++q) M = fmaxf(M, ml[q * G + g].x);
+      float L = 0.f, O = 0.f;
+      for (int q = 0; q < nsplit; ++q) {
+        const float2 v = ml[q * G + g];
+        const float f = expf(v.x - M) * v.y;
+        L += f;
+        O = fmaf(f, os[(q * G + g) * 4 * nd4 + dd], O);
       }
-      u64* dst = p.obuf + ((size_t)j * G + g) * HD + 4 * d4;
-      put(dst, tag, O.x, skip);
-      put(dst + 1, tag, O.y, skip);
-      put(dst + 2, tag, O.z, skip);
-      put(dst + 3, tag, O.w, skip);
+      put(p.obuf + ((size_t)j * G + g) * HD + d0 + dd, tag, O / L, skip);
     }
-    if (tid == 0) p.att_ctr[layer * p.KV + j] = 0u;
-    // the combine weights live in the activation buffer, which the next
-    // stage's input load overwrites: no thread may start that load while
-    // another still reads them
+    // the polled values live in the activation buffer, which the next
+    // stage's input load overwrites
     dev::consumer_sync();
     trace(13);
+    return true;
   }
 
   // Split-K attention over positions 0..pos for the G query heads of one
-  // KV head; the last item of a KV head combines the partials.  K and V
+  // KV head; the head's items then share the combine (attn_combine).  K and V
   // tiles arrive through the ring (issued by the producer before q is
   // ready, rows at a padded stride); the current position's k and v come
   // from the tagged words and are written into the tiles here.  Both
@@ -1274,28 +1281,24 @@ struct Consumer {
     }
     dev::consumer_sync();
     trace(11);
-    // publish this item's partial: per head a row [m, l, -, -, o[HD]] of
-    // HD + 4 floats (16-byte aligned rows; o unnormalised)
-    constexpr int PST = HD + 4;
-    float* part = p.partials + (size_t)blockIdx.x * G * PST;
-    for (int e = tid; e < G * HD / 4; e += kConsumerThreads) {
-      const int g = e / (HD / 4), d4 = e - g * (HD / 4);
-      *reinterpret_cast<float4*>(part + g * PST + 4 + 4 * d4) =
-          *reinterpret_cast<const float4*>(a.orun + g * HD + 4 * d4);
+    // publish this item's partial as tagged words: per head [m, l, then
+    // o / l as fp16 pairs]
+    constexpr int ROW = 2 + HD / 2;
+    u64* part = p.partials + (size_t)blockIdx.x * G * ROW;
+    for (int e = tid; e < G * HD / 2; e += kConsumerThreads) {
+      const int g = e / (HD / 2), i = e - g * (HD / 2);
+      const float inv = 1.0f / a.lrun[g];
+      const __half2 h =
+          __floats2half2_rn(a.orun[g * HD + 2 * i] * inv, a.orun[g * HD + 2 * i + 1] * inv);
+      dev::st_relaxed_u64(part + g * ROW + 2 + i,
+                          (static_cast<u64>(tag) << 32) | *reinterpret_cast<const unsigned*>(&h));
     }
-    if (tid < G)
-      *reinterpret_cast<float2*>(part + tid * PST) = make_float2(a.mrun[tid], a.lrun[tid]);
-    dev::consumer_sync();
-    const int nsplit = it.nsplit;
-    if (tid == 0) {
-      dev::fence_acq_rel_gpu();
-      const unsigned old = atomicAdd(p.att_ctr + layer * p.KV + j, 1u);
-      sm_flags(p)[F_LAST] = (old == (unsigned)(nsplit - 1)) ? 1 : 0;
+    if (tid < G) {
+      dev::st_relaxed_u64(part + tid * ROW, dev::tag_word(tag, a.mrun[tid]));
+      dev::st_relaxed_u64(part + tid * ROW + 1, dev::tag_word(tag, a.lrun[tid]));
     }
-    dev::consumer_sync();
     trace(12);
-    if (sm_flags(p)[F_LAST]) attn_combine<HD>(j, nsplit, tag);
-    return true;
+    return attn_combine<HD>(it, tag);
   }
 
   // O projection + residual -> x_ffn.
@@ -1580,7 +1583,6 @@ __global__ void __launch_bounds__(kThreads, 1) kie_monokernel(const __grid_const
     }
     sm_flags(p)[F_ABORT] = 0;
     sm_flags(p)[F_STOP] = 0;
-    sm_flags(p)[F_LAST] = 0;
     sm_flags(p)[F_KVSTEP] = 0;
     dev::mbar_fence_init();
   }
@@ -1608,7 +1610,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     sm_flags(p)[F_ABORT] = 0;
     sm_flags(p)[F_STOP] = 0;
-    sm_flags(p)[F_LAST] = 0;
     sm_flags(p)[F_KVSTEP] = 0;
     dev::mbar_fence_init();
   }

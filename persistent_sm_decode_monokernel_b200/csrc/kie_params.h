@@ -86,8 +86,7 @@ struct MonoParams {
   SmemLayout sm;
   // scratch (tagged 64-bit words: high 32 bits = epoch tag, low = fp32 bits)
   unsigned long long *x_attn, *x_ffn, *hbuf, *qbuf, *kvnew, *obuf, *slots;
-  float* partials;         // [grid][G][hd + 4]: m, l, 2 unused, o[hd]
-  unsigned int* att_ctr;   // [L][KV] last-arriver counters
+  unsigned long long* partials;  // [grid][G][2 + hd/2] tagged words: m, l, o/l as fp16 pairs
   // run
   int n_steps, pos0, first_tok;
   const int* forced;       // [n_steps] or null
