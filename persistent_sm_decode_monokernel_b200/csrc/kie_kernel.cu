@@ -429,6 +429,25 @@ struct Producer {
     return true;
   }
 
+  // Asks L2 for the K and V rows this CTA's attention item of step i,
+  // layer l will copy, when the layer's weight stream starts: the tiles are
+  // copied into the ring only after the QKV chunks, and from L2 they land in
+  // a fraction of a DRAM round trip under load.
+  __device__ void prefetch_kv(int i, int l) {
+    const int pos = p.pos0 + i;
+    const AttnItem it = attn_item(p, pos);
+    if (!it.valid) return;
+    const int nc = max(0, min(it.t1, pos) - it.t0);
+    if (nc == 0) return;
+    const uint32_t stride = (uint32_t)attn_row_stride(p);
+    for (int kv = 0; kv < 2; ++kv) {
+      const unsigned char* src =
+          reinterpret_cast<const unsigned char*>(kv_rows(p, l, kv, it.j)) + (size_t)it.t0 * stride;
+      for (uint32_t o = 0, n = (uint32_t)nc * stride; o < n; o += 65536u)
+        dev::bulk_prefetch_l2(src + o, min(65536u, n - o));
+    }
+  }
+
   // Waits until every copy this producer issued has landed (the last
   // kRingBars chunks; older ones were consumed before their barrier was
   // reused).
@@ -456,9 +475,11 @@ struct Producer {
     len_lm = stage_len(ST_LM);
     for (int i = 0; i < p.n_steps && ok; ++i) {
       const unsigned char* src = base;
-      for (int l = 0; l < p.L && ok; ++l)
+      for (int l = 0; l < p.L && ok; ++l) {
+        prefetch_kv(i, l);
         ok = stage(ST_QKV, src) && attn(i, l) && stage(ST_O, src) && stage(ST_GU, src) &&
              stage(ST_DOWN, src);
+      }
       if (ok && i >= p.lm_from) ok = stage(ST_LM, src);
     }
     drain();
@@ -950,18 +971,22 @@ struct Consumer {
     const int2 r = p.ranges[ST_QKV * p.grid + blockIdx.x];
     float ss;
     const __half* emb = layer == 0 ? p.tok_emb + (size_t)tok * p.d : nullptr;
-    if (r.y > r.x) {
-      if (!load_vec(p.x_attn, tag, emb, p.d, w.attn_norm, ss, 10)) return false;
-      if (!gemv(ST_QKV)) return false;
-    } else {
-      return true;
-    }
-    const StagePlan pl = sm_plan(p)[ST_QKV];
-    const float rs = 1.0f / sqrtf(ss / (float)p.d + p.eps);
+    if (r.y <= r.x) return true;
     const int half = p.hd >> 1;
     const int nqp = p.H * half, np_all = qkv_pair_units(p);
-    const int np = qkv_pairs_in(p, r.x, r.y);
     const float2* cs = p.rope + (size_t)pos * half;
+    // this thread's first RoPE angle, fetched before the input wait and the
+    // GEMV so that its global round trip is off the critical path
+    float2 cs0 = make_float2(1.f, 0.f);
+    {
+      const int u = r.x + tid;
+      if (u < r.y && u < np_all) cs0 = cs[(u < nqp ? u : u - nqp) % half];
+    }
+    if (!load_vec(p.x_attn, tag, emb, p.d, w.attn_norm, ss, 10)) return false;
+    if (!gemv(ST_QKV)) return false;
+    const StagePlan pl = sm_plan(p)[ST_QKV];
+    const float rs = 1.0f / sqrtf(ss / (float)p.d + p.eps);
+    const int np = qkv_pairs_in(p, r.x, r.y);
     const bool skip = fault_here(ST_QKV);
     const int kvs = p.hd + kKvPad;                    // padded cache row
     __half* kbase = p.kv + (size_t)layer * 2 * p.KV * p.max_seq * kvs;
@@ -973,7 +998,7 @@ struct Consumer {
         const bool isq = u < nqp;
         const int uu = isq ? u : u - nqp;
         const int h = uu / half, i = uu - h * half;
-        const float2 c = cs[i];
+        const float2 c = u == r.x + tid ? cs0 : cs[i];
         const float lo = a * c.x - b * c.y;
         const float hi = b * c.x + a * c.y;
         if (isq) {
