@@ -901,12 +901,15 @@ struct Consumer {
         }
         release();
       }
-      const float s0 = dev::warp_sum(sum8(c0));
-      const float s1 = dev::warp_sum(sum8(c1));
-      if (lane == 0) {
-        rowacc[g0 + warp] = s0;
-        if (two) rowacc[g0 + warp + kConsumerWarps] = s1;
-      }
+      // both rows' sums with one butterfly: after the exchange across the
+      // half-warps, lanes 0-15 reduce row w and lanes 16-31 row w+8
+      const bool upper = (lane & 16) != 0;
+      const float a = sum8(c0), b = sum8(c1);
+      float t = (upper ? b : a) + __shfl_xor_sync(0xffffffffu, upper ? a : b, 16);
+#pragma unroll
+      for (int o = 8; o > 0; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
+      if (lane == 0) rowacc[g0 + warp] = t;
+      if (two && lane == 16) rowacc[g0 + warp + kConsumerWarps] = t;
     };
     for (int g = 0; g < pl.nfull; ++g) group2(g * kGroupRows, kGroupRows, pl.f_nk, pl.f_base, pl.f_rem);
     const int tb = pl.nfull * kGroupRows;
