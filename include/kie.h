@@ -150,7 +150,7 @@ typedef enum {
   KIE_OPT_FAULT_STEP = 5,     /* test hook: step of the withheld publication */
   KIE_OPT_FAULT_LAYER = 6,    /* test hook: layer of the withheld publication */
   KIE_OPT_FAULT_STAGE = 7,    /* test hook: 0 QKV, 1 O, 2 gate/up, 3 down, 4 LM */
-  KIE_OPT_POLL_BACKOFF_NS = 8, /* sleep between re-polls of another CTA's data (default 128) */
+  KIE_OPT_POLL_BACKOFF_NS = 8, /* sleep between re-polls of another CTA's data (default 0) */
   KIE_OPT_TRACE_CLOCK = 9,     /* stage trace in SM cycles (1) instead of ns (0, default) */
   KIE_OPT_L2_PREFETCH_BYTES = 10 /* per CTA, weight-stream bytes requested into L2 ahead of
                                     the shared-memory ring (multiple of 512, <= 16 MiB;

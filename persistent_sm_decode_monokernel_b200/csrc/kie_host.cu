@@ -63,7 +63,7 @@ struct kie_ctx {
 
   // options and capture
   long long timeout_ns = 2000000000LL;
-  unsigned poll_ns = 128;
+  unsigned poll_ns = 0;
   long long l2_prefetch = 0;
   int fault_cta = -1, fault_step = -1, fault_layer = -1, fault_stage = -1;
   float* capture = nullptr;

@@ -665,9 +665,9 @@ struct Consumer {
   // Polls NB pairs of tagged words (pair b at src + 2*k2[b], used when
   // k2[b] < n2) until every word carries `tag`.  All pending pairs are
   // re-read together, so a round costs one L2 round trip; rounds after the
-  // first back off for kPollBackoffNs so that waiting CTAs do not flood L2
-  // while their producers work.  Returns false on abort, timeout or a word
-  // that carries a newer tag (protocol violation).
+  // first sleep p.poll_ns (0 by default: measured fastest) before the next.
+  // Returns false on abort, timeout or a word that carries a newer tag
+  // (protocol violation).
   template <int NB>
   __device__ __forceinline__ bool poll_pairs(const u64* src, const int (&k2)[NB], int n2,
                                              unsigned tag, ulonglong2 (&v)[NB], int where) {
