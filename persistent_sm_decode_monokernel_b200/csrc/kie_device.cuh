@@ -6,6 +6,8 @@
 #include <cstdint>
 #include <cuda_fp16.h>
 
+#include "kie_params.h"
+
 namespace kie {
 namespace dev {
 
@@ -129,7 +131,7 @@ __device__ __forceinline__ unsigned long long tag_word(unsigned int tag, float v
 
 // ---- named barrier for the consumer warps only (barrier 1)
 __device__ __forceinline__ void consumer_sync() {
-  asm volatile("bar.sync 1, %0;" ::"n"(256) : "memory");
+  asm volatile("bar.sync 1, %0;" ::"n"(kConsumerThreads) : "memory");
 }
 // Barrier 1 with an OR-vote: every consumer thread gets the same answer,
 // true if any consumer thread passed `flag` = true.
@@ -141,7 +143,7 @@ __device__ __forceinline__ bool consumer_sync_or(bool flag) {
       "bar.red.or.pred q, 1, %2, p;\n\t"
       "selp.u32 %0, 1, 0, q;\n\t}"
       : "=r"(r)
-      : "r"((uint32_t)flag), "n"(256)
+      : "r"((uint32_t)flag), "n"(kConsumerThreads)
       : "memory");
   return r != 0;
 }

@@ -63,22 +63,25 @@ __device__ __forceinline__ float* sm_rowacc(const MonoParams& p) {
 __device__ __forceinline__ float* sm_misc(const MonoParams& p) {
   return reinterpret_cast<float*>(kie_smem + p.sm.misc_off);
 }
-__device__ __forceinline__ float* sm_part(const MonoParams& p) { return sm_misc(p); }       // [8]
-__device__ __forceinline__ float* sm_red(const MonoParams& p) { return sm_misc(p) + 8; }    // [8]
-__device__ __forceinline__ float* sm_red2(const MonoParams& p) { return sm_misc(p) + 16; }  // [8]
+// per-warp scratch words, kConsumerWarps each (<= 16): partial sums, two
+// reductions with their indices; then flags
+__device__ __forceinline__ float* sm_part(const MonoParams& p) { return sm_misc(p); }
+__device__ __forceinline__ float* sm_red(const MonoParams& p) { return sm_misc(p) + 16; }
+__device__ __forceinline__ float* sm_red2(const MonoParams& p) { return sm_misc(p) + 32; }
 __device__ __forceinline__ int* sm_redi(const MonoParams& p) {
-  return reinterpret_cast<int*>(sm_misc(p) + 24);
+  return reinterpret_cast<int*>(sm_misc(p) + 48);
 }
 __device__ __forceinline__ int* sm_redi2(const MonoParams& p) {
-  return reinterpret_cast<int*>(sm_misc(p) + 32);
+  return reinterpret_cast<int*>(sm_misc(p) + 64);
 }
 __device__ __forceinline__ volatile int* sm_flags(const MonoParams& p) {
-  return reinterpret_cast<volatile int*>(sm_misc(p) + 40);
+  return reinterpret_cast<volatile int*>(sm_misc(p) + 80);
 }
+static_assert(kConsumerWarps <= 16 && 88 <= kMiscHead, "scratch words");
 // residual stream rows this CTA owns (O / down stages)
-__device__ __forceinline__ float* sm_res_attn(const MonoParams& p) { return sm_misc(p) + 64; }
+__device__ __forceinline__ float* sm_res_attn(const MonoParams& p) { return sm_misc(p) + kMiscHead; }
 __device__ __forceinline__ float* sm_res_ffn(const MonoParams& p) {
-  return sm_misc(p) + 64 + p.sm.resid_rows;
+  return sm_misc(p) + kMiscHead + p.sm.resid_rows;
 }
 
 // This CTA's GEMV work in one stage, computed once per launch: kGroupRows
@@ -92,7 +95,7 @@ struct StagePlan {
   int pad[5];
 };
 __device__ __forceinline__ StagePlan* sm_plan(const MonoParams& p) {
-  return reinterpret_cast<StagePlan*>(sm_misc(p) + 64 + 2 * p.sm.resid_rows);
+  return reinterpret_cast<StagePlan*>(sm_misc(p) + kMiscHead + 2 * p.sm.resid_rows);
 }
 __device__ __forceinline__ const unsigned char* sm_ring(const MonoParams& p) {
   return kie_smem + p.sm.ring_off;
@@ -833,7 +836,9 @@ struct Consumer {
         pl.t_nk = t.nk;
         pl.t_base = t.base;
         pl.t_rem = t.rem;
-        pl.t_lw = pl.tail == 1 ? 3 : pl.tail == 2 ? 2 : pl.tail <= 4 ? 1 : 0;
+        int lw = 0;
+        while ((pl.tail << (lw + 1)) <= kConsumerWarps) ++lw;
+        pl.t_lw = lw;
       }
       sm_plan(p)[st] = pl;
     }
@@ -872,9 +877,11 @@ struct Consumer {
       if (lane == 0) dev::mbar_arrive(empty_s + 8 * (cr & (kRingBars - 1)));
       ++cr;
     };
-    // groups with two rows per warp (w and w+8; the second may be missing)
+    // groups of more than kConsumerWarps rows / full groups: warp w owns
+    // rows w (and w + kConsumerWarps when two rows per warp; the second may
+    // be missing)
     auto group2 = [&](int g0, int rg, int nk, int base, int rem) {
-      const bool two = warp + kConsumerWarps < rg;
+      const bool two = kRowsPerWarp == 2 && warp + kConsumerWarps < rg;
       float c0[8], c1[8];
 #pragma unroll
       for (int i = 0; i < 8; ++i) c0[i] = c1[i] = 0.f;
@@ -885,9 +892,9 @@ struct Consumer {
         if (!bad) {
           const uint4* w0 =
               reinterpret_cast<const uint4*>(ring + off + (size_t)warp * n * kPieceBytes) + lane;
-          const uint4* w1 = w0 + (size_t)kConsumerWarps * n * 32;
           const uint4* x = xv + (size_t)p0 * 32;
           if (two) {
+            const uint4* w1 = w0 + (size_t)kConsumerWarps * n * 32;
 #pragma unroll 4
             for (int q = 0; q < n; ++q) {
               const uint4 a = x[q * 32];
@@ -901,15 +908,20 @@ struct Consumer {
         }
         release();
       }
-      // both rows' sums with one butterfly: after the exchange across the
-      // half-warps, lanes 0-15 reduce row w and lanes 16-31 row w+8
-      const bool upper = (lane & 16) != 0;
-      const float a = sum8(c0), b = sum8(c1);
-      float t = (upper ? b : a) + __shfl_xor_sync(0xffffffffu, upper ? a : b, 16);
+      if constexpr (kRowsPerWarp == 2) {
+        // both rows' sums with one butterfly: after the exchange across the
+        // half-warps, lanes 0-15 reduce row w and lanes 16-31 row w+8
+        const bool upper = (lane & 16) != 0;
+        const float a = sum8(c0), b = sum8(c1);
+        float t = (upper ? b : a) + __shfl_xor_sync(0xffffffffu, upper ? a : b, 16);
 #pragma unroll
-      for (int o = 8; o > 0; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
-      if (lane == 0) rowacc[g0 + warp] = t;
-      if (two && lane == 16) rowacc[g0 + warp + kConsumerWarps] = t;
+        for (int o = 8; o > 0; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
+        if (lane == 0) rowacc[g0 + warp] = t;
+        if (two && lane == 16) rowacc[g0 + warp + kConsumerWarps] = t;
+      } else {
+        const float t = dev::warp_sum(sum8(c0));
+        if (lane == 0) rowacc[g0 + warp] = t;
+      }
     };
     for (int g = 0; g < pl.nfull; ++g) group2(g * kGroupRows, kGroupRows, pl.f_nk, pl.f_base, pl.f_rem);
     const int tb = pl.nfull * kGroupRows;
@@ -1132,7 +1144,9 @@ struct Consumer {
     constexpr int QS = HD + 8;                  // halfs per Q tile row
     constexpr int PSW = kAttnBlock + 8;         // halfs per P tile row
     constexpr int KT = HD / 16;                 // k-steps of the score mma
-    constexpr int DTW = HD / 8 / kConsumerWarps;  // 8-dim output tiles per warp
+    // 8-dim output tiles per warp in P.V (warps past HD / 8 have none)
+    constexpr int DTW = HD / 8 >= kConsumerWarps ? HD / 8 / kConsumerWarps : 1;
+    const bool pv_warp = warp * DTW < HD / 8;
     const int G = p.G;
     const int j = it.j;
     const AttnSmem<HD> a(p);
@@ -1266,7 +1280,7 @@ struct Consumer {
       dev::consumer_sync();
       if (b0 == it.t0) trace(15);
       // P.V into the running output (rows gid < G are heads)
-      {
+      if (pv_warp) {
         const float al = gid < G ? a.alpha[gid] : 0.f;
 #pragma unroll
         for (int dt = 0; dt < DTW; ++dt) {
@@ -1299,7 +1313,7 @@ struct Consumer {
       release_chunk();
     }
     // running output of heads gid < G to shared memory
-    if (gid < G) {
+    if (gid < G && pv_warp) {
 #pragma unroll
       for (int dt = 0; dt < DTW; ++dt) {
         const int d = warp * 8 * DTW + dt * 8 + 2 * tig;

@@ -11,20 +11,24 @@ namespace kie {
 // has no weight stream and is not listed here.
 enum Stage : int { ST_QKV = 0, ST_O = 1, ST_GU = 2, ST_DOWN = 3, ST_LM = 4, N_STAGES = 5 };
 
-constexpr int kConsumerWarps = 8;            // warps that compute
-// + one producer warpgroup (only its first lane works): warpgroup-granular
-// register split, see kRegsConsumer / kRegsProducer
-constexpr int kThreads = (kConsumerWarps + 4) * 32;
-// Registers per thread after the split: the launch gives every thread 168
-// (12 warps fit one SM); the producer warpgroup gives up to kRegsProducer
-// and the consumer warpgroups take kRegsConsumer:
-// 8 * kRegsConsumer + 4 * kRegsProducer <= 12 * 168.
-constexpr int kRegsLaunch = 168;
-constexpr int kRegsConsumer = 224;
-constexpr int kRegsProducer = 40;
-static_assert(8 * kRegsConsumer + 4 * kRegsProducer <= 12 * kRegsLaunch, "register split");
+constexpr int kConsumerWarps = 8;            // warps that compute (8 or 16)
 constexpr int kConsumerThreads = kConsumerWarps * 32;
-constexpr int kGroupRows = 16;              // rows streamed together (two per warp)
+// + one producer warpgroup (only its first lane works): warpgroup-granular
+// register split.  The launch gives every thread kRegsLaunch registers
+// (all warps of the CTA fit one SM); the producer warpgroup then gives
+// registers back down to kRegsProducer and the consumer warpgroups take
+// kRegsConsumer, within the launch's total.
+constexpr int kThreads = kConsumerThreads + 128;
+constexpr int kRegsLaunch = kConsumerWarps == 16 ? 96 : 168;
+constexpr int kRegsConsumer = kConsumerWarps == 16 ? 112 : 224;
+constexpr int kRegsProducer = kConsumerWarps == 16 ? 24 : 40;
+static_assert(kConsumerWarps * kRegsConsumer + 4 * kRegsProducer <=
+                  (kConsumerWarps + 4) * kRegsLaunch,
+              "register split exceeds the launch's registers");
+static_assert((kConsumerWarps + 4) * 32 * kRegsLaunch <= 65536, "launch registers");
+constexpr int kGroupRows = 16;              // rows streamed together
+constexpr int kRowsPerWarp = kGroupRows / kConsumerWarps;  // rows of a full group per warp
+static_assert(kRowsPerWarp == 1 || kRowsPerWarp == 2, "group mapping");
 constexpr int kPieceElems = 256;             // one warp pass: 32 lanes x 8 fp16
 constexpr int kPieceBytes = kPieceElems * 2;
 constexpr int kRingBars = 16;                // mbarrier pairs of the byte ring (power of 2)
@@ -41,9 +45,11 @@ constexpr int kTracePerLayer = 24;
 // run of rows lands in shared memory (one bulk copy) at a stride whose 8
 // consecutive rows fall in 8 different bank groups.
 constexpr int kKvPad = 8;
-// Scratch words (reductions, flags) and the per-stage GEMV plans of the
-// standalone GEMV engine's shared memory (no residual rows there).
-constexpr int kEngineMisc = 640;
+// Shared-memory scratch words before the residual rows: per-warp partial
+// sums and reductions, flags (kMiscHead floats).  The standalone GEMV
+// engine's scratch (no residual rows) adds the per-stage GEMV plans.
+constexpr int kMiscHead = 128;
+constexpr int kEngineMisc = 896;
 
 // Device status word block (library scratch, zeroed before each launch).
 struct DevStatus {

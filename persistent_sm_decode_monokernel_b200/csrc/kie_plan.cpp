@@ -109,7 +109,7 @@ bool plan_smem(const Shape& s, int grid, int chunk_bytes, int smem_limit,
     maxres = std::max(maxres, rows_in_range(s, ST_O, ranges[ST_O][c].x, ranges[ST_O][c].y));
   L.resid_rows = maxres;
   const int bars = 2 * kRingBars * 8;
-  const int misc = align_up(64 * 4 + 2 * maxres * 4 + N_STAGES * 64, 128);  // + stage plans
+  const int misc = align_up(kMiscHead * 4 + 2 * maxres * 4 + N_STAGES * 64, 128);  // + stage plans
   const int fixed = align_up(bars, 128) + L.xs_bytes + align_up(maxrows * 4, 128) + misc;
   const int ring = (smem_limit - fixed) / 512 * 512;
   if (ring < 2 * chunk_bytes) return false;
