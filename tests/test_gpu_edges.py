@@ -185,3 +185,36 @@ def test_stats_after_decode(tiny):
     assert st["last_steps"] == 8 and st["last_device_ms"] > 0
     assert 0 <= st["sync_wait_cycles"] <= st["loop_cycles"]
     s.close()
+
+
+def test_l2_prefetch_option_keeps_parity(torch_cuda):
+    from persistent_sm_decode_monokernel_b200 import _kie
+    rep = _forced_parity(synth.WORKLOADS["l16-d1024"].shape, 40, 12,
+                         options=[(_kie.KIE_OPT_L2_PREFETCH_BYTES, 131072)])
+    assert rep.compared == 13
+
+
+def test_trace_of_every_cta(tiny):
+    from persistent_sm_decode_monokernel_b200 import TRACE_PER_LAYER
+    w, m, dev, prompt = tiny
+    s = _session(w.shape, dev, 64)
+    s.prefill(prompt)
+    grid = s.stats()["grid"]
+    buf = s.trace(3, -1)
+    assert tuple(buf.shape) == (3, grid, w.shape.n_layers * TRACE_PER_LAYER + 4)
+    s.decode(3)
+    t = buf.cpu().numpy().astype(np.int64)
+    s.trace_off()
+    s.close()
+    L = w.shape.n_layers
+    for step in range(3):
+        for c in range(grid):
+            row = t[step, c]
+            for l in range(L):
+                e = row[l * TRACE_PER_LAYER:]
+                # QKV begin <= QKV done <= attention done <= O done <= gate/up done <= down done
+                stamps = [e[0], e[2], e[3], e[5], e[7], e[9]]
+                assert all(x > 0 for x in stamps), (step, c, l)
+                assert stamps == sorted(stamps), (step, c, l, stamps)
+            lm = row[L * TRACE_PER_LAYER:L * TRACE_PER_LAYER + 4]
+            assert lm[0] > 0 and lm[3] >= lm[0]
