@@ -518,24 +518,27 @@ __device__ void repack_stage(const MonoParams& p, int st, const LayerW& w, unsig
 // ----------------------------------------------------------------- consumer
 
 // Attention scratch in the activation area of shared memory: q as fp16 hi
-// and lo tiles [16][HD + 8], P tile [16][kAttnBlock + 8] fp16, scores
-// [G][kAttnBlock] fp32 (the combine reuses them), the current position's k
-// and v, the running output [G][HD] and per-head running max, sum and
-// rescale factor.
+// and lo tiles [kMaxGroup][HD + 8] (the mma's padding rows 8-15 are passed
+// as zero registers, never stored), P tile [kMaxGroup][kAttnBlock + 8]
+// fp16, scores [G][kAttnBlock] fp32 (tiles and scores together hold at
+// least kCombineBytesPerHead * G bytes, the combine's scratch), the current
+// position's k and v, the running output [G][HD] and per-head running max,
+// sum and rescale factor.
 template <int HD>
 struct AttnSmem {
+  static constexpr int kTiles = 2 * kMaxGroup * (HD + 8) * 2 + kMaxGroup * (kAttnBlock + 8) * 2;
   __half *qhi, *qlo, *ps;
   float *sc, *kn, *vn, *orun, *mrun, *lrun, *alpha;
   __device__ explicit AttnSmem(const MonoParams& p) {
     unsigned char* b = reinterpret_cast<unsigned char*>(sm_xs(p));
     qhi = reinterpret_cast<__half*>(b);
-    b += 16 * (HD + 8) * 2;
+    b += kMaxGroup * (HD + 8) * 2;
     qlo = reinterpret_cast<__half*>(b);
-    b += 16 * (HD + 8) * 2;
+    b += kMaxGroup * (HD + 8) * 2;
     ps = reinterpret_cast<__half*>(b);
-    b += 16 * (kAttnBlock + 8) * 2;
+    b += kMaxGroup * (kAttnBlock + 8) * 2;
     sc = reinterpret_cast<float*>(b);
-    b += max(p.G * kAttnBlock, 3 * kMaxSplitCombine * kMaxGroup) * 4;
+    b += max(p.G * kAttnBlock * 4, kCombineBytesPerHead * p.G - kTiles);
     kn = reinterpret_cast<float*>(b);
     vn = kn + HD;
     orun = vn + HD;
@@ -1061,8 +1064,8 @@ struct Consumer {
     const int nml = nsplit * G, ntot = nml + nml * nd4;
     // polled values go where q, P and the scores lived (free once the
     // blocks are done): (m, l) [nsplit * G], then o/l [nsplit * G][4 * nd4]
-    // at a 16-byte boundary; with nsplit <= 96 and G <= 8 at most 18,432
-    // bytes, within the q, P and score tiles (>= 22,272 bytes)
+    // at a 16-byte boundary; with nsplit <= 96 at most
+    // kCombineBytesPerHead * G bytes, which the tiles and scores span
     float2* ml = reinterpret_cast<float2*>(AttnSmem<HD>(p).qhi);
     float* os = reinterpret_cast<float*>(ml + ((nml + 1) & ~1));
     constexpr int NB = 4;
@@ -1154,11 +1157,11 @@ struct Consumer {
     const long long c0 = clock64();
     bool bad = false;
     // Q rows >= G and the whole P tile start at zero (those rows stay zero)
-    for (int e = tid; e < (16 - G) * QS; e += kConsumerThreads) {
+    for (int e = tid; e < (kMaxGroup - G) * QS; e += kConsumerThreads) {
       a.qhi[G * QS + e] = __float2half_rn(0.f);
       a.qlo[G * QS + e] = __float2half_rn(0.f);
     }
-    for (int e = tid; e < 16 * PSW / 2; e += kConsumerThreads)
+    for (int e = tid; e < kMaxGroup * PSW / 2; e += kConsumerThreads)
       reinterpret_cast<uint32_t*>(a.ps)[e] = 0u;
     // q (tagged), scaled, as fp16 hi + lo
     {

@@ -45,6 +45,9 @@ constexpr int kTracePerLayer = 24;
 // run of rows lands in shared memory (one bulk copy) at a stride whose 8
 // consecutive rows fall in 8 different bank groups.
 constexpr int kKvPad = 8;
+// Bytes of the attention combine's scratch per query head of a group (the
+// (m, l) of up to kMaxSplitCombine splits and their o/l slices): 96 * 24.
+constexpr int kCombineBytesPerHead = 2304;
 // Shared-memory scratch words before the residual rows: per-warp partial
 // sums and reductions, flags (kMiscHead floats).  The standalone GEMV
 // engine's scratch (no residual rows) adds the per-stage GEMV plans.

@@ -81,10 +81,11 @@ std::vector<int2> partition(const Shape& s, int grid, int stage) {
 }
 
 int attn_smem_bytes(int G, int hd) {
-  int b = 0;
-  b += 2 * 16 * (hd + 8) * 2;        // q as fp16 hi and lo tiles (16 padded rows)
-  b += 16 * (kAttnBlock + 8) * 2;    // P tile, fp16
-  b += std::max(G * kAttnBlock, 3 * kMaxSplitCombine * kMaxGroup) * 4;  // scores / combine
+  const int tiles = 2 * kMaxGroup * (hd + 8) * 2 +   // q as fp16 hi and lo tiles
+                    kMaxGroup * (kAttnBlock + 8) * 2;  // P tile, fp16
+  int b = tiles;
+  // scores; the combine's scratch reuses the tiles and the scores
+  b += std::max(G * kAttnBlock * 4, kCombineBytesPerHead * G - tiles);
   b += 2 * hd * 4;                   // current position's k and v
   b += G * hd * 4;                   // running output
   b += 4 * kMaxGroup * 4;            // running max, sum, rescale, spare
@@ -98,7 +99,7 @@ bool plan_smem(const Shape& s, int grid, int chunk_bytes, int smem_limit,
   const int G = s.H / s.KV;
   const int kmax = std::max(std::max(s.d, s.H * s.hd), s.F);
   SmemLayout L{};
-  L.xs_bytes = align_up(std::max(kmax * 4, attn_smem_bytes(G, s.hd)), 128);
+  L.xs_bytes = align_up(std::max(kmax * 2, attn_smem_bytes(G, s.hd)), 128);  // fp16 input vector
   int maxrows = 0;
   for (int st = 0; st < N_STAGES; ++st)
     for (int c = 0; c < grid; ++c)
