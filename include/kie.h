@@ -218,7 +218,9 @@ KIE_API kie_status kie_set_logits_capture(kie_ctx *ctx, float *dev_logits,
  * partial published, combine done, first K/V tile landed, first block's
  * softmax done (slots 10-15); slots 16-19 and 21: ns the first consumer
  * warp waited for streamed chunks in QKV, O, gate/up, down and attention
- * (durations, not stamps); then LM-head begin, input ready, GEMV done,
+ * (durations, not stamps); slots 22, 23, 20: when the producer started
+ * issuing the layer's QKV chunks, had issued them, and had issued the
+ * attention tiles; then LM-head begin, input ready, GEMV done,
  * pick known.  Steps beyond the
  * capacity are not traced.  NULL turns tracing off. */
 KIE_API kie_status kie_set_trace(kie_ctx *ctx, uint64_t *dev_buf, int32_t capacity, int32_t cta);

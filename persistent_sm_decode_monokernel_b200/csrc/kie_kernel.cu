@@ -374,6 +374,15 @@ struct Producer {
     return true;
   }
 
+  // Stage-trace stamp of the producer lane (slot ev of step i, layer l).
+  __device__ __forceinline__ void trace(int i, int l, int ev) const {
+    if (p.trace && (p.trace_cta < 0 || (int)blockIdx.x == p.trace_cta) && i < p.trace_steps) {
+      const int per = p.L * kTracePerLayer + 4;
+      const int row = p.trace_cta < 0 ? i * p.grid + (int)blockIdx.x : i;
+      p.trace[row * per + l * kTracePerLayer + ev] = (unsigned long long)dev::globaltimer();
+    }
+  }
+
   __device__ bool stage(int st, const unsigned char*& src) {
     const int2 r = p.ranges[st * p.grid + blockIdx.x];
     const int R = range_rows(p, st, r.x, r.y);
@@ -480,8 +489,12 @@ struct Producer {
       const unsigned char* src = base;
       for (int l = 0; l < p.L && ok; ++l) {
         prefetch_kv(i, l);
-        ok = stage(ST_QKV, src) && attn(i, l) && stage(ST_O, src) && stage(ST_GU, src) &&
-             stage(ST_DOWN, src);
+        trace(i, l, 22);
+        ok = stage(ST_QKV, src);
+        trace(i, l, 23);
+        ok = ok && attn(i, l);
+        trace(i, l, 20);
+        ok = ok && stage(ST_O, src) && stage(ST_GU, src) && stage(ST_DOWN, src);
       }
       if (ok && i >= p.lm_from) ok = stage(ST_LM, src);
     }
