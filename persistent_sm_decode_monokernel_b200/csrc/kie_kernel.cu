@@ -12,14 +12,16 @@
 // "GEMV вместо GEMM").
 //
 // B200 design
-//  * Warp specialisation.  Warp 8 is a producer: one lane walks the CTA's
-//    static weight schedule for the whole call and streams it with
-//    cp.async.bulk into a ring of shared-memory slots completed by
+//  * Warp specialisation.  Warpgroup 2 is the producer (one lane works; the
+//    group gives its registers to the consumers with setmaxnreg): it walks
+//    the CTA's static weight schedule for the whole call and streams it
+//    with cp.async.bulk into a byte ring of shared memory completed by
 //    mbarriers.  The schedule does not depend on activations, so the
 //    producer runs ahead across every stage boundary and keeps HBM busy
 //    while the consumers wait for other CTAs.  Warps 0-7 consume: each
-//    16-byte lane load of fp16 weights meets fp32 activations held in shared
-//    memory, FMA in fp32, warp-shuffle reductions.
+//    16-byte lane load of fp16 weights meets the fp16 activations held in
+//    shared memory, fp16 x fp16 products accumulate in fp32, warp-shuffle
+//    reductions.  Attention uses warp-level mma on fp16 tiles.
 //  * Intra-kernel sync by tagged data.  Every vector a stage publishes is
 //    written as 64-bit words {epoch tag, fp32 value}, stored relaxed at gpu
 //    scope; consumers poll the words themselves until the tag of the
@@ -565,7 +567,7 @@ struct Consumer {
   const MonoParams& p;
   int tid, warp, lane;
   uint32_t cidx;   // next chunk to wait for
-  uint32_t crel;   // next chunk to release (chunks are released in order)
+  uint32_t crel;   // next chunk to release (stages release their chunks in order)
   uint32_t cend;   // ring read position (mirrors the producer's placement)
   long long t_sync, t_stream;
   long long w_stage;       // ns warp 0 waited for streamed chunks in the current stage (trace)
@@ -579,9 +581,9 @@ struct Consumer {
     lane = tid & 31;
   }
 
-  // Stage-boundary timestamps of one CTA (measurement): per step
-  // 10 per layer (QKV begin/loaded/done, attention done, O loaded/done,
-  // gate-up loaded/done, down loaded/done) + 4 for the LM head.
+  // Stage trace (measurement, tid 0 only): per step kTracePerLayer slots
+  // per layer (stage boundaries, attention sub-steps, stream waits; the
+  // layout is documented with kie_set_trace) + 4 for the LM head.
   __device__ __forceinline__ void trace_put(int ev, unsigned long long v) const {
     if (p.trace && tid == 0 && (p.trace_cta < 0 || (int)blockIdx.x == p.trace_cta) &&
         step < p.trace_steps) {

@@ -34,8 +34,7 @@ constexpr int kPieceBytes = kPieceElems * 2;
 constexpr int kRingBars = 16;                // mbarrier pairs of the byte ring (power of 2)
 constexpr int kMaxGroup = 8;                 // heads per KV head handled by one CTA
 constexpr int kAttnBlock = 256;              // positions per attention block
-constexpr int kMaxSplitCombine = 96;
-constexpr int kPollBackoffNs = 128;          // sleep between re-polls of tagged words         // attention splits one combine handles
+constexpr int kMaxSplitCombine = 96;         // most attention splits of one KV head
 // per-CTA counters: loop cycles, sync-wait cycles, stream-wait cycles,
 // producer slot-wait cycles, steps done, spare
 constexpr int kStatsPerCta = 8;
