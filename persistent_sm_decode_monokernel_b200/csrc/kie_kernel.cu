@@ -193,6 +193,33 @@ __device__ __forceinline__ Chunking chunking(int rg, int kp, int chunk_bytes) {
   return c;
 }
 
+// The stream order of a stage's chunks (shared by the weight repack, the
+// producer and the consumers): full row groups in pairs whose k-chunks
+// interleave (A0, B0, A1, B1, ...) so that a consumer warp works on the
+// rows of both groups at once, then a leftover full group, then the last,
+// partial group.  f(g0, rg, n, p0) receives each chunk's first row (within
+// the CTA's rows), its row count, its piece count and its first piece;
+// returning false stops the walk.
+template <class F>
+__device__ __forceinline__ bool for_each_chunk(int R, int kp, int chunk_bytes, F&& f) {
+  const int nfull = R / kGroupRows, tail = R - nfull * kGroupRows;
+  const Chunking cf = chunking(kGroupRows, kp, chunk_bytes);
+  int g = 0;
+  for (; g + 1 < nfull; g += 2)
+    for (int kc = 0; kc < cf.nk; ++kc)
+      for (int h = 0; h < 2; ++h)
+        if (!f((g + h) * kGroupRows, kGroupRows, cf.count(kc), cf.first(kc))) return false;
+  if (g < nfull)
+    for (int kc = 0; kc < cf.nk; ++kc)
+      if (!f(g * kGroupRows, kGroupRows, cf.count(kc), cf.first(kc))) return false;
+  if (tail > 0) {
+    const Chunking ct = chunking(tail, kp, chunk_bytes);
+    for (int kc = 0; kc < ct.nk; ++kc)
+      if (!f(nfull * kGroupRows, tail, ct.count(kc), ct.first(kc))) return false;
+  }
+  return true;
+}
+
 // Byte ring placement shared by producer and consumers: a chunk goes right
 // after the previous one, or back to offset 0 when it would not fit.
 __device__ __forceinline__ uint32_t ring_place(uint32_t& wend, uint32_t sz, uint32_t ring_bytes) {
@@ -389,17 +416,13 @@ struct Producer {
     const int2 r = p.ranges[st * p.grid + blockIdx.x];
     const int R = range_rows(p, st, r.x, r.y);
     const int kp = stage_k(p, st) / kPieceElems;
-    for (int g0 = 0; g0 < R; g0 += kGroupRows) {
-      const int rg = min(kGroupRows, R - g0);
-      const Chunking ch = chunking(rg, kp, p.chunk_bytes);
-      for (int kc = 0; kc < ch.nk; ++kc) {
-        const uint32_t sz = (uint32_t)(rg * ch.count(kc) * kPieceBytes);
-        if (p.l2_prefetch > 0) prefetch(sz);
-        if (!chunk(src, sz)) return false;
-        pf_ahead -= sz;
-      }
-    }
-    return true;
+    return for_each_chunk(R, kp, p.chunk_bytes, [&](int, int rg, int n, int) {
+      const uint32_t sz = (uint32_t)(rg * n * kPieceBytes);
+      if (p.l2_prefetch > 0) prefetch(sz);
+      if (!chunk(src, sz)) return false;
+      pf_ahead -= sz;
+      return true;
+    });
   }
 
   // K and V blocks of this CTA's attention item at step i, layer l, for the
@@ -512,22 +535,18 @@ __device__ void repack_stage(const MonoParams& p, int st, const LayerW& w, unsig
   const int2 r = p.ranges[st * p.grid + blockIdx.x];
   const int R = range_rows(p, st, r.x, r.y);
   const int kp = stage_k(p, st) / kPieceElems;
-  for (int g0 = 0; g0 < R; g0 += kGroupRows) {
-    const int rg = min(kGroupRows, R - g0);
-    const Chunking ch = chunking(rg, kp, p.chunk_bytes);
-    for (int kc = 0; kc < ch.nk; ++kc) {
-      const int n = ch.count(kc), p0 = ch.first(kc);
-      const int n16 = n * kPieceBytes / 16;
-      uint4* d = reinterpret_cast<uint4*>(dst);
-      for (int e = threadIdx.x; e < rg * n16; e += blockDim.x) {
-        const int j = e / n16, q = e - j * n16;
-        const uint4* src = reinterpret_cast<const uint4*>(row_ptr(p, st, w, r.x, r.y, g0 + j) +
-                                                          (size_t)p0 * kPieceElems);
-        d[e] = src[q];
-      }
-      dst += (size_t)rg * n * kPieceBytes;
+  for_each_chunk(R, kp, p.chunk_bytes, [&](int g0, int rg, int n, int p0) {
+    const int n16 = n * kPieceBytes / 16;
+    uint4* d = reinterpret_cast<uint4*>(dst);
+    for (int e = threadIdx.x; e < rg * n16; e += blockDim.x) {
+      const int j = e / n16, q = e - j * n16;
+      const uint4* src = reinterpret_cast<const uint4*>(row_ptr(p, st, w, r.x, r.y, g0 + j) +
+                                                        (size_t)p0 * kPieceElems);
+      d[e] = src[q];
     }
-  }
+    dst += (size_t)rg * n * kPieceBytes;
+    return true;
+  });
 }
 
 // ----------------------------------------------------------------- consumer
@@ -941,7 +960,74 @@ struct Consumer {
         if (lane == 0) rowacc[g0 + warp] = t;
       }
     };
-    for (int g = 0; g < pl.nfull; ++g) group2(g * kGroupRows, kGroupRows, pl.f_nk, pl.f_base, pl.f_rem);
+    // pairs of full groups (their chunks interleave in the stream): warp w
+    // owns its rows of both groups, one activation load per piece serves all
+    // of them
+    auto group_pair = [&](int g0) {
+      constexpr int RW = 2 * kRowsPerWarp;             // rows per warp
+      float c[RW][8];
+#pragma unroll
+      for (int r = 0; r < RW; ++r)
+#pragma unroll
+        for (int i = 0; i < 8; ++i) c[r][i] = 0.f;
+      for (int kc = 0; kc < pl.f_nk; ++kc) {
+        const int n = pl.f_base + (kc < pl.f_rem ? 1 : 0), p0 = kc * pl.f_base + min(kc, pl.f_rem);
+        const uint32_t sz = (uint32_t)(kGroupRows * n * kPieceBytes);
+        uint32_t offa, offb;
+        if (!wait(sz, offa)) bad = true;
+        if (!wait(sz, offb)) bad = true;
+        if (!bad) {
+          const uint4* x = xv + (size_t)p0 * 32;
+          const uint4* wa = reinterpret_cast<const uint4*>(ring + offa + (size_t)warp * n * kPieceBytes) + lane;
+          const uint4* wb = reinterpret_cast<const uint4*>(ring + offb + (size_t)warp * n * kPieceBytes) + lane;
+          const size_t second = (size_t)kConsumerWarps * n * 32;   // row w + kConsumerWarps
+#pragma unroll 2
+          for (int q = 0; q < n; ++q) {
+            const uint4 xa = x[q * 32];
+            dot_piece(wa[q * 32], xa, c[0]);
+            dot_piece(wb[q * 32], xa, c[1]);
+            if constexpr (kRowsPerWarp == 2) {
+              dot_piece(wa[second + q * 32], xa, c[2]);
+              dot_piece(wb[second + q * 32], xa, c[3]);
+            }
+          }
+        }
+        release();
+        release();
+      }
+      // butterfly over the warp's rows: after the exchanges each group of
+      // 32 / RW lanes holds one row's partial sums
+      float v[RW];
+#pragma unroll
+      for (int r = 0; r < RW; ++r) v[r] = sum8(c[r]);
+      if constexpr (RW == 4) {
+        // rows: 0 = A w, 1 = B w, 2 = A w+K, 3 = B w+K (K = kConsumerWarps)
+        const bool up = (lane & 16) != 0;
+        const float k0 = up ? v[2] : v[0], s0 = up ? v[0] : v[2];
+        const float k1 = up ? v[3] : v[1], s1 = up ? v[1] : v[3];
+        const float t0 = k0 + __shfl_xor_sync(0xffffffffu, s0, 16);
+        const float t1 = k1 + __shfl_xor_sync(0xffffffffu, s1, 16);
+        const bool mid = (lane & 8) != 0;
+        float u = (mid ? t1 : t0) + __shfl_xor_sync(0xffffffffu, mid ? t0 : t1, 8);
+#pragma unroll
+        for (int o = 4; o > 0; o >>= 1) u += __shfl_xor_sync(0xffffffffu, u, o);
+        // lane 0: A w, 8: B w, 16: A w+K, 24: B w+K
+        if ((lane & 7) == 0) {
+          const int row = (lane & 8 ? kGroupRows : 0) + (lane & 16 ? kConsumerWarps : 0) + warp;
+          rowacc[g0 + row] = u;
+        }
+      } else {
+        // rows: 0 = A w, 1 = B w
+        const bool up = (lane & 16) != 0;
+        float u = (up ? v[1] : v[0]) + __shfl_xor_sync(0xffffffffu, up ? v[0] : v[1], 16);
+#pragma unroll
+        for (int o = 8; o > 0; o >>= 1) u += __shfl_xor_sync(0xffffffffu, u, o);
+        if ((lane & 15) == 0) rowacc[g0 + (up ? kGroupRows : 0) + warp] = u;
+      }
+    };
+    int g = 0;
+    for (; g + 1 < pl.nfull; g += 2) group_pair(g * kGroupRows);
+    if (g < pl.nfull) group2(g * kGroupRows, kGroupRows, pl.f_nk, pl.f_base, pl.f_rem);
     const int tb = pl.nfull * kGroupRows;
     if (pl.tail > kConsumerWarps) {
       group2(tb, pl.tail, pl.t_nk, pl.t_base, pl.t_rem);
@@ -1534,15 +1620,12 @@ struct Consumer {
     const int R = range_rows(p, st, ub, ue);
     const int kp = stage_k(p, st) / kPieceElems;
     bool bad = false;
-    for (int g0 = 0; g0 < R; g0 += kGroupRows) {
-      const int rg = min(kGroupRows, R - g0);
-      const Chunking ch = chunking(rg, kp, p.chunk_bytes);
-      for (int kc = 0; kc < ch.nk; ++kc) {
-        uint32_t off;
-        if (!wait_chunk((uint32_t)(rg * ch.count(kc) * kPieceBytes), off)) bad = true;
-        release_chunk();
-      }
-    }
+    for_each_chunk(R, kp, p.chunk_bytes, [&](int, int rg, int n, int) {
+      uint32_t off;
+      if (!wait_chunk((uint32_t)(rg * n * kPieceBytes), off)) bad = true;
+      release_chunk();
+      return true;
+    });
     return !dev::consumer_sync_or(bad);
   }
 

@@ -20,8 +20,8 @@ constexpr int kConsumerThreads = kConsumerWarps * 32;
 // kRegsConsumer, within the launch's total.
 constexpr int kThreads = kConsumerThreads + 128;
 constexpr int kRegsLaunch = kConsumerWarps == 16 ? 96 : 168;
-constexpr int kRegsConsumer = kConsumerWarps == 16 ? 112 : 224;
-constexpr int kRegsProducer = kConsumerWarps == 16 ? 24 : 40;
+constexpr int kRegsConsumer = kConsumerWarps == 16 ? 112 : 216;
+constexpr int kRegsProducer = kConsumerWarps == 16 ? 24 : 56;
 static_assert(kConsumerWarps * kRegsConsumer + 4 * kRegsProducer <=
                   (kConsumerWarps + 4) * kRegsLaunch,
               "register split exceeds the launch's registers");
