@@ -6,7 +6,9 @@ with the CUDA path.  Only `tests/`, `__graft_entry__.smoke()` and the CPU
 baseline leg of `bench.py` may import it; the library itself never does.
 
 Every function carries its definition in its docstring; `tests/test_oracle_pins.py`
-pins each of them to closed forms, invariants and brute force.  Parity status
+pins each of them to closed forms, invariants and brute force, and
+`tests/test_oracle_sampling.py` pins the sampler (`oracle.sampling`) to
+numpy's own Philox generator and to the softmax distribution it must draw.  Parity status
 of each function: all pinned (none is "parity unpinned").
 """
 from .model import (  # noqa: F401
