@@ -2,11 +2,12 @@
 """Batch-1 decode benchmark of the persistent decode kernel on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
-                    [--impl reference] [--no-cpu-baseline]
+                    [--temperature T --seed S] [--impl reference] [--no-cpu-baseline]
 
 A step is one request's decode: the session is rewound to the end of the
-prompt (P positions of KV already in HBM) and kie_decode runs S greedy steps
-in ONE launch of the persistent kernel.  W untimed steps, then K timed
+prompt (P positions of KV already in HBM) and kie_decode runs S steps
+(greedy, or temperature sampling with --temperature) in ONE launch of the
+persistent kernel.  W untimed steps, then K timed
 steps bracketed by a barrier and a device synchronize, timed with CUDA
 events on the launching stream.  `value` is decode tokens/s per request:
 N * K * S / (max over ranks of the timed region).  With N > 1 every rank
@@ -227,19 +228,32 @@ def run_reference(args, w, rank, world):
         return 0
     model = synth.make_model(w.shape, seed=w.seed)
     from oracle import OracleModel, argmax_lowest
+    from oracle import sampling
     from threadpoolctl import threadpool_info
     om = OracleModel(model, dtype=np.float32)
     prompt = synth.make_prompt(w.shape.vocab, w.prompt_len, seed=w.seed)
     st, lg = om.prefill_batched(prompt)
-    tok = argmax_lowest(lg)
+
+    def pick(logits, pos):
+        if args.temperature > 0:
+            return sampling.sample_id(logits, args.temperature, args.seed, pos)
+        return argmax_lowest(logits)
+
+    tok = pick(lg, w.prompt_len - 1)
     per_step = args.ref_tokens_per_step
+
+    def step():
+        nonlocal tok
+        pos = st.pos
+        tok = pick(om.decode_step(st, tok), pos)
+
     for _ in range(args.warmup):
         for _ in range(per_step):
-            tok = argmax_lowest(om.decode_step(st, tok))
+            step()
     t0 = time.perf_counter()
     for _ in range(args.steps):
         for _ in range(per_step):
-            tok = argmax_lowest(om.decode_step(st, tok))
+            step()
     el = time.perf_counter() - t0
     value = args.steps * per_step / el
     threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
@@ -251,7 +265,7 @@ def run_reference(args, w, rank, world):
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1000.0 * el / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-        "config": workload_config(w),
+        "config": run_config(w, args),
         "cpu_baseline": {"value": value, "unit": "tok/s", "cores": threads, "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": value, "unit": "tok/s", "h2d_bytes_per_step": 0,
@@ -259,6 +273,14 @@ def run_reference(args, w, rank, world):
     }
     print(json.dumps(line), flush=True)
     return 0
+
+
+def run_config(w: synth.Workload, args):
+    """The workload plus the token-selection rule of this run."""
+    sel = "greedy" if args.temperature <= 0 else {
+        "sampling": "temperature (Gumbel-max, Philox4x64-10)",
+        "temperature": args.temperature, "seed": args.seed}
+    return dict(workload_config(w), token_selection=sel)
 
 
 def workload_config(w: synth.Workload):
@@ -287,6 +309,7 @@ def run_gpu(args, w, dist, rank, world):
     prompt = synth.make_prompt(w.shape.vocab, w.prompt_len, seed=w.seed)
     stream = torch.cuda.current_stream()
     sess = Session(w.shape, dev, max_seq=w.max_seq, stream=stream)
+    sess.set_sampling(args.temperature, args.seed)
     sess.prefill(prompt)
     P, S = w.prompt_len, w.decode_steps
     out = np.empty(S, dtype=np.int32)
@@ -354,7 +377,8 @@ def run_gpu(args, w, dist, rank, world):
         "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1000.0 * t_max / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f16 weights+KV, f32 accumulate",
-        "data": "synthetic", "config": workload_config(w),
+        "data": "synthetic",
+        "config": run_config(w, args),
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "peak_source": peak_kind,
                      "frac_vs_nominal_8tbs": achieved / NOMINAL_HBM_GBS,
@@ -391,6 +415,9 @@ def main(argv=None):
                     choices=sorted(synth.WORKLOADS) + sorted(synth.PROFILE_WORKLOADS))
     ap.add_argument("--decode-steps", type=int, default=None,
                     help="decode steps per launch (default: the workload's); for profiler runs")
+    ap.add_argument("--temperature", type=float, default=0.0,
+                    help="0 = greedy (default); > 0 = in-kernel temperature sampling")
+    ap.add_argument("--seed", type=int, default=0, help="sampling seed")
     ap.add_argument("--impl", default="kie", choices=["kie", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ref-tokens-per-step", type=int, default=4)

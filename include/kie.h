@@ -12,7 +12,9 @@
  * EOS check, without returning to the CPU and without a launch per token.
  * The projections are matrix-vector products on the vector ALUs, not tensor
  * cores (same page, section "Архитектура и особенности", "GEMV вместо GEMM").
- * Token selection is greedy (argmax, lowest index on ties).
+ * Token selection is greedy (argmax, lowest index on ties) by default, or
+ * temperature sampling inside the kernel (kie_set_sampling); a set of up to
+ * KIE_MAX_EOS_IDS ids ends a decode (kie_set_eos_ids).
  *
  * Model (pre-norm decoder; the pages never print the block, this is the
  * reading the library implements):
@@ -173,21 +175,23 @@ KIE_API kie_status kie_create(const kie_model_desc *desc, const kie_weights *wei
 
 /* Runs the prompt through the model in one launch, writing K/V for
  * positions 0..n-1 (the session restarts at position 0), and returns in
- * *first_id the greedy id picked from the last position's logits.
+ * *first_id the id picked (greedy or sampled, kie_set_sampling) from the
+ * last position's logits.
  * prompt_ids: HOST array [n] with ids in [0, vocab).  first_id may be NULL. */
 KIE_API kie_status kie_prefill(kie_ctx *ctx, const int32_t *prompt_ids, int32_t n,
                        int32_t *first_id);
 
-/* Runs n_steps greedy decode steps in ONE launch.  Step i feeds the
+/* Runs n_steps decode steps in ONE launch.  Step i feeds the
  * previous id (the id from kie_prefill or the last id of the previous
  * decode call for i = 0) at the next position and writes the picked id to
- * out_ids[i] (HOST array [n_steps]).  Stops after emitting eos_id; *n_out
+ * out_ids[i] (HOST array [n_steps]).  Stops after emitting an end id
+ * (eos_id, or the set of kie_set_eos_ids); *n_out
  * (nullable) receives the number of ids written.  n_steps = 0 is a no-op. */
 KIE_API kie_status kie_decode(kie_ctx *ctx, int32_t n_steps, int32_t *out_ids,
                       int32_t *n_out);
 
 /* Teacher-forced decode, one launch: step i feeds ids[i] (HOST [n]) at the
- * next position instead of the previous pick, and still writes the greedy
+ * next position instead of the previous pick, and still writes the
  * pick to out_ids[i] (HOST [n], nullable).  Afterwards the session
  * continues from the last pick.  Used to compare logits against a
  * reference on a fixed token stream. */
@@ -224,6 +228,31 @@ KIE_API kie_status kie_set_logits_capture(kie_ctx *ctx, float *dev_logits,
  * pick known.  Steps beyond the
  * capacity are not traced.  NULL turns tracing off. */
 KIE_API kie_status kie_set_trace(kie_ctx *ctx, uint64_t *dev_buf, int32_t capacity, int32_t cta);
+
+/* Token selection (the pages' in-kernel "LM-head sampling", revietech.ru,
+ * "Kog выжимает максимум из GPU: 3000 токенов/с", section "Что такое
+ * monokernel"; the pages give no sampler, temperature sampling is the
+ * reading taken).  temperature == 0: greedy argmax (the default).
+ * temperature > 0: every step that picks an id draws it from
+ * softmax(logits / temperature) inside the kernel, as the argmax over the
+ * vocabulary of  logit_i / temperature + G_i,  G_i = -log(-log(U_i)), with
+ *   U_i = ((w >> 11) + 0.5) * 2^-53,
+ *   w   = word (i % 4) of Philox4x64-10(counter = (i / 4, t, 0, 0), key = (seed, 0))
+ * (Salmon et al., "Parallel random numbers: as easy as 1, 2, 3", SC 2011)
+ * and t the 0-based position of the token whose logits are sampled.  A draw
+ * depends only on (seed, t, logits), so kie_rewind followed by the same
+ * decode reproduces it.  Applies to kie_prefill's first id, kie_decode and
+ * kie_decode_forced.  Returns KIE_ERR_INVALID_ARG for a NULL ctx or a
+ * temperature that is negative, infinite or NaN.  Host only. */
+KIE_API kie_status kie_set_sampling(kie_ctx *ctx, float temperature, uint64_t seed);
+
+/* Ids that end a decode: a step whose picked id is one of ids[0 .. n) is
+ * the last one (it is written and counted in *n_out).  n = 0 goes back to
+ * the model descriptor's eos_id (none if -1).  ids: HOST array, copied.
+ * KIE_ERR_INVALID_ARG for a NULL ctx, n outside 0 .. KIE_MAX_EOS_IDS, a NULL
+ * ids with n > 0 or an id outside [0, vocab).  Host only. */
+#define KIE_MAX_EOS_IDS 8
+KIE_API kie_status kie_set_eos_ids(kie_ctx *ctx, const int32_t *ids, int32_t n);
 
 KIE_API kie_status kie_set_option(kie_ctx *ctx, kie_option opt, int64_t value);
 KIE_API kie_status kie_get_stats(const kie_ctx *ctx, kie_stats *out);

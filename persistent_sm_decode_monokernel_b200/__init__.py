@@ -14,8 +14,9 @@ import numpy as np
 from . import _kie
 from ._kie import (KieError, kie_check_desc, kie_create, kie_decode, kie_decode_forced,  # noqa: F401
                    kie_destroy, kie_get_stats, kie_kv_cache_bytes, kie_last_error,
-                   kie_plan_units, kie_prefill, kie_rewind, kie_set_logits_capture,
-                   kie_set_option, kie_set_trace, load_library, make_desc)
+                   kie_plan_units, kie_prefill, kie_rewind, kie_set_eos_ids,
+                   kie_set_logits_capture, kie_set_option, kie_set_sampling, kie_set_trace,
+                   load_library, make_desc)
 
 TRACE_PER_LAYER = 24   # trace slots per layer (kie.h, kie_set_trace)
 
@@ -100,6 +101,14 @@ class Session:
 
     def set_option(self, opt: int, value: int) -> None:
         kie_set_option(self.ctx, opt, value)
+
+    def set_sampling(self, temperature: float, seed: int = 0) -> None:
+        """temperature 0 = greedy (default); > 0 samples in the kernel."""
+        kie_set_sampling(self.ctx, temperature, seed)
+
+    def set_eos_ids(self, ids: Sequence[int]) -> None:
+        """Ids that end a decode ([] = the descriptor's eos_id)."""
+        kie_set_eos_ids(self.ctx, ids)
 
     def stats(self):
         return kie_get_stats(self.ctx)

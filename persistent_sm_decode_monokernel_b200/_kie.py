@@ -28,6 +28,7 @@ KIE_ERR_PROTOCOL = 7
 KIE_ERR_TOO_LARGE = 8
 
 KIE_NOALLOC_MAX_WEIGHT_BYTES = 16 * 1024 * 1024
+KIE_MAX_EOS_IDS = 8
 
 KIE_OPT_TIMEOUT_NS = 1
 KIE_OPT_CHUNK_BYTES = 2
@@ -89,6 +90,8 @@ SIGNATURES = {
     "kie_rewind": (ctypes.c_int, [_P, _I32]),
     "kie_set_logits_capture": (ctypes.c_int, [_P, _P, _I32]),
     "kie_set_option": (ctypes.c_int, [_P, ctypes.c_int, ctypes.c_int64]),
+    "kie_set_sampling": (ctypes.c_int, [_P, ctypes.c_float, ctypes.c_uint64]),
+    "kie_set_eos_ids": (ctypes.c_int, [_P, _PI32, _I32]),
     "kie_set_trace": (ctypes.c_int, [_P, _P, _I32, _I32]),
     "kie_get_stats": (ctypes.c_int, [_P, ctypes.POINTER(KieStats)]),
     "kie_status_str": (ctypes.c_char_p, [ctypes.c_int]),
@@ -200,7 +203,7 @@ def kie_prefill(ctx, ids: Sequence[int]) -> int:
 
 
 def kie_decode(ctx, n_steps: int, out: Optional[np.ndarray] = None) -> np.ndarray:
-    """Greedy decode of n_steps ids in one launch; returns the ids written."""
+    """Decode of n_steps ids in one launch; returns the ids written."""
     if out is None:
         out = np.empty(max(n_steps, 1), dtype=np.int32)
     n_out = ctypes.c_int32()
@@ -235,6 +238,18 @@ def kie_set_trace(ctx, buf=None, capacity: int = 0, cta: int = 0) -> None:
 
 def kie_set_option(ctx, opt: int, value: int) -> None:
     _check(load_library().kie_set_option(ctx, opt, int(value)), "kie_set_option", ctx)
+
+
+def kie_set_sampling(ctx, temperature: float, seed: int = 0) -> None:
+    """temperature 0 = greedy; > 0 = in-kernel temperature sampling."""
+    _check(load_library().kie_set_sampling(ctx, float(temperature), int(seed) & ((1 << 64) - 1)),
+           "kie_set_sampling", ctx)
+
+
+def kie_set_eos_ids(ctx, ids: Sequence[int]) -> None:
+    a = np.ascontiguousarray(np.asarray(list(ids), dtype=np.int32))
+    _check(load_library().kie_set_eos_ids(ctx, a.ctypes.data_as(_PI32) if a.size else None,
+                                          a.size), "kie_set_eos_ids", ctx)
 
 
 def kie_get_stats(ctx) -> Dict[str, float]:

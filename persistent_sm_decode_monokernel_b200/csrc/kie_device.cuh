@@ -206,6 +206,34 @@ __device__ __forceinline__ void regs_inc() {
   asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;\n" ::"n"(N) : "memory");
 }
 
+// ---- Philox4x64-10 (Salmon, Moraes, Dror and Shaw, "Parallel random
+// numbers: as easy as 1, 2, 3", SC 2011): word `w` (0..3) of the block for
+// counter (c0, c1, 0, 0) under key (k0, 0).  Ten rounds; each multiplies
+// counter words 0 and 2 by the round multipliers (full 128-bit products),
+// folds the high halves into words 1 and 3 with the key and permutes; the
+// key advances by the Weyl increments between rounds.
+__device__ __forceinline__ unsigned long long philox4x64_10_word(unsigned long long c0,
+                                                                 unsigned long long c1,
+                                                                 unsigned long long k0, int w) {
+  constexpr unsigned long long M0 = 0xD2E7470EE14C6C93ull, M1 = 0xCA5A826395121157ull;
+  constexpr unsigned long long W0 = 0x9E3779B97F4A7C15ull, W1 = 0xBB67AE8584CAA73Bull;
+  unsigned long long x0 = c0, x1 = c1, x2 = 0, x3 = 0, k1 = 0;
+#pragma unroll
+  for (int r = 0; r < 10; ++r) {
+    if (r) {
+      k0 += W0;
+      k1 += W1;
+    }
+    const unsigned long long hi0 = __umul64hi(M0, x0), lo0 = M0 * x0;
+    const unsigned long long hi1 = __umul64hi(M1, x2), lo1 = M1 * x2;
+    x0 = hi1 ^ x1 ^ k0;
+    x1 = lo1;
+    x2 = hi0 ^ x3 ^ k1;
+    x3 = lo0;
+  }
+  return w == 0 ? x0 : w == 1 ? x1 : w == 2 ? x2 : x3;
+}
+
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);

@@ -68,6 +68,11 @@ struct kie_ctx {
   int fault_cta = -1, fault_step = -1, fault_layer = -1, fault_stage = -1;
   float* capture = nullptr;
   int capture_rows = 0;
+  // token selection: temperature 0 = greedy; ids that end a decode (empty:
+  // the model descriptor's eos_id, if any)
+  double temperature = 0.0;
+  unsigned long long seed = 0;
+  std::vector<int32_t> eos_ids;
   unsigned long long* trace = nullptr;
   int trace_cta = 0, trace_steps = 0, trace_clock = 0;
 
@@ -154,7 +159,16 @@ kie_status launch(kie_ctx* c, int n_steps, int pos0, const int32_t* host_ids, bo
   p.G = d.n_heads / d.n_kv_heads;
   p.eps = d.rms_eps;
   p.max_seq = d.max_seq;
-  p.eos = d.eos_id;
+  if (!c->eos_ids.empty()) {
+    p.n_eos = (int)c->eos_ids.size();
+    for (int k = 0; k < p.n_eos; ++k) p.eos_ids[k] = c->eos_ids[k];
+  } else if (d.eos_id >= 0) {
+    p.n_eos = 1;
+    p.eos_ids[0] = d.eos_id;
+  }
+  p.sample = c->temperature > 0.0 ? 1 : 0;
+  p.inv_temp = c->temperature > 0.0 ? 1.0 / c->temperature : 0.0;
+  p.seed = c->seed;
   p.layers = c->dlayers;
   p.tok_emb = c->tok_emb;
   p.final_norm = c->final_norm;
@@ -522,6 +536,28 @@ kie_status kie_set_logits_capture(kie_ctx* c, float* dev_logits, int32_t rows) {
   if (dev_logits && rows < 1) return set_err(c, KIE_ERR_INVALID_ARG, "capacity_rows < 1");
   c->capture = dev_logits;
   c->capture_rows = dev_logits ? rows : 0;
+  return KIE_OK;
+}
+
+static_assert(KIE_MAX_EOS_IDS == kie::kMaxEosIds, "EOS id set size");
+
+kie_status kie_set_sampling(kie_ctx* c, float temperature, uint64_t seed) {
+  if (!c) return KIE_ERR_INVALID_ARG;
+  if (!std::isfinite(temperature) || temperature < 0.f)
+    return set_err(c, KIE_ERR_INVALID_ARG, "temperature must be finite and >= 0");
+  c->temperature = (double)temperature;
+  c->seed = seed;
+  return KIE_OK;
+}
+
+kie_status kie_set_eos_ids(kie_ctx* c, const int32_t* ids, int32_t n) {
+  if (!c) return KIE_ERR_INVALID_ARG;
+  if (n < 0 || n > KIE_MAX_EOS_IDS) return set_err(c, KIE_ERR_INVALID_ARG, "eos id count out of range");
+  if (n > 0 && !ids) return set_err(c, KIE_ERR_INVALID_ARG, "ids is NULL");
+  for (int i = 0; i < n; ++i)
+    if (ids[i] < 0 || ids[i] >= c->desc.vocab)
+      return set_err(c, KIE_ERR_INVALID_ARG, "eos id out of range");
+  c->eos_ids.assign(ids, ids + n);
   return KIE_OK;
 }
 

@@ -1521,10 +1521,29 @@ struct Consumer {
     }
   }
 
-  // Final RMSNorm + LM head + argmax; or, on steps that pick no id, only
-  // the per-step fenced publish.  Returns false on abort; *tok_out gets the
-  // greedy id (uniform across the grid).
-  __device__ __noinline__ bool stage_lm(bool pick, int step_row, unsigned tag, int* tok_out) {
+  // Score of vocabulary entry u whose logit is v, at position pos: the
+  // logit itself (greedy), or v / T + G with G = -log(-log(U)) standard
+  // Gumbel noise, U from word u % 4 of Philox4x64-10 block (u / 4, pos)
+  // under key (seed, 0), mapped to the open interval (0, 1).  The argmax of
+  // the noisy scores is a draw from softmax(logits / T).
+  __device__ __forceinline__ float pick_score(float v, int u, int pos) const {
+    if (!p.sample) return v;
+    const unsigned long long w =
+        dev::philox4x64_10_word((unsigned long long)(u >> 2), (unsigned long long)pos, p.seed, u & 3);
+    const double uu = ((double)(w >> 11) + 0.5) * 0x1p-53;
+    return (float)((double)v * p.inv_temp - log(-log(uu)));
+  }
+  __device__ __forceinline__ bool is_eos(int t) const {
+    for (int k = 0; k < p.n_eos; ++k)
+      if (t == p.eos_ids[k]) return true;
+    return false;
+  }
+
+  // Final RMSNorm + LM head + token pick (argmax of pick_score); or, on
+  // steps that pick no id, only the per-step fenced publish.  Returns false
+  // on abort; *tok_out gets the picked id (uniform across the grid).
+  __device__ __noinline__ bool stage_lm(bool pick, int step_row, unsigned tag, int pos,
+                                        int* tok_out) {
     stage = ST_LM;
     float best = -INFINITY;
     int bi = INT_MAX;
@@ -1542,8 +1561,9 @@ struct Consumer {
       for (int u = r.x + tid; u < r.y; u += kConsumerThreads) {
         const float v = row_result(pl, u - r.x) * rs;
         if (cap) cap[u] = v;
-        if (better(v, u, best, bi)) {
-          best = v;
+        const float sc = pick_score(v, u, pos);
+        if (better(sc, u, best, bi)) {
+          best = sc;
           bi = u;
         }
       }
@@ -1690,7 +1710,7 @@ struct Consumer {
       const bool pick = i >= p.lm_from;
       int next = 0;
       trace(0);
-      const bool lm_ok = stage_lm(pick, i - p.lm_from, epoch_of(p, i, p.L), &next);
+      const bool lm_ok = stage_lm(pick, i - p.lm_from, epoch_of(p, i, p.L), pos, &next);
       trace(3);
       w_stage = 0;
       if (!lm_ok) {
@@ -1699,7 +1719,7 @@ struct Consumer {
       }
       done = i + 1;
       if (pick && blockIdx.x == 0 && tid == 0) p.out_ids[i] = next;
-      if (pick && p.eos >= 0 && next == p.eos) break;
+      if (pick && is_eos(next)) break;
       if (p.forced && i + 1 < p.n_steps) tok = p.forced[i + 1];
       else tok = next;
     }

@@ -52,6 +52,8 @@ constexpr int kCombineBytesPerHead = 2304;
 // engine's scratch (no residual rows) adds the per-stage GEMV plans.
 constexpr int kMiscHead = 128;
 constexpr int kEngineMisc = 896;
+// Most ids of the set that ends a decode (end-of-sequence ids).
+constexpr int kMaxEosIds = 8;
 
 // Device status word block (library scratch, zeroed before each launch).
 struct DevStatus {
@@ -76,7 +78,14 @@ struct MonoParams {
   // model
   int L, d, H, KV, hd, F, V, G;
   float eps;
-  int max_seq, eos;
+  int max_seq;
+  int n_eos;               // a picked id equal to one of eos_ids[0 .. n_eos) ends the decode
+  int eos_ids[kMaxEosIds];
+  // token selection: greedy argmax (sample == 0), or the argmax of
+  // logit * inv_temp + Gumbel noise from Philox4x64-10 keyed by seed
+  int sample;
+  double inv_temp;
+  unsigned long long seed;
   // weights (device)
   const LayerW* layers;
   const __half* tok_emb;

@@ -131,3 +131,11 @@ def test_status_strings(lib):
     for s in range(9):
         assert lib.kie_status_str(s)
     assert lib.kie_status_str(99) == b"unknown status"
+
+
+def test_selection_setters_reject_null_context(lib):
+    assert lib.kie_set_sampling(None, 1.0, 5) == _kie.KIE_ERR_INVALID_ARG
+    ids = (ctypes.c_int32 * 2)(1, 2)
+    assert lib.kie_set_eos_ids(None, ids, 2) == _kie.KIE_ERR_INVALID_ARG
+    assert _kie.KIE_MAX_EOS_IDS == int(re.search(
+        r"#define KIE_MAX_EOS_IDS (\d+)", open(os.path.join(ROOT, "include", "kie.h")).read()).group(1))
