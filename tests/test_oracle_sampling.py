@@ -75,7 +75,7 @@ def test_gumbel_max_draws_softmax(T):
     logits = np.array([0.5, -1.0, 2.0, 0.0, 1.2, -0.3], dtype=np.float32)
     n = 40000
     u = S.uniforms(11, np.arange(n), logits.shape[0])
-    draws = np.argmax(logits.astype(np.float64) / T + S.gumbel(u), axis=1)
+    draws = np.argmax(S.perturbed_scores(logits, T, 11, np.arange(n)), axis=1)
     freq = np.bincount(draws, minlength=logits.shape[0])
     p = _softmax(logits.astype(np.float64) / T)
     chi2 = float(((freq - n * p) ** 2 / (n * p)).sum())
@@ -104,3 +104,73 @@ def test_limits():
 def test_score_margin():
     assert S.score_margin(np.array([1.0, 3.0, 2.5])) == pytest.approx(0.5)
     assert S.score_margin(np.array([1.0])) == float("inf")
+
+
+# ---- planted mistakes: each must make one of the pins above fail
+
+def _philox_early_key_bump(counter, key):
+    c0, c1, c2, c3 = (int(v) & MASK for v in counter)
+    k0, k1 = (int(v) & MASK for v in key)
+    for _ in range(10):
+        k0 = (k0 + S.PHILOX_W0) & MASK
+        k1 = (k1 + S.PHILOX_W1) & MASK
+        p0, p1 = S.PHILOX_M0 * c0, S.PHILOX_M1 * c2
+        c0, c1, c2, c3 = (p1 >> 64) ^ c1 ^ k0, p1 & MASK, (p0 >> 64) ^ c3 ^ k1, p0 & MASK
+    return [c0, c1, c2, c3]
+
+
+def _philox_many_swapped_multipliers(c0, c1, key0):
+    saved = S.PHILOX_M0, S.PHILOX_M1
+    try:
+        S.PHILOX_M0, S.PHILOX_M1 = saved[1], saved[0]
+        return _ORIG["philox4x64_10_many"](c0, c1, key0)
+    finally:
+        S.PHILOX_M0, S.PHILOX_M1 = saved
+
+
+def _uniforms_no_half(seed, position, n):
+    return _ORIG["uniforms"](seed, position, n) - 0.5 * 2.0 ** -53
+
+
+def _uniforms_swapped_counter(seed, position, n):
+    nb = (n + 3) // 4
+    pos = np.asarray(position, dtype=np.uint64)
+    words = S.philox4x64_10_many(pos[..., None], np.arange(nb, dtype=np.uint64), seed)
+    words = words.reshape(pos.shape + (4 * nb,))[..., :n]
+    return ((words >> np.uint64(11)).astype(np.float64) + 0.5) * 2.0 ** -53
+
+
+def _gumbel_wrong_sign(u):
+    return np.log(-np.log(u))
+
+
+def _scores_times_t(logits, temperature, seed, position):
+    lg = np.asarray(logits, dtype=np.float64)
+    return lg * float(temperature) + S.gumbel(S.uniforms(seed, position, lg.shape[0]))
+
+
+def _sample_id_argmin(logits, temperature, seed, position):
+    if temperature <= 0:
+        return int(np.argmin(np.asarray(logits)))
+    return int(np.argmax(S.perturbed_scores(logits, temperature, seed, position)))
+
+
+_ORIG = {k: getattr(S, k) for k in ("philox4x64_10_many", "uniforms")}
+
+MUTATIONS = [
+    ("philox4x64_10", _philox_early_key_bump,
+     lambda: test_philox_block_matches_numpy((0, 0, 0, 0), (0, 0))),
+    ("philox4x64_10_many", _philox_many_swapped_multipliers, test_vectorised_philox_matches_numpy),
+    ("uniforms", _uniforms_no_half, test_uniform_layout_and_range),
+    ("uniforms", _uniforms_swapped_counter, test_uniform_layout_and_range),
+    ("gumbel", _gumbel_wrong_sign, lambda: test_gumbel_max_draws_softmax(1.0)),
+    ("perturbed_scores", _scores_times_t, lambda: test_gumbel_max_draws_softmax(0.7)),
+    ("sample_id", _sample_id_argmin, test_limits),
+]
+
+
+@pytest.mark.parametrize("name,bad,pin", MUTATIONS, ids=[m[1].__name__ for m in MUTATIONS])
+def test_pin_catches_planted_mistake(monkeypatch, name, bad, pin):
+    monkeypatch.setattr(S, name, bad)
+    with pytest.raises(AssertionError):
+        pin()
