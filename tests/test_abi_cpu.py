@@ -139,3 +139,52 @@ def test_selection_setters_reject_null_context(lib):
     assert lib.kie_set_eos_ids(None, ids, 2) == _kie.KIE_ERR_INVALID_ARG
     assert _kie.KIE_MAX_EOS_IDS == int(re.search(
         r"#define KIE_MAX_EOS_IDS (\d+)", open(os.path.join(ROOT, "include", "kie.h")).read()).group(1))
+
+
+C_CLIENT = r"""
+#include <stdio.h>
+#include "kie.h"
+
+int main(void) {
+  kie_model_desc d;
+  int32_t b = -1, e = -1;
+  d.n_layers = 2; d.d_model = 256; d.n_heads = 4; d.n_kv_heads = 4; d.head_dim = 64;
+  d.ffn_dim = 768; d.vocab = 2048; d.rope_base = 10000.0f; d.rms_eps = 1e-5f;
+  d.max_seq = 48; d.eos_id = -1;
+  printf("check %d\n", (int)kie_check_desc(&d));
+  printf("kv %lu\n", (unsigned long)kie_kv_cache_bytes(&d));
+  printf("plan %d", (int)kie_plan_units(&d, 148, 4, 3, &b, &e));
+  printf(" %d %d\n", (int)b, (int)e);
+  printf("sampling %d\n", (int)kie_set_sampling(NULL, 1.0f, 7u));
+  printf("eos %d %d\n", (int)kie_set_eos_ids(NULL, NULL, 0), KIE_MAX_EOS_IDS);
+  printf("str %s\n", kie_status_str(KIE_ERR_CAPACITY));
+  return 0;
+}
+"""
+
+
+def test_header_is_plain_c_and_links(lib, tmp_path):
+    """A C99 program compiles against include/kie.h with warnings as errors,
+    links libkie.so and gets the same answers from the host-only calls."""
+    import shutil
+    import subprocess
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("no C compiler")
+    src = tmp_path / "client.c"
+    src.write_text(C_CLIENT)
+    exe = tmp_path / "client"
+    libdir = os.path.dirname(_kie.LIB_PATH)
+    subprocess.run([gcc, "-std=c99", "-Wall", "-Wextra", "-Werror", "-pedantic",
+                    "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe),
+                    "-L", libdir, "-l:libkie.so", f"-Wl,-rpath,{libdir}"], check=True)
+    out = subprocess.run([str(exe)], check=True, capture_output=True, text=True).stdout.split("\n")
+    s = synth.WORKLOADS["tiny-l2-d256"].shape
+    d = _desc(s, 48)
+    b, e = _kie.kie_plan_units(d, 148, 4, 3)
+    assert out[0] == "check 0"
+    assert out[1] == f"kv {2 * 2 * 4 * 48 * (64 + 8) * 2}"
+    assert out[2] == f"plan 0 {b} {e}"
+    assert out[3] == f"sampling {_kie.KIE_ERR_INVALID_ARG}"
+    assert out[4] == f"eos {_kie.KIE_ERR_INVALID_ARG} {_kie.KIE_MAX_EOS_IDS}"
+    assert out[5] == "str " + lib.kie_status_str(_kie.KIE_ERR_CAPACITY).decode()
