@@ -242,7 +242,8 @@ KIE_API kie_status kie_set_trace(kie_ctx *ctx, uint64_t *dev_buf, int32_t capaci
  * and t the 0-based position of the token whose logits are sampled.  A draw
  * depends only on (seed, t, logits), so kie_rewind followed by the same
  * decode reproduces it.  Applies to kie_prefill's first id, kie_decode and
- * kie_decode_forced.  Returns KIE_ERR_INVALID_ARG for a NULL ctx or a
+ * kie_decode_forced.  0 < temperature < 1e-20 is taken as 0 (greedy, the
+ * limit of the draw; the scaled logits would overflow fp32).  Returns KIE_ERR_INVALID_ARG for a NULL ctx or a
  * temperature that is negative, infinite or NaN.  Host only. */
 KIE_API kie_status kie_set_sampling(kie_ctx *ctx, float temperature, uint64_t seed);
 

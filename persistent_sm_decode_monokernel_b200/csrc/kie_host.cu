@@ -545,7 +545,9 @@ kie_status kie_set_sampling(kie_ctx* c, float temperature, uint64_t seed) {
   if (!c) return KIE_ERR_INVALID_ARG;
   if (!std::isfinite(temperature) || temperature < 0.f)
     return set_err(c, KIE_ERR_INVALID_ARG, "temperature must be finite and >= 0");
-  c->temperature = (double)temperature;
+  // Below 1e-20 the scaled logits would leave the fp32 range the kernel
+  // compares in, and the draw is the greedy pick anyway (T -> 0 limit).
+  c->temperature = temperature < 1e-20f ? 0.0 : (double)temperature;
   c->seed = seed;
   return KIE_OK;
 }

@@ -159,6 +159,10 @@ def test_seed_reproducible_rewind_and_temperature_zero(tiny):
     s.set_sampling(0.0, 11)             # back to greedy
     s.rewind(len(prompt))
     assert list(s.decode(20)) == greedy
+    for tiny_t in (1e-30, 1e-6):        # the T -> 0 limit is the greedy pick
+        s.set_sampling(tiny_t, 11)
+        s.rewind(len(prompt))
+        assert list(s.decode(20)) == greedy
     # the first id of a sampled prefill is drawn too (position P - 1)
     s.set_sampling(1e6, 3)
     g = s.prefill(prompt)
