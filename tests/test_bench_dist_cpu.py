@@ -64,3 +64,28 @@ def test_profiled_traffic_rejects_other_kernel(tmp_path, monkeypatch):
     w = synth.WORKLOADS["l28-d2560"]
     traffic, why = bench.profiled_traffic(w, 1024)
     assert traffic is None or traffic > 0
+
+
+def test_reference_arm_under_torchrun_prints_one_line_on_rank0():
+    """`bench.py --impl reference` launched like the GPU arm (two ranks):
+    rank 0 times the oracle and prints the contract's JSON line, the other
+    rank exits 0 without work."""
+    import json
+    import subprocess
+    import sys
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node", "2",
+           "--master-addr", "127.0.0.1", "--master-port", str(_free_port()),
+           os.path.join(bench.ROOT, "bench.py"), "--impl", "reference", "--workload", "tiny-l2-d256",
+           "--gpus", "2", "--steps", "2", "--warmup", "1", "--temperature", "0.9", "--seed", "5"]
+    r = subprocess.run(cmd, capture_output=True, text=True, timeout=600, cwd=bench.ROOT)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1, r.stdout
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["unit"] == "tok/s" and d["value"] > 0
+    assert d["n_gpus"] == 2 and d["steps"] == 2 and d["warmup"] == 1
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
+    assert d["cpu_baseline"]["value"] == d["value"]
+    assert d["e2e"] == {"value": d["value"], "unit": "tok/s", "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0}
+    assert d["config"]["token_selection"]["temperature"] == 0.9
