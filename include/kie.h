@@ -1,7 +1,7 @@
 /*
  * kie.h -- C ABI of the batch-1 decode monokernel library (libkie.so).
  *
- * The library runs batch-1 greedy autoregressive decode of a dense
+ * The library runs batch-1 autoregressive decode of a dense
  * decoder-only transformer as ONE persistent CUDA kernel per call: every
  * layer and every token step (RMSNorm, QKV GEMV, RoPE, KV-cache append,
  * attention over the cache, O projection, SwiGLU FFN GEMVs, LM-head GEMV,
