@@ -87,7 +87,8 @@ typedef enum {
   KIE_ERR_STATE = 5,        /* decode before prefill, or the context is failed */
   KIE_ERR_TIMEOUT = 6,      /* a device-side wait gave up (bounded spin) */
   KIE_ERR_PROTOCOL = 7,     /* a device-side consistency check failed */
-  KIE_ERR_TOO_LARGE = 8     /* larger than the fixed scratch of kie_gemv_f16_noalloc */
+  KIE_ERR_TOO_LARGE = 8,    /* larger than the fixed scratch of kie_gemv_f16_noalloc */
+  KIE_ERR_HOST_MEMORY = 9   /* a host allocation failed (no C++ exception crosses the ABI) */
 } kie_status;
 
 /* Model shape.  Supported: head_dim 64 or 128; n_heads a multiple of

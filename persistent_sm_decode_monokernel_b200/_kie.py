@@ -26,6 +26,7 @@ KIE_ERR_STATE = 5
 KIE_ERR_TIMEOUT = 6
 KIE_ERR_PROTOCOL = 7
 KIE_ERR_TOO_LARGE = 8
+KIE_ERR_HOST_MEMORY = 9
 
 KIE_NOALLOC_MAX_WEIGHT_BYTES = 16 * 1024 * 1024
 KIE_MAX_EOS_IDS = 8

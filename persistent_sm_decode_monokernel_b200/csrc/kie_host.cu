@@ -11,6 +11,7 @@
 #include <vector>
 
 #include "kie.h"
+#include "kie_guard.h"
 #include "kie_kernel.h"
 #include "kie_params.h"
 #include "kie_plan.h"
@@ -312,195 +313,203 @@ kie_status kie_check_desc(const kie_model_desc* d) {
 
 kie_status kie_plan_units(const kie_model_desc* d, int32_t grid, int32_t stage, int32_t cta,
                           int32_t* begin, int32_t* end) {
-  if (!d || !begin || !end) return KIE_ERR_INVALID_ARG;
-  kie_status s = kie_check_desc(d);
-  if (s != KIE_OK) return s;
-  if (grid < 1 || stage < 0 || stage >= kie::N_STAGES || cta < 0 || cta >= grid)
-    return KIE_ERR_INVALID_ARG;
-  const auto r = kie::partition(shape_of(*d), grid, stage);
-  *begin = r[cta].x;
-  *end = r[cta].y;
-  return KIE_OK;
+  return kie::no_throw([&]() -> kie_status {
+    if (!d || !begin || !end) return KIE_ERR_INVALID_ARG;
+    kie_status s = kie_check_desc(d);
+    if (s != KIE_OK) return s;
+    if (grid < 1 || stage < 0 || stage >= kie::N_STAGES || cta < 0 || cta >= grid)
+      return KIE_ERR_INVALID_ARG;
+    const auto r = kie::partition(shape_of(*d), grid, stage);
+    *begin = r[cta].x;
+    *end = r[cta].y;
+    return KIE_OK;
+  });
 }
 
 kie_status kie_create(const kie_model_desc* d, const kie_weights* w, void* kv_cache,
                       void* cuda_stream, kie_ctx** out) {
-  if (!out) return KIE_ERR_INVALID_ARG;
-  *out = nullptr;
-  if (!d || !w || !kv_cache || !w->layers || !w->tok_emb || !w->final_norm || !w->lm_head)
-    return KIE_ERR_INVALID_ARG;
-  kie_status s = kie_check_desc(d);
-  if (s != KIE_OK) return s;
-  if (!aligned16(kv_cache) || !aligned16(w->tok_emb) || !aligned16(w->final_norm) ||
-      !aligned16(w->lm_head))
-    return KIE_ERR_INVALID_ARG;
-  for (int l = 0; l < d->n_layers; ++l) {
-    const kie_layer_weights& lw = w->layers[l];
-    const void* ps[] = {lw.attn_norm, lw.wq, lw.wk, lw.wv, lw.wo, lw.ffn_norm, lw.w_gate, lw.w_up,
-                        lw.w_down};
-    for (const void* q : ps)
-      if (!q || !aligned16(q)) return KIE_ERR_INVALID_ARG;
-  }
-
-  kie_ctx* c = new kie_ctx();
-  c->desc = *d;
-  c->shape = shape_of(*d);
-  c->stream = static_cast<cudaStream_t>(cuda_stream);
-  c->tok_emb = static_cast<const __half*>(w->tok_emb);
-  c->final_norm = static_cast<const __half*>(w->final_norm);
-  c->lm_head = static_cast<const __half*>(w->lm_head);
-  c->kv = static_cast<__half*>(kv_cache);
-  for (int l = 0; l < d->n_layers; ++l) {
-    const kie_layer_weights& lw = w->layers[l];
-    c->hlayers.push_back(LayerW{static_cast<const __half*>(lw.attn_norm),
-                                static_cast<const __half*>(lw.wq), static_cast<const __half*>(lw.wk),
-                                static_cast<const __half*>(lw.wv), static_cast<const __half*>(lw.wo),
-                                static_cast<const __half*>(lw.ffn_norm),
-                                static_cast<const __half*>(lw.w_gate),
-                                static_cast<const __half*>(lw.w_up),
-                                static_cast<const __half*>(lw.w_down)});
-  }
-  auto fail = [&](kie_status st) {
-    free_all(c);
-    delete c;
-    return st;
-  };
-  auto cuda_bad = [&](cudaError_t e) { return e != cudaSuccess; };
-
-  if (cuda_bad(cudaGetDevice(&c->device))) return fail(KIE_ERR_CUDA);
-  int n_sm = 0, smem_optin = 0;
-  if (cuda_bad(cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, c->device)) ||
-      cuda_bad(cudaDeviceGetAttribute(&smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin,
-                                      c->device)))
-    return fail(KIE_ERR_CUDA);
-
-  // grid: one CTA per SM, but never more CTAs than units of the smallest stage
-  int grid = n_sm;
-  for (int st = 0; st < kie::N_STAGES; ++st)
-    grid = std::min(grid, kie::stage_units(c->shape, st));
-  c->grid = grid;
-  c->hranges.resize(kie::N_STAGES);
-  for (int st = 0; st < kie::N_STAGES; ++st) c->hranges[st] = kie::partition(c->shape, grid, st);
-  // largest chunk that leaves room for two in the ring: 64 KB, else 32 KB
-  bool planned = false;
-  for (int cb : {65536, 32768}) {
-    c->chunk_bytes = cb;
-    if ((planned = kie::plan_smem(c->shape, grid, cb, smem_optin, c->hranges, &c->sm,
-                                  &c->ring_bytes)))
-      break;
-  }
-  if (!planned) return fail(KIE_ERR_UNSUPPORTED);
-  c->smem = c->sm.total;
-  int per_sm = 0;
-  if (cuda_bad(kie::mono_configure(d->head_dim, c->smem, &per_sm))) return fail(KIE_ERR_CUDA);
-  if (per_sm < 1) return fail(KIE_ERR_UNSUPPORTED);
-  c->max_split = std::max(1, std::min(grid / d->n_kv_heads, kie::kMaxSplitCombine));
-
-  const int G = d->n_heads / d->n_kv_heads;
-  const size_t qd = (size_t)d->n_heads * d->head_dim, kvd = (size_t)d->n_kv_heads * d->head_dim;
-  c->tagged_words = 2 * (size_t)d->d_model + d->ffn_dim + qd + 2 * kvd + qd + 2 * (size_t)grid;
-  std::vector<int2> flat;
-  for (auto& v : c->hranges) flat.insert(flat.end(), v.begin(), v.end());
-  const size_t half = d->head_dim / 2;
-  std::vector<float2> rope((size_t)d->max_seq * half);
-  for (int t = 0; t < d->max_seq; ++t)
-    for (size_t i = 0; i < half; ++i) {
-      const double th = std::pow((double)d->rope_base, -2.0 * (double)i / d->head_dim);
-      const double a = (double)t * th;
-      rope[(size_t)t * half + i] = make_float2((float)std::cos(a), (float)std::sin(a));
+  return kie::no_throw([&]() -> kie_status {
+    if (!out) return KIE_ERR_INVALID_ARG;
+    *out = nullptr;
+    if (!d || !w || !kv_cache || !w->layers || !w->tok_emb || !w->final_norm || !w->lm_head)
+      return KIE_ERR_INVALID_ARG;
+    kie_status s = kie_check_desc(d);
+    if (s != KIE_OK) return s;
+    if (!aligned16(kv_cache) || !aligned16(w->tok_emb) || !aligned16(w->final_norm) ||
+        !aligned16(w->lm_head))
+      return KIE_ERR_INVALID_ARG;
+    for (int l = 0; l < d->n_layers; ++l) {
+      const kie_layer_weights& lw = w->layers[l];
+      const void* ps[] = {lw.attn_norm, lw.wq, lw.wk, lw.wv, lw.wo, lw.ffn_norm, lw.w_gate, lw.w_up,
+                          lw.w_down};
+      for (const void* q : ps)
+        if (!q || !aligned16(q)) return KIE_ERR_INVALID_ARG;
     }
 
-  if (cuda_bad(cudaMalloc(&c->dlayers, sizeof(LayerW) * d->n_layers)) ||
-      cuda_bad(cudaMalloc(&c->rope, sizeof(float2) * rope.size())) ||
-      cuda_bad(cudaMalloc(&c->ranges, sizeof(int2) * flat.size())) ||
-      cuda_bad(cudaMalloc(&c->tagged, 8 * c->tagged_words)) ||
-      cuda_bad(cudaMalloc(&c->partials, partial_bytes(c))) ||
-      cuda_bad(cudaMalloc(&c->d_ids, sizeof(int32_t) * d->max_seq)) ||
-      cuda_bad(cudaMalloc(&c->d_io, kStatusBytes + sizeof(int32_t) * d->max_seq)) ||
-      cuda_bad(cudaMalloc(&c->cta_stats, sizeof(unsigned long long) * kie::kStatsPerCta * grid)) ||
-      cuda_bad(cudaMallocHost(&c->h_io, kStatusBytes + sizeof(int32_t) * d->max_seq)) ||
-      cuda_bad(cudaEventCreate(&c->ev0)) || cuda_bad(cudaEventCreate(&c->ev1)))
-    return fail(KIE_ERR_CUDA);
-  unsigned long long* t = c->tagged;
-  c->x_attn = t;  t += d->d_model;
-  c->x_ffn = t;   t += d->d_model;
-  c->hbuf = t;    t += d->ffn_dim;
-  c->qbuf = t;    t += qd;
-  c->kvnew = t;   t += 2 * kvd;
-  c->obuf = t;    t += qd;
-  c->slots = t;
-  if (cuda_bad(cudaMemcpyAsync(c->dlayers, c->hlayers.data(), sizeof(LayerW) * d->n_layers,
-                               cudaMemcpyHostToDevice, c->stream)) ||
-      cuda_bad(cudaMemcpyAsync(c->rope, rope.data(), sizeof(float2) * rope.size(),
-                               cudaMemcpyHostToDevice, c->stream)) ||
-      cuda_bad(cudaMemcpyAsync(c->ranges, flat.data(), sizeof(int2) * flat.size(),
-                               cudaMemcpyHostToDevice, c->stream)) ||
-      cuda_bad(cudaMemsetAsync(c->tagged, 0, 8 * c->tagged_words, c->stream)) ||
-      cuda_bad(cudaMemsetAsync(c->partials, 0, partial_bytes(c), c->stream)) ||
-      cuda_bad(cudaMemsetAsync(c->cta_stats, 0, sizeof(unsigned long long) * kie::kStatsPerCta * grid,
-                               c->stream)) ||
-      cuda_bad(cudaStreamSynchronize(c->stream)))
-    return fail(KIE_ERR_CUDA);
+    kie_ctx* c = new kie_ctx();
+    c->desc = *d;
+    c->shape = shape_of(*d);
+    c->stream = static_cast<cudaStream_t>(cuda_stream);
+    c->tok_emb = static_cast<const __half*>(w->tok_emb);
+    c->final_norm = static_cast<const __half*>(w->final_norm);
+    c->lm_head = static_cast<const __half*>(w->lm_head);
+    c->kv = static_cast<__half*>(kv_cache);
+    for (int l = 0; l < d->n_layers; ++l) {
+      const kie_layer_weights& lw = w->layers[l];
+      c->hlayers.push_back(LayerW{static_cast<const __half*>(lw.attn_norm),
+                                  static_cast<const __half*>(lw.wq), static_cast<const __half*>(lw.wk),
+                                  static_cast<const __half*>(lw.wv), static_cast<const __half*>(lw.wo),
+                                  static_cast<const __half*>(lw.ffn_norm),
+                                  static_cast<const __half*>(lw.w_gate),
+                                  static_cast<const __half*>(lw.w_up),
+                                  static_cast<const __half*>(lw.w_down)});
+    }
+    auto fail = [&](kie_status st) {
+      free_all(c);
+      delete c;
+      return st;
+    };
+    auto cuda_bad = [&](cudaError_t e) { return e != cudaSuccess; };
 
-  if (repack(c) != KIE_OK) return fail(KIE_ERR_CUDA);
-  c->stats.grid = grid;
-  c->stats.ring_bytes = c->ring_bytes;
-  c->stats.chunk_bytes = c->chunk_bytes;
-  c->stats.smem_bytes = c->smem;
-  *out = c;
-  return KIE_OK;
+    if (cuda_bad(cudaGetDevice(&c->device))) return fail(KIE_ERR_CUDA);
+    int n_sm = 0, smem_optin = 0;
+    if (cuda_bad(cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, c->device)) ||
+        cuda_bad(cudaDeviceGetAttribute(&smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin,
+                                        c->device)))
+      return fail(KIE_ERR_CUDA);
+
+    // grid: one CTA per SM, but never more CTAs than units of the smallest stage
+    int grid = n_sm;
+    for (int st = 0; st < kie::N_STAGES; ++st)
+      grid = std::min(grid, kie::stage_units(c->shape, st));
+    c->grid = grid;
+    c->hranges.resize(kie::N_STAGES);
+    for (int st = 0; st < kie::N_STAGES; ++st) c->hranges[st] = kie::partition(c->shape, grid, st);
+    // largest chunk that leaves room for two in the ring: 64 KB, else 32 KB
+    bool planned = false;
+    for (int cb : {65536, 32768}) {
+      c->chunk_bytes = cb;
+      if ((planned = kie::plan_smem(c->shape, grid, cb, smem_optin, c->hranges, &c->sm,
+                                    &c->ring_bytes)))
+        break;
+    }
+    if (!planned) return fail(KIE_ERR_UNSUPPORTED);
+    c->smem = c->sm.total;
+    int per_sm = 0;
+    if (cuda_bad(kie::mono_configure(d->head_dim, c->smem, &per_sm))) return fail(KIE_ERR_CUDA);
+    if (per_sm < 1) return fail(KIE_ERR_UNSUPPORTED);
+    c->max_split = std::max(1, std::min(grid / d->n_kv_heads, kie::kMaxSplitCombine));
+
+    const int G = d->n_heads / d->n_kv_heads;
+    const size_t qd = (size_t)d->n_heads * d->head_dim, kvd = (size_t)d->n_kv_heads * d->head_dim;
+    c->tagged_words = 2 * (size_t)d->d_model + d->ffn_dim + qd + 2 * kvd + qd + 2 * (size_t)grid;
+    std::vector<int2> flat;
+    for (auto& v : c->hranges) flat.insert(flat.end(), v.begin(), v.end());
+    const size_t half = d->head_dim / 2;
+    std::vector<float2> rope((size_t)d->max_seq * half);
+    for (int t = 0; t < d->max_seq; ++t)
+      for (size_t i = 0; i < half; ++i) {
+        const double th = std::pow((double)d->rope_base, -2.0 * (double)i / d->head_dim);
+        const double a = (double)t * th;
+        rope[(size_t)t * half + i] = make_float2((float)std::cos(a), (float)std::sin(a));
+      }
+
+    if (cuda_bad(cudaMalloc(&c->dlayers, sizeof(LayerW) * d->n_layers)) ||
+        cuda_bad(cudaMalloc(&c->rope, sizeof(float2) * rope.size())) ||
+        cuda_bad(cudaMalloc(&c->ranges, sizeof(int2) * flat.size())) ||
+        cuda_bad(cudaMalloc(&c->tagged, 8 * c->tagged_words)) ||
+        cuda_bad(cudaMalloc(&c->partials, partial_bytes(c))) ||
+        cuda_bad(cudaMalloc(&c->d_ids, sizeof(int32_t) * d->max_seq)) ||
+        cuda_bad(cudaMalloc(&c->d_io, kStatusBytes + sizeof(int32_t) * d->max_seq)) ||
+        cuda_bad(cudaMalloc(&c->cta_stats, sizeof(unsigned long long) * kie::kStatsPerCta * grid)) ||
+        cuda_bad(cudaMallocHost(&c->h_io, kStatusBytes + sizeof(int32_t) * d->max_seq)) ||
+        cuda_bad(cudaEventCreate(&c->ev0)) || cuda_bad(cudaEventCreate(&c->ev1)))
+      return fail(KIE_ERR_CUDA);
+    unsigned long long* t = c->tagged;
+    c->x_attn = t;  t += d->d_model;
+    c->x_ffn = t;   t += d->d_model;
+    c->hbuf = t;    t += d->ffn_dim;
+    c->qbuf = t;    t += qd;
+    c->kvnew = t;   t += 2 * kvd;
+    c->obuf = t;    t += qd;
+    c->slots = t;
+    if (cuda_bad(cudaMemcpyAsync(c->dlayers, c->hlayers.data(), sizeof(LayerW) * d->n_layers,
+                                 cudaMemcpyHostToDevice, c->stream)) ||
+        cuda_bad(cudaMemcpyAsync(c->rope, rope.data(), sizeof(float2) * rope.size(),
+                                 cudaMemcpyHostToDevice, c->stream)) ||
+        cuda_bad(cudaMemcpyAsync(c->ranges, flat.data(), sizeof(int2) * flat.size(),
+                                 cudaMemcpyHostToDevice, c->stream)) ||
+        cuda_bad(cudaMemsetAsync(c->tagged, 0, 8 * c->tagged_words, c->stream)) ||
+        cuda_bad(cudaMemsetAsync(c->partials, 0, partial_bytes(c), c->stream)) ||
+        cuda_bad(cudaMemsetAsync(c->cta_stats, 0, sizeof(unsigned long long) * kie::kStatsPerCta * grid,
+                                 c->stream)) ||
+        cuda_bad(cudaStreamSynchronize(c->stream)))
+      return fail(KIE_ERR_CUDA);
+
+    if (repack(c) != KIE_OK) return fail(KIE_ERR_CUDA);
+    c->stats.grid = grid;
+    c->stats.ring_bytes = c->ring_bytes;
+    c->stats.chunk_bytes = c->chunk_bytes;
+    c->stats.smem_bytes = c->smem;
+    *out = c;
+    return KIE_OK;
+  });
 }
 
 kie_status kie_prefill(kie_ctx* c, const int32_t* ids, int32_t n, int32_t* first_id) {
-  kie_status s = usable(c);
-  if (s != KIE_OK) return s;
-  if (!ids || n < 1) return set_err(c, KIE_ERR_INVALID_ARG, "prefill needs n >= 1 ids");
-  if (n > c->desc.max_seq) return set_err(c, KIE_ERR_CAPACITY, "prompt longer than max_seq");
-  for (int i = 0; i < n; ++i)
-    if (ids[i] < 0 || ids[i] >= c->desc.vocab)
-      return set_err(c, KIE_ERR_INVALID_ARG, "prompt id out of range");
-  c->primed = false;
-  int done = 0;
-  s = launch(c, n, 0, ids, true, 0, n - 1, &done);
-  if (s != KIE_OK) return s;
-  const int32_t g0 = reinterpret_cast<const int32_t*>(c->h_io + kStatusBytes)[n - 1];
-  c->fed.assign(ids, ids + n);
-  c->pos = n;
-  c->next_tok = g0;
-  c->primed = true;
-  if (first_id) *first_id = g0;
-  c->stats.pos = c->pos;
-  return KIE_OK;
+  return kie::no_throw([&]() -> kie_status {
+    kie_status s = usable(c);
+    if (s != KIE_OK) return s;
+    if (!ids || n < 1) return set_err(c, KIE_ERR_INVALID_ARG, "prefill needs n >= 1 ids");
+    if (n > c->desc.max_seq) return set_err(c, KIE_ERR_CAPACITY, "prompt longer than max_seq");
+    for (int i = 0; i < n; ++i)
+      if (ids[i] < 0 || ids[i] >= c->desc.vocab)
+        return set_err(c, KIE_ERR_INVALID_ARG, "prompt id out of range");
+    c->primed = false;
+    int done = 0;
+    s = launch(c, n, 0, ids, true, 0, n - 1, &done);
+    if (s != KIE_OK) return s;
+    const int32_t g0 = reinterpret_cast<const int32_t*>(c->h_io + kStatusBytes)[n - 1];
+    c->fed.assign(ids, ids + n);
+    c->pos = n;
+    c->next_tok = g0;
+    c->primed = true;
+    if (first_id) *first_id = g0;
+    c->stats.pos = c->pos;
+    return KIE_OK;
+  });
 }
 
 static kie_status decode_impl(kie_ctx* c, int32_t n, const int32_t* forced_ids,
                               int32_t* out_ids, int32_t* n_out) {
-  kie_status s = usable(c);
-  if (s != KIE_OK) return s;
-  if (n_out) *n_out = 0;
-  if (n < 0) return set_err(c, KIE_ERR_INVALID_ARG, "n_steps < 0");
-  if (!c->primed) return set_err(c, KIE_ERR_STATE, "decode before prefill");
-  if (n == 0) return KIE_OK;
-  if (!out_ids && !forced_ids) return set_err(c, KIE_ERR_INVALID_ARG, "out_ids is NULL");
-  if ((long long)c->pos + n > c->desc.max_seq)
-    return set_err(c, KIE_ERR_CAPACITY, "decode would pass max_seq positions");
-  if (forced_ids)
-    for (int i = 0; i < n; ++i)
-      if (forced_ids[i] < 0 || forced_ids[i] >= c->desc.vocab)
-        return set_err(c, KIE_ERR_INVALID_ARG, "forced id out of range");
-  int done = 0;
-  s = launch(c, n, c->pos, forced_ids, forced_ids != nullptr, c->next_tok, 0, &done);
-  if (s != KIE_OK) return s;
-  const int32_t* picks = reinterpret_cast<const int32_t*>(c->h_io + kStatusBytes);
-  if (out_ids) std::memcpy(out_ids, picks, sizeof(int32_t) * done);
-  for (int i = 0; i < done; ++i) {
-    c->fed.push_back(forced_ids ? forced_ids[i] : (i == 0 ? c->next_tok : picks[i - 1]));
-  }
-  c->pos += done;
-  if (done > 0) c->next_tok = picks[done - 1];
-  if (n_out) *n_out = done;
-  c->stats.pos = c->pos;
-  return KIE_OK;
+  return kie::no_throw([&]() -> kie_status {
+    kie_status s = usable(c);
+    if (s != KIE_OK) return s;
+    if (n_out) *n_out = 0;
+    if (n < 0) return set_err(c, KIE_ERR_INVALID_ARG, "n_steps < 0");
+    if (!c->primed) return set_err(c, KIE_ERR_STATE, "decode before prefill");
+    if (n == 0) return KIE_OK;
+    if (!out_ids && !forced_ids) return set_err(c, KIE_ERR_INVALID_ARG, "out_ids is NULL");
+    if ((long long)c->pos + n > c->desc.max_seq)
+      return set_err(c, KIE_ERR_CAPACITY, "decode would pass max_seq positions");
+    if (forced_ids)
+      for (int i = 0; i < n; ++i)
+        if (forced_ids[i] < 0 || forced_ids[i] >= c->desc.vocab)
+          return set_err(c, KIE_ERR_INVALID_ARG, "forced id out of range");
+    int done = 0;
+    s = launch(c, n, c->pos, forced_ids, forced_ids != nullptr, c->next_tok, 0, &done);
+    if (s != KIE_OK) return s;
+    const int32_t* picks = reinterpret_cast<const int32_t*>(c->h_io + kStatusBytes);
+    if (out_ids) std::memcpy(out_ids, picks, sizeof(int32_t) * done);
+    for (int i = 0; i < done; ++i) {
+      c->fed.push_back(forced_ids ? forced_ids[i] : (i == 0 ? c->next_tok : picks[i - 1]));
+    }
+    c->pos += done;
+    if (done > 0) c->next_tok = picks[done - 1];
+    if (n_out) *n_out = done;
+    c->stats.pos = c->pos;
+    return KIE_OK;
+  });
 }
 
 kie_status kie_decode(kie_ctx* c, int32_t n, int32_t* out_ids, int32_t* n_out) {
@@ -508,13 +517,15 @@ kie_status kie_decode(kie_ctx* c, int32_t n, int32_t* out_ids, int32_t* n_out) {
 }
 
 kie_status kie_decode_forced(kie_ctx* c, const int32_t* ids, int32_t n, int32_t* out_ids) {
-  if (c && n > 0 && !ids) return set_err(c, KIE_ERR_INVALID_ARG, "ids is NULL");
-  std::vector<int32_t> tmp;
-  if (!out_ids && n > 0) {
-    tmp.resize(n);
-    out_ids = tmp.data();
-  }
-  return decode_impl(c, n, ids, out_ids, nullptr);
+  return kie::no_throw([&]() -> kie_status {
+    if (c && n > 0 && !ids) return set_err(c, KIE_ERR_INVALID_ARG, "ids is NULL");
+    std::vector<int32_t> tmp;
+    if (!out_ids && n > 0) {
+      tmp.resize(n);
+      out_ids = tmp.data();
+    }
+    return decode_impl(c, n, ids, out_ids, nullptr);
+  });
 }
 
 kie_status kie_rewind(kie_ctx* c, int32_t pos) {
@@ -553,144 +564,148 @@ kie_status kie_set_sampling(kie_ctx* c, float temperature, uint64_t seed) {
 }
 
 kie_status kie_set_eos_ids(kie_ctx* c, const int32_t* ids, int32_t n) {
-  if (!c) return KIE_ERR_INVALID_ARG;
-  if (n < 0 || n > KIE_MAX_EOS_IDS) return set_err(c, KIE_ERR_INVALID_ARG, "eos id count out of range");
-  if (n > 0 && !ids) return set_err(c, KIE_ERR_INVALID_ARG, "ids is NULL");
-  for (int i = 0; i < n; ++i)
-    if (ids[i] < 0 || ids[i] >= c->desc.vocab)
-      return set_err(c, KIE_ERR_INVALID_ARG, "eos id out of range");
-  c->eos_ids.assign(ids, ids + n);
-  return KIE_OK;
+  return kie::no_throw([&]() -> kie_status {
+    if (!c) return KIE_ERR_INVALID_ARG;
+    if (n < 0 || n > KIE_MAX_EOS_IDS) return set_err(c, KIE_ERR_INVALID_ARG, "eos id count out of range");
+    if (n > 0 && !ids) return set_err(c, KIE_ERR_INVALID_ARG, "ids is NULL");
+    for (int i = 0; i < n; ++i)
+      if (ids[i] < 0 || ids[i] >= c->desc.vocab)
+        return set_err(c, KIE_ERR_INVALID_ARG, "eos id out of range");
+    c->eos_ids.assign(ids, ids + n);
+    return KIE_OK;
+  });
 }
 
 kie_status kie_gemv_f16(const void* W, const float* x, float* y, int32_t N, int32_t K,
                         int32_t iters, int32_t mode, int32_t chunk_bytes, void* stream,
                         float* ms_out, double* stats_out) {
-  if (!W || !x || (!y && mode == 1) || N < 1 || K < 256 || K % 256 || iters < 1 ||
-      (mode != 0 && mode != 1) || chunk_bytes < 8192 || chunk_bytes % 512)
-    return KIE_ERR_INVALID_ARG;
-  if (!aligned16(W) || !aligned16(x)) return KIE_ERR_INVALID_ARG;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  int dev = 0, n_sm = 0, smem_optin = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess ||
-      cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
-      cudaDeviceGetAttribute(&smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) !=
-          cudaSuccess)
-    return KIE_ERR_CUDA;
-  const int grid = std::min(n_sm, N);
-  // one layer whose four layer stages own no rows; the LM-head stage is W
-  kie::Shape sh{1, K, 1, 1, 64, 256, N};
-  std::vector<std::vector<int2>> ranges(kie::N_STAGES, std::vector<int2>(grid, make_int2(0, 0)));
-  ranges[kie::ST_LM] = kie::partition(sh, grid, kie::ST_LM);
-  std::vector<int2> flat;
-  for (auto& v : ranges) flat.insert(flat.end(), v.begin(), v.end());
-  int maxrows = 0;
-  std::vector<unsigned long long> off(grid);
-  size_t total = 0;
-  for (int c = 0; c < grid; ++c) {
-    maxrows = std::max(maxrows, ranges[kie::ST_LM][c].y - ranges[kie::ST_LM][c].x);
-    off[c] = total;
-    total += (size_t)(ranges[kie::ST_LM][c].y - ranges[kie::ST_LM][c].x) * K * 2;
-  }
-  kie::SmemLayout L{};
-  L.xs_bytes = (K * 4 + 127) / 128 * 128;
-  L.rowacc_rows = maxrows;
-  L.resid_rows = 0;
-  const int fixed = 256 + L.xs_bytes + (maxrows * 4 + 127) / 128 * 128 + kie::kEngineMisc;
-  const int ring = (smem_optin - fixed) / 512 * 512;
-  if (ring < 2 * chunk_bytes) return KIE_ERR_UNSUPPORTED;
-  L.ring_off = 0;
-  L.bar_off = ring;
-  L.xs_off = L.bar_off + 256;
-  L.rowacc_off = L.xs_off + L.xs_bytes;
-  L.misc_off = L.rowacc_off + (maxrows * 4 + 127) / 128 * 128;
-  L.total = L.misc_off + kie::kEngineMisc;
-
-  int2* d_ranges = nullptr;
-  DevStatus* d_status = nullptr;
-  unsigned long long* d_stats = nullptr;
-  unsigned long long* d_off = nullptr;
-  unsigned char* d_packed = nullptr;
-  LayerW* d_layer = nullptr;
-  cudaEvent_t e0 = nullptr, e1 = nullptr;
-  kie_status ret = KIE_OK;
-  if (cudaMalloc(&d_ranges, sizeof(int2) * flat.size()) != cudaSuccess ||
-      cudaMalloc(&d_status, sizeof(DevStatus)) != cudaSuccess ||
-      cudaMalloc(&d_stats, sizeof(unsigned long long) * kie::kStatsPerCta * grid) != cudaSuccess ||
-      cudaMalloc(&d_off, sizeof(unsigned long long) * grid) != cudaSuccess ||
-      cudaMalloc(&d_packed, total) != cudaSuccess ||
-      cudaMalloc(&d_layer, sizeof(LayerW)) != cudaSuccess ||
-      cudaEventCreate(&e0) != cudaSuccess || cudaEventCreate(&e1) != cudaSuccess) {
-    ret = KIE_ERR_CUDA;
-  }
-  MonoParams p{};
-  if (ret == KIE_OK) {
-    p.L = 1;
-    p.d = K;
-    p.H = 1;
-    p.KV = 1;
-    p.hd = 64;
-    p.F = 256;
-    p.V = N;
-    p.G = 1;
-    p.layers = d_layer;
-    p.lm_head = static_cast<const __half*>(W);
-    p.ranges = d_ranges;
-    p.grid = grid;
-    p.ring_bytes = ring;
-    p.chunk_bytes = chunk_bytes;
-    p.packed = d_packed;
-    p.packed_off = d_off;
-    p.sm = L;
-    p.status = d_status;
-    p.cta_stats = d_stats;
-    p.timeout_ns = 2000000000LL;
-    p.poll_ns = 128;
-    p.fault_cta = -1;
-    if (cudaMemcpyAsync(d_ranges, flat.data(), sizeof(int2) * flat.size(),
-                        cudaMemcpyHostToDevice, st) != cudaSuccess ||
-        cudaMemcpyAsync(d_off, off.data(), sizeof(unsigned long long) * grid,
-                        cudaMemcpyHostToDevice, st) != cudaSuccess ||
-        cudaMemsetAsync(d_status, 0, sizeof(DevStatus), st) != cudaSuccess ||
-        cudaMemsetAsync(d_stats, 0, sizeof(unsigned long long) * kie::kStatsPerCta * grid, st) !=
-            cudaSuccess ||
-        cudaMemsetAsync(d_layer, 0, sizeof(LayerW), st) != cudaSuccess ||
-        kie::repack_launch(p, d_packed, st) != cudaSuccess ||
-        kie::gemv_configure(L.total) != cudaSuccess || cudaEventRecord(e0, st) != cudaSuccess ||
-        kie::gemv_launch(p, mode, x, y, iters, grid, L.total, st) != cudaSuccess ||
-        cudaEventRecord(e1, st) != cudaSuccess || cudaStreamSynchronize(st) != cudaSuccess)
-      ret = KIE_ERR_CUDA;
-  }
-  if (ret == KIE_OK) {
-    float ms = 0.f;
-    cudaEventElapsedTime(&ms, e0, e1);
-    if (ms_out) *ms_out = ms;
-    DevStatus hs{};
-    cudaMemcpy(&hs, d_status, sizeof hs, cudaMemcpyDeviceToHost);
-    if (hs.code != kie::DEV_OK) ret = hs.code == kie::DEV_TIMEOUT ? KIE_ERR_TIMEOUT : KIE_ERR_PROTOCOL;
-    if (stats_out) {
-      std::vector<unsigned long long> h((size_t)kie::kStatsPerCta * grid);
-      cudaMemcpy(h.data(), d_stats, sizeof(unsigned long long) * h.size(), cudaMemcpyDeviceToHost);
-      double stream = 0, prod = 0;
-      for (int c = 0; c < grid; ++c) {
-        stream += (double)h[(size_t)kie::kStatsPerCta * c + 2];
-        prod += (double)h[(size_t)kie::kStatsPerCta * c + 3];
-      }
-      stats_out[0] = stream / grid;
-      stats_out[1] = prod / grid;
-      stats_out[2] = grid;
-      stats_out[3] = ring;
+  return kie::no_throw([&]() -> kie_status {
+    if (!W || !x || (!y && mode == 1) || N < 1 || K < 256 || K % 256 || iters < 1 ||
+        (mode != 0 && mode != 1) || chunk_bytes < 8192 || chunk_bytes % 512)
+      return KIE_ERR_INVALID_ARG;
+    if (!aligned16(W) || !aligned16(x)) return KIE_ERR_INVALID_ARG;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    int dev = 0, n_sm = 0, smem_optin = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) !=
+            cudaSuccess)
+      return KIE_ERR_CUDA;
+    const int grid = std::min(n_sm, N);
+    // one layer whose four layer stages own no rows; the LM-head stage is W
+    kie::Shape sh{1, K, 1, 1, 64, 256, N};
+    std::vector<std::vector<int2>> ranges(kie::N_STAGES, std::vector<int2>(grid, make_int2(0, 0)));
+    ranges[kie::ST_LM] = kie::partition(sh, grid, kie::ST_LM);
+    std::vector<int2> flat;
+    for (auto& v : ranges) flat.insert(flat.end(), v.begin(), v.end());
+    int maxrows = 0;
+    std::vector<unsigned long long> off(grid);
+    size_t total = 0;
+    for (int c = 0; c < grid; ++c) {
+      maxrows = std::max(maxrows, ranges[kie::ST_LM][c].y - ranges[kie::ST_LM][c].x);
+      off[c] = total;
+      total += (size_t)(ranges[kie::ST_LM][c].y - ranges[kie::ST_LM][c].x) * K * 2;
     }
-  }
-  cudaFree(d_ranges);
-  cudaFree(d_status);
-  cudaFree(d_stats);
-  cudaFree(d_off);
-  cudaFree(d_packed);
-  cudaFree(d_layer);
-  if (e0) cudaEventDestroy(e0);
-  if (e1) cudaEventDestroy(e1);
-  return ret;
+    kie::SmemLayout L{};
+    L.xs_bytes = (K * 4 + 127) / 128 * 128;
+    L.rowacc_rows = maxrows;
+    L.resid_rows = 0;
+    const int fixed = 256 + L.xs_bytes + (maxrows * 4 + 127) / 128 * 128 + kie::kEngineMisc;
+    const int ring = (smem_optin - fixed) / 512 * 512;
+    if (ring < 2 * chunk_bytes) return KIE_ERR_UNSUPPORTED;
+    L.ring_off = 0;
+    L.bar_off = ring;
+    L.xs_off = L.bar_off + 256;
+    L.rowacc_off = L.xs_off + L.xs_bytes;
+    L.misc_off = L.rowacc_off + (maxrows * 4 + 127) / 128 * 128;
+    L.total = L.misc_off + kie::kEngineMisc;
+
+    int2* d_ranges = nullptr;
+    DevStatus* d_status = nullptr;
+    unsigned long long* d_stats = nullptr;
+    unsigned long long* d_off = nullptr;
+    unsigned char* d_packed = nullptr;
+    LayerW* d_layer = nullptr;
+    cudaEvent_t e0 = nullptr, e1 = nullptr;
+    kie_status ret = KIE_OK;
+    if (cudaMalloc(&d_ranges, sizeof(int2) * flat.size()) != cudaSuccess ||
+        cudaMalloc(&d_status, sizeof(DevStatus)) != cudaSuccess ||
+        cudaMalloc(&d_stats, sizeof(unsigned long long) * kie::kStatsPerCta * grid) != cudaSuccess ||
+        cudaMalloc(&d_off, sizeof(unsigned long long) * grid) != cudaSuccess ||
+        cudaMalloc(&d_packed, total) != cudaSuccess ||
+        cudaMalloc(&d_layer, sizeof(LayerW)) != cudaSuccess ||
+        cudaEventCreate(&e0) != cudaSuccess || cudaEventCreate(&e1) != cudaSuccess) {
+      ret = KIE_ERR_CUDA;
+    }
+    MonoParams p{};
+    if (ret == KIE_OK) {
+      p.L = 1;
+      p.d = K;
+      p.H = 1;
+      p.KV = 1;
+      p.hd = 64;
+      p.F = 256;
+      p.V = N;
+      p.G = 1;
+      p.layers = d_layer;
+      p.lm_head = static_cast<const __half*>(W);
+      p.ranges = d_ranges;
+      p.grid = grid;
+      p.ring_bytes = ring;
+      p.chunk_bytes = chunk_bytes;
+      p.packed = d_packed;
+      p.packed_off = d_off;
+      p.sm = L;
+      p.status = d_status;
+      p.cta_stats = d_stats;
+      p.timeout_ns = 2000000000LL;
+      p.poll_ns = 128;
+      p.fault_cta = -1;
+      if (cudaMemcpyAsync(d_ranges, flat.data(), sizeof(int2) * flat.size(),
+                          cudaMemcpyHostToDevice, st) != cudaSuccess ||
+          cudaMemcpyAsync(d_off, off.data(), sizeof(unsigned long long) * grid,
+                          cudaMemcpyHostToDevice, st) != cudaSuccess ||
+          cudaMemsetAsync(d_status, 0, sizeof(DevStatus), st) != cudaSuccess ||
+          cudaMemsetAsync(d_stats, 0, sizeof(unsigned long long) * kie::kStatsPerCta * grid, st) !=
+              cudaSuccess ||
+          cudaMemsetAsync(d_layer, 0, sizeof(LayerW), st) != cudaSuccess ||
+          kie::repack_launch(p, d_packed, st) != cudaSuccess ||
+          kie::gemv_configure(L.total) != cudaSuccess || cudaEventRecord(e0, st) != cudaSuccess ||
+          kie::gemv_launch(p, mode, x, y, iters, grid, L.total, st) != cudaSuccess ||
+          cudaEventRecord(e1, st) != cudaSuccess || cudaStreamSynchronize(st) != cudaSuccess)
+        ret = KIE_ERR_CUDA;
+    }
+    if (ret == KIE_OK) {
+      float ms = 0.f;
+      cudaEventElapsedTime(&ms, e0, e1);
+      if (ms_out) *ms_out = ms;
+      DevStatus hs{};
+      cudaMemcpy(&hs, d_status, sizeof hs, cudaMemcpyDeviceToHost);
+      if (hs.code != kie::DEV_OK) ret = hs.code == kie::DEV_TIMEOUT ? KIE_ERR_TIMEOUT : KIE_ERR_PROTOCOL;
+      if (stats_out) {
+        std::vector<unsigned long long> h((size_t)kie::kStatsPerCta * grid);
+        cudaMemcpy(h.data(), d_stats, sizeof(unsigned long long) * h.size(), cudaMemcpyDeviceToHost);
+        double stream = 0, prod = 0;
+        for (int c = 0; c < grid; ++c) {
+          stream += (double)h[(size_t)kie::kStatsPerCta * c + 2];
+          prod += (double)h[(size_t)kie::kStatsPerCta * c + 3];
+        }
+        stats_out[0] = stream / grid;
+        stats_out[1] = prod / grid;
+        stats_out[2] = grid;
+        stats_out[3] = ring;
+      }
+    }
+    cudaFree(d_ranges);
+    cudaFree(d_status);
+    cudaFree(d_stats);
+    cudaFree(d_off);
+    cudaFree(d_packed);
+    cudaFree(d_layer);
+    if (e0) cudaEventDestroy(e0);
+    if (e1) cudaEventDestroy(e1);
+    return ret;
+  });
 }
 
 kie_status kie_set_trace(kie_ctx* c, uint64_t* dev_buf, int32_t capacity, int32_t cta) {
@@ -705,56 +720,58 @@ kie_status kie_set_trace(kie_ctx* c, uint64_t* dev_buf, int32_t capacity, int32_
 }
 
 kie_status kie_set_option(kie_ctx* c, kie_option opt, int64_t v) {
-  if (!c) return KIE_ERR_INVALID_ARG;
-  switch (opt) {
-    case KIE_OPT_TIMEOUT_NS:
-      if (v < 1000) return KIE_ERR_INVALID_ARG;
-      c->timeout_ns = v;
-      return KIE_OK;
-    case KIE_OPT_CHUNK_BYTES: {
-      if (c->failed) return set_err(c, KIE_ERR_STATE, "context failed earlier; destroy it");
-      if (v < 8192 || v % 512 || v > (1 << 20)) return KIE_ERR_INVALID_ARG;
-      int smem_optin = 0;
-      if (cudaDeviceGetAttribute(&smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin,
-                                 c->device) != cudaSuccess)
-        return set_err(c, KIE_ERR_CUDA, "device attribute query failed");
-      kie::SmemLayout sm{};
-      int ring = 0;
-      if (!kie::plan_smem(c->shape, c->grid, (int)v, smem_optin, c->hranges, &sm, &ring))
-        return set_err(c, KIE_ERR_UNSUPPORTED, "chunk size does not fit shared memory");
-      int per_sm = 0;
-      if (kie::mono_configure(c->desc.head_dim, sm.total, &per_sm) != cudaSuccess || per_sm < 1)
-        return set_err(c, KIE_ERR_UNSUPPORTED, "kernel does not fit with this chunk size");
-      c->chunk_bytes = (int)v;
-      c->sm = sm;
-      c->ring_bytes = ring;
-      c->smem = sm.total;
-      c->stats.ring_bytes = ring;
-      c->stats.chunk_bytes = (int)v;
-      c->stats.smem_bytes = sm.total;
-      return repack(c);
+  return kie::no_throw([&]() -> kie_status {
+    if (!c) return KIE_ERR_INVALID_ARG;
+    switch (opt) {
+      case KIE_OPT_TIMEOUT_NS:
+        if (v < 1000) return KIE_ERR_INVALID_ARG;
+        c->timeout_ns = v;
+        return KIE_OK;
+      case KIE_OPT_CHUNK_BYTES: {
+        if (c->failed) return set_err(c, KIE_ERR_STATE, "context failed earlier; destroy it");
+        if (v < 8192 || v % 512 || v > (1 << 20)) return KIE_ERR_INVALID_ARG;
+        int smem_optin = 0;
+        if (cudaDeviceGetAttribute(&smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin,
+                                   c->device) != cudaSuccess)
+          return set_err(c, KIE_ERR_CUDA, "device attribute query failed");
+        kie::SmemLayout sm{};
+        int ring = 0;
+        if (!kie::plan_smem(c->shape, c->grid, (int)v, smem_optin, c->hranges, &sm, &ring))
+          return set_err(c, KIE_ERR_UNSUPPORTED, "chunk size does not fit shared memory");
+        int per_sm = 0;
+        if (kie::mono_configure(c->desc.head_dim, sm.total, &per_sm) != cudaSuccess || per_sm < 1)
+          return set_err(c, KIE_ERR_UNSUPPORTED, "kernel does not fit with this chunk size");
+        c->chunk_bytes = (int)v;
+        c->sm = sm;
+        c->ring_bytes = ring;
+        c->smem = sm.total;
+        c->stats.ring_bytes = ring;
+        c->stats.chunk_bytes = (int)v;
+        c->stats.smem_bytes = sm.total;
+        return repack(c);
+      }
+      case KIE_OPT_MIN_SPLIT_LEN:
+        if (v < 1 || v > (1 << 20)) return KIE_ERR_INVALID_ARG;
+        c->min_split_len = (int)v;
+        return KIE_OK;
+      case KIE_OPT_TRACE_CLOCK:
+        c->trace_clock = v ? 1 : 0;
+        return KIE_OK;
+      case KIE_OPT_POLL_BACKOFF_NS:
+        if (v < 0 || v > 100000) return KIE_ERR_INVALID_ARG;
+        c->poll_ns = (unsigned)v;
+        return KIE_OK;
+      case KIE_OPT_L2_PREFETCH_BYTES:
+        if (v < 0 || v % 512 || v > (16 << 20)) return KIE_ERR_INVALID_ARG;
+        c->l2_prefetch = v;
+        return KIE_OK;
+      case KIE_OPT_FAULT_CTA: c->fault_cta = (int)v; return KIE_OK;
+      case KIE_OPT_FAULT_STEP: c->fault_step = (int)v; return KIE_OK;
+      case KIE_OPT_FAULT_LAYER: c->fault_layer = (int)v; return KIE_OK;
+      case KIE_OPT_FAULT_STAGE: c->fault_stage = (int)v; return KIE_OK;
     }
-    case KIE_OPT_MIN_SPLIT_LEN:
-      if (v < 1 || v > (1 << 20)) return KIE_ERR_INVALID_ARG;
-      c->min_split_len = (int)v;
-      return KIE_OK;
-    case KIE_OPT_TRACE_CLOCK:
-      c->trace_clock = v ? 1 : 0;
-      return KIE_OK;
-    case KIE_OPT_POLL_BACKOFF_NS:
-      if (v < 0 || v > 100000) return KIE_ERR_INVALID_ARG;
-      c->poll_ns = (unsigned)v;
-      return KIE_OK;
-    case KIE_OPT_L2_PREFETCH_BYTES:
-      if (v < 0 || v % 512 || v > (16 << 20)) return KIE_ERR_INVALID_ARG;
-      c->l2_prefetch = v;
-      return KIE_OK;
-    case KIE_OPT_FAULT_CTA: c->fault_cta = (int)v; return KIE_OK;
-    case KIE_OPT_FAULT_STEP: c->fault_step = (int)v; return KIE_OK;
-    case KIE_OPT_FAULT_LAYER: c->fault_layer = (int)v; return KIE_OK;
-    case KIE_OPT_FAULT_STAGE: c->fault_stage = (int)v; return KIE_OK;
-  }
-  return KIE_ERR_INVALID_ARG;
+    return KIE_ERR_INVALID_ARG;
+  });
 }
 
 kie_status kie_get_stats(const kie_ctx* cc, kie_stats* out) {
@@ -795,6 +812,7 @@ const char* kie_status_str(kie_status s) {
     case KIE_ERR_TIMEOUT: return "device wait timed out";
     case KIE_ERR_PROTOCOL: return "device protocol violation";
     case KIE_ERR_TOO_LARGE: return "size exceeds the fixed scratch of the no-allocation entry point";
+    case KIE_ERR_HOST_MEMORY: return "host memory allocation failed";
   }
   return "unknown status";
 }

@@ -21,6 +21,7 @@
 #include <vector>
 
 #include "kie.h"
+#include "kie_guard.h"
 #include "kie_kernel.h"
 #include "kie_params.h"
 #include "kie_plan.h"
@@ -82,104 +83,106 @@ extern "C" {
 
 kie_status kie_gemv_f16_noalloc(const void* W, const float* x, float* y, int32_t N, int32_t K,
                                 void* cuda_stream) {
-  constexpr int kChunkBytes = 32768;
-  if (!W || !x || !y || N < 1 || K < 256 || K % 256) return KIE_ERR_INVALID_ARG;
-  if (!aligned16(W) || !aligned16(x)) return KIE_ERR_INVALID_ARG;
-  if ((uint64_t)N * (uint64_t)K * 2u > KIE_NOALLOC_MAX_WEIGHT_BYTES) return KIE_ERR_TOO_LARGE;
+  return kie::no_throw([&]() -> kie_status {
+    constexpr int kChunkBytes = 32768;
+    if (!W || !x || !y || N < 1 || K < 256 || K % 256) return KIE_ERR_INVALID_ARG;
+    if (!aligned16(W) || !aligned16(x)) return KIE_ERR_INVALID_ARG;
+    if ((uint64_t)N * (uint64_t)K * 2u > KIE_NOALLOC_MAX_WEIGHT_BYTES) return KIE_ERR_TOO_LARGE;
 
-  unsigned char* scratch = nullptr;
-  kie_status ret = scratch_on_current_device(&scratch);
-  if (ret != KIE_OK) return ret;
+    unsigned char* scratch = nullptr;
+    kie_status ret = scratch_on_current_device(&scratch);
+    if (ret != KIE_OK) return ret;
 
-  cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
-  int dev = 0, n_sm = 0, smem_optin = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess ||
-      cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
-      cudaDeviceGetAttribute(&smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) !=
-          cudaSuccess)
-    return KIE_ERR_CUDA;
-  const int grid = std::min(std::min(n_sm, kMaxCtas), (int)N);
+    cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
+    int dev = 0, n_sm = 0, smem_optin = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) !=
+            cudaSuccess)
+      return KIE_ERR_CUDA;
+    const int grid = std::min(std::min(n_sm, kMaxCtas), (int)N);
 
-  // The rows split as the LM-head stage splits a vocabulary; the four layer
-  // stages of the one-layer plan own no rows.
-  kie::Shape sh{1, K, 1, 1, 64, 256, N};
-  const std::vector<int2> lm = kie::partition(sh, grid, kie::ST_LM);
-  int2 ranges[kie::N_STAGES * kMaxCtas] = {};
-  unsigned long long off[kMaxCtas] = {};
-  int maxrows = 0;
-  size_t total = 0;
-  for (int c = 0; c < grid; ++c) {
-    ranges[kie::ST_LM * grid + c] = lm[c];
-    maxrows = std::max(maxrows, lm[c].y - lm[c].x);
-    off[c] = total;
-    total += (size_t)(lm[c].y - lm[c].x) * K * 2;
-  }
+    // The rows split as the LM-head stage splits a vocabulary; the four layer
+    // stages of the one-layer plan own no rows.
+    kie::Shape sh{1, K, 1, 1, 64, 256, N};
+    const std::vector<int2> lm = kie::partition(sh, grid, kie::ST_LM);
+    int2 ranges[kie::N_STAGES * kMaxCtas] = {};
+    unsigned long long off[kMaxCtas] = {};
+    int maxrows = 0;
+    size_t total = 0;
+    for (int c = 0; c < grid; ++c) {
+      ranges[kie::ST_LM * grid + c] = lm[c];
+      maxrows = std::max(maxrows, lm[c].y - lm[c].x);
+      off[c] = total;
+      total += (size_t)(lm[c].y - lm[c].x) * K * 2;
+    }
 
-  kie::SmemLayout L{};
-  L.xs_bytes = (K * 4 + 127) / 128 * 128;
-  L.rowacc_rows = maxrows;
-  L.resid_rows = 0;
-  const int rowacc_bytes = (maxrows * 4 + 127) / 128 * 128;
-  const int fixed = 256 + L.xs_bytes + rowacc_bytes + kie::kEngineMisc;
-  const int ring = (smem_optin - fixed) / 512 * 512;
-  if (ring < 2 * kChunkBytes) return KIE_ERR_UNSUPPORTED;
-  L.ring_off = 0;
-  L.bar_off = ring;
-  L.xs_off = L.bar_off + 256;
-  L.rowacc_off = L.xs_off + L.xs_bytes;
-  L.misc_off = L.rowacc_off + rowacc_bytes;
-  L.total = L.misc_off + kie::kEngineMisc;
+    kie::SmemLayout L{};
+    L.xs_bytes = (K * 4 + 127) / 128 * 128;
+    L.rowacc_rows = maxrows;
+    L.resid_rows = 0;
+    const int rowacc_bytes = (maxrows * 4 + 127) / 128 * 128;
+    const int fixed = 256 + L.xs_bytes + rowacc_bytes + kie::kEngineMisc;
+    const int ring = (smem_optin - fixed) / 512 * 512;
+    if (ring < 2 * kChunkBytes) return KIE_ERR_UNSUPPORTED;
+    L.ring_off = 0;
+    L.bar_off = ring;
+    L.xs_off = L.bar_off + 256;
+    L.rowacc_off = L.xs_off + L.xs_bytes;
+    L.misc_off = L.rowacc_off + rowacc_bytes;
+    L.total = L.misc_off + kie::kEngineMisc;
 
-  auto* d_status = reinterpret_cast<DevStatus*>(scratch + kOffStatus);
-  auto* d_layer = reinterpret_cast<LayerW*>(scratch + kOffLayer);
-  auto* d_ranges = reinterpret_cast<int2*>(scratch + kOffRanges);
-  auto* d_off = reinterpret_cast<unsigned long long*>(scratch + kOffPackedOff);
-  auto* d_stats = reinterpret_cast<unsigned long long*>(scratch + kOffStats);
-  unsigned char* d_packed = scratch + kOffPacked;
+    auto* d_status = reinterpret_cast<DevStatus*>(scratch + kOffStatus);
+    auto* d_layer = reinterpret_cast<LayerW*>(scratch + kOffLayer);
+    auto* d_ranges = reinterpret_cast<int2*>(scratch + kOffRanges);
+    auto* d_off = reinterpret_cast<unsigned long long*>(scratch + kOffPackedOff);
+    auto* d_stats = reinterpret_cast<unsigned long long*>(scratch + kOffStats);
+    unsigned char* d_packed = scratch + kOffPacked;
 
-  MonoParams p{};
-  p.L = 1;
-  p.d = K;
-  p.H = 1;
-  p.KV = 1;
-  p.hd = 64;
-  p.F = 256;
-  p.V = N;
-  p.G = 1;
-  p.layers = d_layer;
-  p.lm_head = static_cast<const __half*>(W);
-  p.ranges = d_ranges;
-  p.grid = grid;
-  p.ring_bytes = ring;
-  p.chunk_bytes = kChunkBytes;
-  p.packed = d_packed;
-  p.packed_off = d_off;
-  p.sm = L;
-  p.status = d_status;
-  p.cta_stats = d_stats;
-  p.timeout_ns = 2000000000LL;
-  p.poll_ns = 128;
-  p.fault_cta = -1;
+    MonoParams p{};
+    p.L = 1;
+    p.d = K;
+    p.H = 1;
+    p.KV = 1;
+    p.hd = 64;
+    p.F = 256;
+    p.V = N;
+    p.G = 1;
+    p.layers = d_layer;
+    p.lm_head = static_cast<const __half*>(W);
+    p.ranges = d_ranges;
+    p.grid = grid;
+    p.ring_bytes = ring;
+    p.chunk_bytes = kChunkBytes;
+    p.packed = d_packed;
+    p.packed_off = d_off;
+    p.sm = L;
+    p.status = d_status;
+    p.cta_stats = d_stats;
+    p.timeout_ns = 2000000000LL;
+    p.poll_ns = 128;
+    p.fault_cta = -1;
 
-  // The previous call's status, layer table and counters are still in the
-  // array: clear them; ranges and offsets are rewritten in full.
-  DevStatus hs{};
-  if (cudaMemsetAsync(d_status, 0, sizeof(DevStatus), st) != cudaSuccess ||
-      cudaMemsetAsync(d_layer, 0, sizeof(LayerW), st) != cudaSuccess ||
-      cudaMemsetAsync(d_stats, 0, sizeof(unsigned long long) * kie::kStatsPerCta * grid, st) !=
-          cudaSuccess ||
-      cudaMemcpyAsync(d_ranges, ranges, sizeof(int2) * kie::N_STAGES * grid,
-                      cudaMemcpyHostToDevice, st) != cudaSuccess ||
-      cudaMemcpyAsync(d_off, off, sizeof(unsigned long long) * grid, cudaMemcpyHostToDevice,
-                      st) != cudaSuccess ||
-      kie::repack_launch(p, d_packed, st) != cudaSuccess ||
-      kie::gemv_configure(L.total) != cudaSuccess ||
-      kie::gemv_launch(p, 1, x, y, 1, grid, L.total, st) != cudaSuccess ||
-      cudaMemcpyAsync(&hs, d_status, sizeof hs, cudaMemcpyDeviceToHost, st) != cudaSuccess ||
-      cudaStreamSynchronize(st) != cudaSuccess)
-    return KIE_ERR_CUDA;
-  if (hs.code != kie::DEV_OK) return hs.code == kie::DEV_TIMEOUT ? KIE_ERR_TIMEOUT : KIE_ERR_PROTOCOL;
-  return KIE_OK;
+    // The previous call's status, layer table and counters are still in the
+    // array: clear them; ranges and offsets are rewritten in full.
+    DevStatus hs{};
+    if (cudaMemsetAsync(d_status, 0, sizeof(DevStatus), st) != cudaSuccess ||
+        cudaMemsetAsync(d_layer, 0, sizeof(LayerW), st) != cudaSuccess ||
+        cudaMemsetAsync(d_stats, 0, sizeof(unsigned long long) * kie::kStatsPerCta * grid, st) !=
+            cudaSuccess ||
+        cudaMemcpyAsync(d_ranges, ranges, sizeof(int2) * kie::N_STAGES * grid,
+                        cudaMemcpyHostToDevice, st) != cudaSuccess ||
+        cudaMemcpyAsync(d_off, off, sizeof(unsigned long long) * grid, cudaMemcpyHostToDevice,
+                        st) != cudaSuccess ||
+        kie::repack_launch(p, d_packed, st) != cudaSuccess ||
+        kie::gemv_configure(L.total) != cudaSuccess ||
+        kie::gemv_launch(p, 1, x, y, 1, grid, L.total, st) != cudaSuccess ||
+        cudaMemcpyAsync(&hs, d_status, sizeof hs, cudaMemcpyDeviceToHost, st) != cudaSuccess ||
+        cudaStreamSynchronize(st) != cudaSuccess)
+      return KIE_ERR_CUDA;
+    if (hs.code != kie::DEV_OK) return hs.code == kie::DEV_TIMEOUT ? KIE_ERR_TIMEOUT : KIE_ERR_PROTOCOL;
+    return KIE_OK;
+  });
 }
 
 }  // extern "C"
