@@ -135,3 +135,57 @@ def score_margin(scores: np.ndarray) -> float:
     """Top-1 minus top-2 of the perturbed scores."""
     s = np.sort(np.asarray(scores, dtype=np.float64))
     return float(s[-1] - s[-2]) if s.shape[0] > 1 else float("inf")
+
+
+# ---- filtered sampling (top-k, top-p).  The kernel does not draw these
+# yet; they are defined here first so that its draws can be checked.
+#
+# top-k keeps the k largest logits (ties broken by the lower index); top-p
+# (nucleus) keeps, of the remaining entries ordered by probability under
+# softmax(logits / T) (ties by the lower index), the shortest prefix whose
+# probability mass reaches p, renormalised over the kept set.  The draw is
+# the Gumbel-max one above restricted to the kept set, with the same
+# noise, so an entry's score does not depend on the filter.
+
+def _order(values: np.ndarray) -> np.ndarray:
+    """Indices by value, largest first, ties by the lower index."""
+    v = np.asarray(values, dtype=np.float64)
+    return np.lexsort((np.arange(v.shape[0]), -v))
+
+
+def top_k_set(logits: np.ndarray, k: int) -> np.ndarray:
+    """Indices of the k largest logits (all of them for k <= 0 or k >= V)."""
+    lg = np.asarray(logits)
+    if k <= 0 or k >= lg.shape[0]:
+        return np.arange(lg.shape[0])
+    return np.sort(_order(lg)[:k])
+
+
+def top_p_set(logits: np.ndarray, temperature: float, p: float,
+              among: np.ndarray = None) -> np.ndarray:
+    """The nucleus: of the entries `among` (default all), ordered by
+    probability under softmax(logits / T) restricted to them, the shortest
+    prefix whose mass reaches p (at least one entry; all for p >= 1)."""
+    lg = np.asarray(logits, dtype=np.float64)
+    idx = np.arange(lg.shape[0]) if among is None else np.asarray(among)
+    if p >= 1.0:
+        return np.sort(idx)
+    z = lg[idx] / float(temperature)
+    pr = np.exp(z - z.max())
+    pr /= pr.sum()
+    o = _order(pr)
+    mass = np.cumsum(pr[o])
+    n = int(np.searchsorted(mass, p, side="left")) + 1
+    return np.sort(idx[o[:min(n, idx.shape[0])]])
+
+
+def sample_id_filtered(logits: np.ndarray, temperature: float, seed: int, position: int,
+                       top_k: int = 0, top_p: float = 1.0) -> int:
+    """Draw restricted to top-k, then top-p of what top-k kept.  T <= 0 is
+    greedy (the argmax lies in every non-empty kept set)."""
+    if temperature <= 0:
+        return int(np.argmax(np.asarray(logits)))
+    keep = top_k_set(logits, top_k)
+    keep = top_p_set(logits, temperature, top_p, among=keep)
+    sc = perturbed_scores(logits, temperature, seed, position)
+    return int(keep[np.argmax(sc[keep])])

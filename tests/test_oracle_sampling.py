@@ -106,6 +106,76 @@ def test_score_margin():
     assert S.score_margin(np.array([1.0])) == float("inf")
 
 
+# ---- filtered sampling (top-k, top-p)
+
+def test_top_k_set_hand_examples_and_ties():
+    lg = np.array([1.0, 2.0, 2.0, 0.0, 3.0])
+    assert list(S.top_k_set(lg, 1)) == [4]
+    assert list(S.top_k_set(lg, 2)) == [1, 4]          # tie at the boundary: lower index
+    assert list(S.top_k_set(lg, 3)) == [1, 2, 4]
+    assert list(S.top_k_set(lg, 0)) == list(range(5))
+    assert list(S.top_k_set(lg, 9)) == list(range(5))
+
+
+def test_top_p_set_hand_example_and_brute_force():
+    pi = np.array([0.4, 0.25, 0.15, 0.1, 0.06, 0.04])
+    lg = np.log(pi)
+    assert list(S.top_p_set(lg, 1.0, 0.3)) == [0]
+    assert list(S.top_p_set(lg, 1.0, 0.6)) == [0, 1]
+    assert list(S.top_p_set(lg, 1.0, 0.75)) == [0, 1, 2]
+    assert list(S.top_p_set(lg, 1.0, 0.97)) == [0, 1, 2, 3, 4, 5]
+    assert list(S.top_p_set(lg, 1.0, 1.0)) == list(range(6))
+    rng = np.random.default_rng(9)
+    for _ in range(200):
+        v = int(rng.integers(2, 12))
+        x = rng.standard_normal(v)
+        T = float(rng.uniform(0.3, 2.0))
+        p = float(rng.uniform(0.05, 0.99))
+        e = np.exp(x / T - np.max(x / T))
+        pr = e / e.sum()
+        order = sorted(range(v), key=lambda i: (-pr[i], i))
+        kept, mass = [], 0.0
+        for i in order:
+            kept.append(i)
+            mass += pr[i]
+            if mass >= p:
+                break
+        assert list(S.top_p_set(x, T, p)) == sorted(kept)
+
+
+@pytest.mark.parametrize("k,p", [(3, 1.0), (0, 0.75), (4, 0.75)])
+def test_filtered_draws_follow_the_renormalised_softmax(k, p):
+    pi = np.array([0.4, 0.25, 0.15, 0.1, 0.06, 0.04])
+    logits = np.log(pi).astype(np.float32)
+    T = 1.0
+    keep = S.top_p_set(logits, T, p, among=S.top_k_set(logits, k))
+    n = 40000
+    sc = S.perturbed_scores(logits, T, 21, np.arange(n))
+    masked = np.full_like(sc, -np.inf)
+    masked[:, keep] = sc[:, keep]
+    draws = np.argmax(masked, axis=1)
+    assert set(np.unique(draws)) <= set(keep.tolist())
+    freq = np.bincount(draws, minlength=logits.shape[0])[keep]
+    q = pi[keep] / pi[keep].sum()
+    chi2 = float(((freq - n * q) ** 2 / (n * q)).sum())
+    assert chi2 < 30.0, (chi2, freq, n * q)
+    # the per-position function agrees with the vectorised draw
+    for pos in range(0, n, 4999):
+        assert S.sample_id_filtered(logits, T, 21, pos, top_k=k, top_p=p) == int(draws[pos])
+
+
+def test_filtered_limits():
+    rng = np.random.default_rng(4)
+    for pos in range(30):
+        lg = rng.standard_normal(500).astype(np.float32)
+        g = int(np.argmax(lg))
+        assert S.sample_id_filtered(lg, 0.8, 3, pos, top_k=1) == g
+        assert S.sample_id_filtered(lg, 0.8, 3, pos, top_p=1e-9) == g
+        assert S.sample_id_filtered(lg, 0.0, 3, pos, top_k=5, top_p=0.5) == g
+        assert S.sample_id_filtered(lg, 0.8, 3, pos, top_k=500) == S.sample_id(lg, 0.8, 3, pos)
+        assert S.sample_id_filtered(lg, 0.8, 3, pos, top_p=1.0) == S.sample_id(lg, 0.8, 3, pos)
+
+
 # ---- planted mistakes: each must make one of the pins above fail
 
 def _philox_early_key_bump(counter, key):
@@ -155,7 +225,19 @@ def _sample_id_argmin(logits, temperature, seed, position):
     return int(np.argmax(S.perturbed_scores(logits, temperature, seed, position)))
 
 
-_ORIG = {k: getattr(S, k) for k in ("philox4x64_10_many", "uniforms")}
+def _top_k_one_more(logits, k):
+    lg = np.asarray(logits)
+    if k <= 0 or k >= lg.shape[0]:
+        return np.arange(lg.shape[0])
+    return np.sort(S._order(lg)[:k + 1])
+
+
+def _top_p_stops_short(logits, temperature, p, among=None):
+    kept = _ORIG["top_p_set"](logits, temperature, p, among)
+    return kept if kept.shape[0] == 1 or p >= 1.0 else kept[:-1]
+
+
+_ORIG = {k: getattr(S, k) for k in ("philox4x64_10_many", "uniforms", "top_p_set")}
 
 MUTATIONS = [
     ("philox4x64_10", _philox_early_key_bump,
@@ -166,6 +248,8 @@ MUTATIONS = [
     ("gumbel", _gumbel_wrong_sign, lambda: test_gumbel_max_draws_softmax(1.0)),
     ("perturbed_scores", _scores_times_t, lambda: test_gumbel_max_draws_softmax(0.7)),
     ("sample_id", _sample_id_argmin, test_limits),
+    ("top_k_set", _top_k_one_more, test_top_k_set_hand_examples_and_ties),
+    ("top_p_set", _top_p_stops_short, test_top_p_set_hand_example_and_brute_force),
 ]
 
 
