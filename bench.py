@@ -196,7 +196,7 @@ def reduce_max_sum(dist, elapsed_s: float, tokens: float, device=None):
 
 # ------------------------------------------------------------- CPU oracle
 
-def cpu_oracle_rate(w: synth.Workload, model, budget_s: float = 12.0, max_steps: int = 64,
+def cpu_oracle_rate(w: synth.Workload, model, budget_s: float = 15.0, max_steps: int = 256,
                     warmup: int = 1):
     """Times the oracle's incremental decode (fp32, numpy/BLAS on the host
     cores) after a batched prefill of the prompt.  Returns (tok/s, info)."""
