@@ -92,3 +92,48 @@ def test_pin_catches_planted_mistake(monkeypatch, name, bad, pin):
     monkeypatch.setattr(pins, name, bad, raising=False)
     with pytest.raises(AssertionError):
         pin()
+
+
+# ---- mistakes in the model-level wiring of q and k (both oracle paths)
+
+def _k_cached_without_rope():
+    # both paths call apply_rope for q, then for k, in every layer and step:
+    # rotate the odd calls only, so k enters the cache unrotated
+    orig = om.apply_rope
+    calls = [0]
+
+    def rope(x, cos, sin):
+        calls[0] += 1
+        return orig(x, cos, sin) if calls[0] % 2 == 1 else x
+    return rope
+
+
+def _q_reshaped_hd_by_h():
+    # q = (Wq a).reshape(hd, H).T: head h dim i read from element i*H + h,
+    # the same as Wq's rows permuted that way in both paths
+    orig = om.OracleModel.w
+
+    def w(self, name):
+        a = orig(self, name)
+        if name.endswith(".wq"):
+            perm = [i * self.H + h for h in range(self.H) for i in range(self.hd)]
+            a = a[perm]
+        return a
+    return w
+
+
+MODEL_MUTATIONS = [
+    ("apply_rope", _k_cached_without_rope),
+    ("OracleModel.w", _q_reshaped_hd_by_h),
+]
+
+
+@pytest.mark.parametrize("name,make", MODEL_MUTATIONS, ids=[m[1].__name__ for m in MODEL_MUTATIONS])
+def test_scalar_loop_pin_catches_model_level_mistake(monkeypatch, name, make):
+    bad = make()
+    if name == "OracleModel.w":
+        monkeypatch.setattr(om.OracleModel, "w", bad)
+    else:
+        monkeypatch.setattr(om, name, bad)
+    with pytest.raises(AssertionError):
+        pins.test_one_layer_model_equals_scalar_loops_at_three_positions()

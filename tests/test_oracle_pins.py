@@ -311,6 +311,96 @@ def test_ffn_branch_closed_form_gate_gets_silu():
     np.testing.assert_allclose(om.forward([tok])[0], want, rtol=1e-12, atol=1e-13)
 
 
+def _one_layer_scalar_loops(m, toks):
+    """Logits of a one-layer model at every position of `toks`, written as
+    scalar loops straight from the block's definition (no numpy algebra):
+    q_h from rows h*hd .. h*hd+hd-1 of Wq, k_j and v_j likewise from Wk and
+    Wv, RoPE on q AND k at the token's own position t (pairs (i, i+hd/2),
+    angle t * base^(-2i/hd)), scores over u <= t scaled by 1/sqrt(hd),
+    softmax, weighted sum of v, Wo, residual, RMSNorm, SwiGLU FFN, residual,
+    final RMSNorm and the LM head.  Python floats are IEEE doubles."""
+    s = m.shape
+    d, H, KV, hd, F, V = s.d_model, s.n_heads, s.n_kv_heads, s.head_dim, s.ffn_dim, s.vocab
+    G, half, eps = H // KV, hd // 2, s.rms_eps
+    f = {k: v.astype(np.float64).tolist() for k, v in m.tensors.items()}
+
+    def norm(x, g):
+        ms = sum(xi * xi for xi in x) / len(x)
+        r = 1.0 / math.sqrt(ms + eps)
+        return [g[c] * x[c] * r for c in range(len(x))]
+
+    def matvec(W, x):
+        return [sum(W[r][c] * x[c] for c in range(len(x))) for r in range(len(W))]
+
+    def rope(vec, t):
+        out = list(vec)
+        for i in range(half):
+            ang = t * s.rope_base ** (-2.0 * i / hd)
+            c, sn = math.cos(ang), math.sin(ang)
+            out[i] = vec[i] * c - vec[i + half] * sn
+            out[i + half] = vec[i + half] * c + vec[i] * sn
+        return out
+
+    keys, vals, logits = [], [], []
+    for t, tok in enumerate(toks):
+        h = list(f["tok_emb"][tok])
+        a = norm(h, f["0.attn_norm"])
+        q = [rope([sum(f["0.wq"][hh * hd + i][c] * a[c] for c in range(d)) for i in range(hd)], t)
+             for hh in range(H)]
+        keys.append([rope([sum(f["0.wk"][j * hd + i][c] * a[c] for c in range(d))
+                           for i in range(hd)], t) for j in range(KV)])
+        vals.append([[sum(f["0.wv"][j * hd + i][c] * a[c] for c in range(d)) for i in range(hd)]
+                     for j in range(KV)])
+        o = []
+        for hh in range(H):
+            j = hh // G
+            sc = [sum(q[hh][i] * keys[u][j][i] for i in range(hd)) / math.sqrt(hd)
+                  for u in range(t + 1)]
+            mx = max(sc)
+            e = [math.exp(x - mx) for x in sc]
+            z = sum(e)
+            o += [sum(e[u] / z * vals[u][j][i] for u in range(t + 1)) for i in range(hd)]
+        att = matvec(f["0.wo"], o)
+        h = [h[r] + att[r] for r in range(d)]
+        b = norm(h, f["0.ffn_norm"])
+        gz, uz = matvec(f["0.w_gate"], b), matvec(f["0.w_up"], b)
+        act = [gz[k] / (1.0 + math.exp(-gz[k])) * uz[k] for k in range(F)]
+        dn = matvec(f["0.w_down"], act)
+        h = [h[r] + dn[r] for r in range(d)]
+        logits.append(matvec(f["lm_head"], norm(h, f["final_norm"])))
+    return np.array(logits)
+
+
+def _qk_pin_model():
+    # weights ~N(0, 0.5) so that the softmax is far from uniform and the
+    # rotation angles (1 and 2 rad at i = 0) move the scores
+    shp = _tiny_shape(n_layers=1, d_model=16, n_heads=4, n_kv_heads=2, head_dim=8,
+                      ffn_dim=12, vocab=11, rope_base=100.0)
+    m = _random_gains(synth.make_model(shp, seed=12), seed=13)
+    rng = np.random.default_rng(14)
+    for k, v in m.tensors.items():
+        if not k.endswith("norm"):
+            m.tensors[k] = (0.5 * rng.standard_normal(v.shape)).astype(np.float16)
+    return m
+
+
+def test_one_layer_model_equals_scalar_loops_at_three_positions():
+    # pins how rows of Wq / Wk / Wv map to heads, RoPE of both q and k at
+    # each token's position, the causal range and GQA wiring at the model
+    # level, in both oracle paths
+    m = _qk_pin_model()
+    toks = [3, 7, 3]
+    want = _one_layer_scalar_loops(m, toks)
+    om = OracleModel(m, dtype=np.float64)
+    np.testing.assert_allclose(om.forward(toks), want, rtol=1e-12, atol=1e-12)
+    st = om.new_state()
+    inc = np.stack([om.decode_step(st, t) for t in toks])
+    np.testing.assert_allclose(inc, want, rtol=1e-12, atol=1e-12)
+    # the positions differ: a model that ignored q, k or the rotation would
+    # give position 2 the logits of a one-token context of the same token
+    assert np.max(np.abs(want[2] - want[0])) > 1e-2
+
+
 def test_argmax_lowest_index_on_ties_bruteforce():
     rng = np.random.default_rng(10)
     for trial in range(50):
