@@ -8,7 +8,11 @@ baseline leg of `bench.py` may import it; the library itself never does.
 Every function carries its definition in its docstring; `tests/test_oracle_pins.py`
 pins each of them to closed forms, invariants and brute force, and
 `tests/test_oracle_sampling.py` pins the sampler (`oracle.sampling`) to
-numpy's own Philox generator and to the softmax distribution it must draw.  Parity status
+numpy's own Philox generator and to the softmax distribution it must draw,
+and `tests/test_oracle_fp8.py` pins the FP8 weight quantisation
+(`oracle.fp8`: E4M3 codes, per-row scales, the dequantised model) to the
+format's closed forms, torch's and ml_dtypes' E4M3 conversions and brute
+force.  Parity status
 of each function: all pinned (none is "parity unpinned").
 """
 from .model import (  # noqa: F401
