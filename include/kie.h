@@ -161,20 +161,28 @@ typedef enum {
 } kie_option;
 
 /* Bytes of the caller-provided KV cache: 2*n_layers*n_kv_heads*max_seq*(head_dim+8)*2.
- * Returns 0 for a NULL or invalid desc.  Host only. */
+ * This is MORE than the unpadded 2*n_layers*n_kv_heads*max_seq*head_dim*2 of
+ * a plain [layer][K|V][kv_head][pos][head_dim] fp16 cache: every position's
+ * row carries 8 unused fp16 elements (see the layout above), 3% more at
+ * head_dim 128 and 6% at 64.  Size the buffer with this call, not with the
+ * unpadded formula.  Returns 0 for a NULL or invalid desc.  Host only. */
 KIE_API size_t kie_kv_cache_bytes(const kie_model_desc *desc);
 
 /* Checks a shape against the limits above.  Host only, no CUDA call. */
 KIE_API kie_status kie_check_desc(const kie_model_desc *desc);
 
-/* Creates a context on the current CUDA device.  `kv_cache` is the
+/* Creates a context on the current CUDA device (the pages' resident decode
+ * program, revietech.ru, "Kog выжимает максимум из GPU: 3000 токенов/с",
+ * section "Что такое monokernel", set up once per model: plan, packed
+ * weight stream, scratch).  `kv_cache` is the
  * caller's device buffer (kie_kv_cache_bytes bytes); `cuda_stream` is a
  * cudaStream_t (NULL = legacy default stream).  On success *out receives
  * the context; on failure *out is set to NULL. */
 KIE_API kie_status kie_create(const kie_model_desc *desc, const kie_weights *weights,
                       void *kv_cache, void *cuda_stream, kie_ctx **out);
 
-/* Runs the prompt through the model in one launch, writing K/V for
+/* Prefill, the first phase the pages' resident program runs (same page and
+ * section): runs the prompt through the model in one launch, writing K/V for
  * positions 0..n-1 (the session restarts at position 0), and returns in
  * *first_id the id picked (greedy or sampled, kie_set_sampling) from the
  * last position's logits.
@@ -182,7 +190,9 @@ KIE_API kie_status kie_create(const kie_model_desc *desc, const kie_weights *wei
 KIE_API kie_status kie_prefill(kie_ctx *ctx, const int32_t *prompt_ids, int32_t n,
                        int32_t *first_id);
 
-/* Runs n_steps decode steps in ONE launch.  Step i feeds the
+/* Decode with token selection and the end-id check inside the kernel, no
+ * launch per token and no return to the CPU between tokens (same page and
+ * section).  Runs n_steps decode steps in ONE launch.  Step i feeds the
  * previous id (the id from kie_prefill or the last id of the previous
  * decode call for i = 0) at the next position and writes the picked id to
  * out_ids[i] (HOST array [n_steps]).  Stops after emitting an end id
@@ -261,6 +271,9 @@ KIE_API kie_status kie_get_stats(const kie_ctx *ctx, kie_stats *out);
 KIE_API const char *kie_status_str(kie_status s);
 /* Text of the last error on this context ("" if none); valid until the next call. */
 KIE_API const char *kie_last_error(const kie_ctx *ctx);
+/* Ends a context (the counterpart of kie_create; same page and section):
+ * frees the library-owned packed weights and scratch; the caller's weights
+ * and KV cache are not touched.  KIE_ERR_INVALID_ARG for NULL. */
 KIE_API kie_status kie_destroy(kie_ctx *ctx);
 
 /* The decode kernel's weight-stream GEMV engine run alone, for unit tests
@@ -300,7 +313,12 @@ KIE_API kie_status kie_gemv_f16(const void *W, const float *x, float *y, int32_t
  *
  * The first call on a device looks up the array's address on that device
  * (cudaGetSymbolAddress, which may load the library's device code there);
- * make that first call before any stream capture.  Every call clears the
+ * make that first call before any stream capture.  The address belongs to
+ * the device's current driver context: after cudaDeviceReset, or with
+ * another context made current, the next call looks it up again (so that
+ * call is again a first call).  Another host thread's kie_gemv_f16 does not
+ * disturb a call, but it is GPU work like any other: overlapping the two on
+ * the GPU is fine, overlapping two calls of this entry point is not.  Every call clears the
  * parts of the array that must start at zero; all calls on a device share
  * the array, so calls that overlap on the GPU (two streams, two host
  * threads) race and give wrong results: serialise them.  Synchronous on

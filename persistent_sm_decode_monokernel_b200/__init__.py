@@ -39,10 +39,20 @@ class Session:
     ffn_dim, vocab, rope_base, rms_eps.  weights: device fp16 tensors named
     tok_emb, final_norm, lm_head and "{l}.{attn_norm,wq,wk,wv,wo,ffn_norm,
     w_gate,w_up,w_down}".  The KV cache is allocated here with torch.
+
+    kie_create keeps its own packed copy of every weight matrix and from
+    then on reads only tok_emb and the norm gains of `weights`.  With
+    keep_matrices=False the session drops its references to the matrices
+    right after kie_create (their memory is freed once the caller drops
+    its own), which halves the weights' device footprint; re-planning the
+    chunk size (KIE_OPT_CHUNK_BYTES) then raises, since it re-reads them.
     """
 
+    # the tensors kie_create's packed copy does not replace
+    _KEPT = ("tok_emb", "final_norm")
+
     def __init__(self, shape, weights: Mapping[str, object], max_seq: int, eos_id: int = -1,
-                 stream=None):
+                 stream=None, keep_matrices: bool = True):
         import torch
         load_library()
         self.shape = shape
@@ -60,6 +70,15 @@ class Session:
         self.stream = stream
         self.ctx = kie_create(self.desc, weights, self.kv, stream.cuda_stream)
         self._capture = None
+        if not keep_matrices:
+            self.release_matrices()
+
+    def release_matrices(self) -> None:
+        """Drops this session's references to the weight matrices (kept:
+        the embedding and the norm gains, which the kernel still reads)."""
+        self.weights = {k: v for k, v in self.weights.items()
+                        if k in self._KEPT or k.endswith("norm")}
+        self._matrices_released = True
 
     def prefill(self, ids: Sequence[int]) -> int:
         return kie_prefill(self.ctx, ids)
@@ -100,6 +119,9 @@ class Session:
         self._trace = None
 
     def set_option(self, opt: int, value: int) -> None:
+        if opt == _kie.KIE_OPT_CHUNK_BYTES and getattr(self, "_matrices_released", False):
+            raise ValueError("KIE_OPT_CHUNK_BYTES re-reads the weight matrices, which this "
+                             "session has released (keep_matrices=False)")
         kie_set_option(self.ctx, opt, value)
 
     def set_sampling(self, temperature: float, seed: int = 0) -> None:

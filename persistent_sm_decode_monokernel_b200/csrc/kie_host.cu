@@ -670,7 +670,7 @@ kie_status kie_gemv_f16(const void* W, const float* x, float* y, int32_t N, int3
               cudaSuccess ||
           cudaMemsetAsync(d_layer, 0, sizeof(LayerW), st) != cudaSuccess ||
           kie::repack_launch(p, d_packed, st) != cudaSuccess ||
-          kie::gemv_configure(L.total) != cudaSuccess || cudaEventRecord(e0, st) != cudaSuccess ||
+          kie::gemv_configure() != cudaSuccess || cudaEventRecord(e0, st) != cudaSuccess ||
           kie::gemv_launch(p, mode, x, y, iters, grid, L.total, st) != cudaSuccess ||
           cudaEventRecord(e1, st) != cudaSuccess || cudaStreamSynchronize(st) != cudaSuccess)
         ret = KIE_ERR_CUDA;

@@ -1814,9 +1814,18 @@ cudaError_t repack_launch(const MonoParams& p, unsigned char* packed, cudaStream
   return cudaGetLastError();
 }
 
-cudaError_t gemv_configure(int smem_bytes) {
+// Lets kie_gemv_kernel use up to the current device's opt-in maximum of
+// dynamic shared memory.  Always the same value, so calls from several host
+// threads (the allocating and the no-allocation GEMV entry points) cannot
+// undo each other's setting between configure and launch.
+cudaError_t gemv_configure() {
+  int dev = 0, optin = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e == cudaSuccess)
+    e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+  if (e != cudaSuccess) return e;
   return cudaFuncSetAttribute((const void*)kie_gemv_kernel,
-                              cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes);
+                              cudaFuncAttributeMaxDynamicSharedMemorySize, optin);
 }
 
 cudaError_t gemv_launch(const MonoParams& p, int mode, const float* x, float* y, int iters,

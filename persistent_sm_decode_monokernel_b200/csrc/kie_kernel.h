@@ -20,7 +20,9 @@ cudaError_t repack_launch(const MonoParams& p, unsigned char* packed, cudaStream
 
 // Standalone weight-stream GEMV (the LM-head stage over an arbitrary
 // matrix): y = W x, `iters` times; mode 0 streams without computing.
-cudaError_t gemv_configure(int smem_bytes);
+// gemv_configure raises the kernel's dynamic shared-memory limit to the
+// current device's opt-in maximum (the same value on every call).
+cudaError_t gemv_configure();
 cudaError_t gemv_launch(const MonoParams& p, int mode, const float* x, float* y, int iters,
                         int grid, int smem_bytes, cudaStream_t s);
 

@@ -13,6 +13,7 @@
 // contents there; whatever must start at zero is cleared on the stream by
 // each call.  Two calls whose work overlaps on the GPU (different streams,
 // or different host threads) race on it; callers serialise them.
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <algorithm>
@@ -55,23 +56,65 @@ static_assert(kOffPacked <= 64 * 1024, "scratch header grew past 64 KB");
 static __device__ __align__(256) unsigned char kie_noalloc_scratch[kScratchBytes];
 
 std::mutex g_setup_mu;
-unsigned char* g_scratch_addr[kMaxDevices] = {};
 
-// Device address of the scratch on the current device, looked up on the
-// first call made on that device (this loads the library's device code on
-// it if nothing has yet).
+// Address of the array per device, together with the id of the driver
+// context it was looked up in.  A module's device addresses belong to one
+// context: after cudaDeviceReset, or with another driver context made
+// current on the same device, the array lives at a new address, so a cached
+// address is only reused while the current context's id (unique for the
+// life of the process) still matches.
+struct ScratchAddr {
+  unsigned long long ctx_id;
+  unsigned char* addr;
+};
+ScratchAddr g_scratch[kMaxDevices] = {};
+
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long*);
+
+// Id of the current driver context; false if the driver cannot tell or no
+// context is current yet (then the address is looked up again).
+bool current_ctx_id(unsigned long long* id) {
+  static CtxGetCurrentFn get_current = nullptr;
+  static CtxGetIdFn get_id = nullptr;
+  static bool resolved = false;
+  if (!resolved) {
+    void* f0 = nullptr;
+    void* f1 = nullptr;
+    cudaDriverEntryPointQueryResult q0{}, q1{};
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f0, cudaEnableDefault, &q0) == cudaSuccess &&
+        cudaGetDriverEntryPoint("cuCtxGetId", &f1, cudaEnableDefault, &q1) == cudaSuccess &&
+        q0 == cudaDriverEntryPointSuccess && q1 == cudaDriverEntryPointSuccess) {
+      get_current = reinterpret_cast<CtxGetCurrentFn>(f0);
+      get_id = reinterpret_cast<CtxGetIdFn>(f1);
+    }
+    resolved = true;
+  }
+  CUcontext ctx = nullptr;
+  return get_current && get_id && get_current(&ctx) == CUDA_SUCCESS && ctx &&
+         get_id(ctx, id) == CUDA_SUCCESS;
+}
+
+// Device address of the scratch in the current device's current context,
+// looked up (cudaGetSymbolAddress, which loads the library's device code
+// into that context if nothing has yet) on the first call made in that
+// context, and reused while the context stays the same.
 kie_status scratch_on_current_device(unsigned char** out) {
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess) return KIE_ERR_CUDA;
   if (dev < 0 || dev >= kMaxDevices) return KIE_ERR_UNSUPPORTED;
   std::lock_guard<std::mutex> lock(g_setup_mu);
-  if (!g_scratch_addr[dev]) {
+  unsigned long long id = 0;
+  const bool have_id = current_ctx_id(&id);
+  ScratchAddr& e = g_scratch[dev];
+  if (!have_id || !e.addr || e.ctx_id != id) {
     void* ptr = nullptr;
     if (cudaGetSymbolAddress(&ptr, kie_noalloc_scratch) != cudaSuccess || !ptr)
       return KIE_ERR_CUDA;
-    g_scratch_addr[dev] = static_cast<unsigned char*>(ptr);
+    e.addr = static_cast<unsigned char*>(ptr);
+    e.ctx_id = have_id ? id : 0ull;
   }
-  *out = g_scratch_addr[dev];
+  *out = e.addr;
   return KIE_OK;
 }
 
@@ -175,7 +218,7 @@ kie_status kie_gemv_f16_noalloc(const void* W, const float* x, float* y, int32_t
         cudaMemcpyAsync(d_off, off, sizeof(unsigned long long) * grid, cudaMemcpyHostToDevice,
                         st) != cudaSuccess ||
         kie::repack_launch(p, d_packed, st) != cudaSuccess ||
-        kie::gemv_configure(L.total) != cudaSuccess ||
+        kie::gemv_configure() != cudaSuccess ||
         kie::gemv_launch(p, 1, x, y, 1, grid, L.total, st) != cudaSuccess ||
         cudaMemcpyAsync(&hs, d_status, sizeof hs, cudaMemcpyDeviceToHost, st) != cudaSuccess ||
         cudaStreamSynchronize(st) != cudaSuccess)

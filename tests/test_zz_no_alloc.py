@@ -63,6 +63,46 @@ def test_noalloc_matches_allocating_gemv_twice(torch_cuda):
         assert ((got - ref).abs() <= _bound(W, x)).all(), float((got - ref).abs().max())
 
 
+def test_noalloc_after_rejected_call_and_after_larger_grid(torch_cuda):
+    """A call the entry point rejects (misaligned x) leaves the array as it
+    was, and a call on a matrix with fewer rows than the GPU has SMs (a
+    smaller grid) after one with more rows must not read the row split or
+    offsets the larger call left beyond its own grid."""
+    torch = torch_cuda
+    from persistent_sm_decode_monokernel_b200 import _kie
+    lib = _kie.load_library()
+    stream = torch.cuda.current_stream().cuda_stream
+    g = torch.Generator(device="cpu").manual_seed(21)
+    n_sm = torch.cuda.get_device_properties(0).multi_processor_count
+    big = ((torch.randn(4 * n_sm, 512, generator=g) * 0.02).half().cuda(),
+           torch.randn(512, generator=g).float().cuda())
+    small = ((torch.randn(n_sm // 3, 768, generator=g) * 0.02).half().cuda(),
+             torch.randn(768 + 4, generator=g).float().cuda())
+    outs = []
+    for W, x in (big, small):
+        N, K = W.shape
+        xk = x[:K].contiguous()
+        y_ref = torch.full((N,), float("nan"), device="cuda")
+        _kie.kie_gemv_f16(W, xk, y_ref, iters=1, mode=1, chunk_bytes=32768, stream=stream)
+        y = torch.full((N,), float("nan"), device="cuda")
+        torch.cuda.synchronize()
+        if W is small[0]:
+            # x + 1 element is 4-byte but not 16-byte aligned: rejected before
+            # the array is touched
+            st = lib.kie_gemv_f16_noalloc(ctypes.c_void_p(W.data_ptr()),
+                                          ctypes.c_void_p(x.data_ptr() + 4),
+                                          ctypes.c_void_p(y.data_ptr()), N, K,
+                                          ctypes.c_void_p(stream))
+            assert st == _kie.KIE_ERR_INVALID_ARG
+        _kie.kie_gemv_f16_noalloc(W, xk, y, stream=stream)
+        torch.cuda.synchronize()
+        got, ref = y.cpu(), y_ref.cpu()
+        assert torch.isfinite(got).all()
+        assert ((got - ref).abs() <= _bound(W, xk)).all(), float((got - ref).abs().max())
+        outs.append(got)
+    assert outs[1].numel() < n_sm
+
+
 def test_noalloc_rejects_sizes_beyond_its_scratch(torch_cuda):
     from persistent_sm_decode_monokernel_b200 import _kie
     lib = _kie.load_library()
