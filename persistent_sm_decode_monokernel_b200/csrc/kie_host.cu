@@ -374,8 +374,7 @@ kie_status kie_create(const kie_model_desc* d, const kie_weights* w, void* kv_ca
     if (cuda_bad(cudaGetDevice(&c->device))) return fail(KIE_ERR_CUDA);
     int n_sm = 0, smem_optin = 0;
     if (cuda_bad(cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, c->device)) ||
-        cuda_bad(cudaDeviceGetAttribute(&smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin,
-                                        c->device)))
+        cuda_bad(kie::dynamic_smem_limit(&smem_optin)))
       return fail(KIE_ERR_CUDA);
 
     // grid: one CTA per SM, but never more CTAs than units of the smallest stage
@@ -588,8 +587,7 @@ kie_status kie_gemv_f16(const void* W, const float* x, float* y, int32_t N, int3
     int dev = 0, n_sm = 0, smem_optin = 0;
     if (cudaGetDevice(&dev) != cudaSuccess ||
         cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
-        cudaDeviceGetAttribute(&smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) !=
-            cudaSuccess)
+        kie::dynamic_smem_limit(&smem_optin) != cudaSuccess)
       return KIE_ERR_CUDA;
     const int grid = std::min(n_sm, N);
     // one layer whose four layer stages own no rows; the LM-head stage is W
@@ -731,8 +729,7 @@ kie_status kie_set_option(kie_ctx* c, kie_option opt, int64_t v) {
         if (c->failed) return set_err(c, KIE_ERR_STATE, "context failed earlier; destroy it");
         if (v < 8192 || v % 512 || v > (1 << 20)) return KIE_ERR_INVALID_ARG;
         int smem_optin = 0;
-        if (cudaDeviceGetAttribute(&smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin,
-                                   c->device) != cudaSuccess)
+        if (kie::dynamic_smem_limit(&smem_optin) != cudaSuccess)
           return set_err(c, KIE_ERR_CUDA, "device attribute query failed");
         kie::SmemLayout sm{};
         int ring = 0;

@@ -54,6 +54,16 @@ enum : int { F_ABORT = 0, F_STOP = 1, F_KVSTEP = 3 };
 // their address space, so the compiler emits shared-memory loads for them.
 extern __shared__ __align__(128) unsigned char kie_smem[];
 
+// The kernel's parameter block, copied to shared memory when a kernel starts:
+// every function reads it with shared-memory loads, including the
+// non-inlined stage functions, which could not know that a reference to the
+// kernel parameter points at constant memory.
+__shared__ MonoParams kie_p;
+// Consumer thread 0's counters: cycles waiting for other CTAs' outputs,
+// cycles waiting for the weight stream, and the ns the current stage waited
+// for the stream (stage trace).
+__shared__ long long kie_ctr[3];
+
 // Views of the dynamic shared memory, always derived from the __shared__
 // symbol so that every access compiles to a shared-memory instruction.
 __device__ __forceinline__ float* sm_xs(const MonoParams& p) {
@@ -79,7 +89,11 @@ __device__ __forceinline__ int* sm_redi2(const MonoParams& p) {
 __device__ __forceinline__ volatile int* sm_flags(const MonoParams& p) {
   return reinterpret_cast<volatile int*>(sm_misc(p) + 80);
 }
-static_assert(kConsumerWarps <= 16 && 88 <= kMiscHead, "scratch words");
+// monotonic start of the chunk on each ring barrier pair (producer only)
+__device__ __forceinline__ uint32_t* sm_starts(const MonoParams& p) {
+  return reinterpret_cast<uint32_t*>(sm_misc(p) + 96);
+}
+static_assert(kConsumerWarps <= 16 && 96 + kRingBars <= kMiscHead, "scratch words");
 // residual stream rows this CTA owns (O / down stages)
 __device__ __forceinline__ float* sm_res_attn(const MonoParams& p) { return sm_misc(p) + kMiscHead; }
 __device__ __forceinline__ float* sm_res_ffn(const MonoParams& p) {
@@ -283,13 +297,20 @@ __device__ __forceinline__ bool global_error(const MonoParams& p) {
 
 // ----------------------------------------------------------------- producer
 
+// Runs inlined in the kernel body (no stack object): `p` is the kernel
+// parameter itself, whose fields compile to constant-bank operands.
 struct Producer {
   const MonoParams& p;
   uint64_t pol;
   uint32_t idx;    // chunks issued
   uint32_t cons;   // chunks known to be consumed
-  uint32_t wend;   // ring write position
-  uint32_t live_off[kRingBars], live_end[kRingBars];
+  uint32_t wend;   // ring write position (offset)
+  // Monotonic write position: bytes placed so far plus the bytes skipped at
+  // each wrap, so chunk i occupies the monotonic range [s_i, e_i) and its ring
+  // bytes are that range modulo the ring size (32-bit, compared by signed
+  // difference: a live span is far below 2^31).  s_i is kept in shared memory
+  // per barrier pair (sm_starts).
+  uint32_t head;
   long long t_wait;  // cycles spent waiting for ring space
   // L2 prefetch of the weight stream (p.l2_prefetch > 0): the bytes from
   // the copy cursor to p.l2_prefetch beyond it are kept requested into L2,
@@ -302,7 +323,7 @@ struct Producer {
   int pf_step;
 
   __device__ explicit Producer(const MonoParams& pp)
-      : p(pp), pol(dev::policy_evict_first()), idx(0), cons(0), wend(0), t_wait(0),
+      : p(pp), pol(dev::policy_evict_first()), idx(0), cons(0), wend(0), head(0), t_wait(0),
         wbase(nullptr), len_layers(0), len_lm(0), pf_ahead(0), pf_off(0), pf_step(0) {}
 
   __device__ long long stage_len(int st) const {
@@ -351,19 +372,34 @@ struct Producer {
     return ok;
   }
 
-  // Frees ring bytes [off, end) and a barrier pair for the next chunk:
-  // waits, oldest first, until no live chunk overlaps the range and fewer
-  // than kRingBars chunks are live.  (When both the live region and the new
-  // chunk wrap, the overlapped chunks are not the oldest, so every live
-  // chunk is checked.)
-  __device__ bool acquire(uint32_t off, uint32_t end) {
+  // Places the next chunk of sz bytes: its ring offset (the consumers'
+  // ring_place) and its monotonic start.
+  __device__ __forceinline__ uint32_t place(uint32_t sz, uint32_t& start) {
+    const uint32_t ring = (uint32_t)p.ring_bytes;
+    uint32_t off = wend;
+    if (wend + sz > ring) {
+      head += ring - wend;   // the bytes skipped at the wrap
+      off = 0;
+    }
+    start = head;
+    head += sz;
+    wend = off + sz;
+    return off;
+  }
+
+  // Frees the ring bytes of a chunk ending at monotonic position `end` and a
+  // barrier pair for it.  The live chunks lie in [oldest start, new start);
+  // once the oldest starts at or after end - ring they all lie in
+  // [end - ring, new start), which shares no ring byte with the new chunk.
+  // Chunks are released in order, so wait oldest first: one comparison per
+  // released chunk.
+  __device__ __forceinline__ bool acquire(uint32_t end) {
+    const uint32_t bound = end - (uint32_t)p.ring_bytes;
+    const uint32_t* starts = sm_starts(p);
     while (cons < idx) {
-      bool blocked = idx - cons >= (uint32_t)kRingBars;
-      for (uint32_t j = cons; j < idx && !blocked; ++j) {
-        const uint32_t b = j & (kRingBars - 1);
-        blocked = off < live_end[b] && live_off[b] < end;
-      }
-      if (!blocked) break;
+      if (idx - cons < (uint32_t)kRingBars &&
+          (int)(starts[cons & (kRingBars - 1)] - bound) >= 0)
+        break;
       if (!wait_consumed(cons)) return false;
       ++cons;
     }
@@ -373,14 +409,14 @@ struct Producer {
   // One chunk = one bulk copy of the next `sz` bytes of the CTA's stream.
   __device__ bool chunk(const unsigned char*& src, uint32_t sz) {
     if (sm_flags(p)[F_STOP]) return false;
-    const uint32_t off = ring_place(wend, sz, (uint32_t)p.ring_bytes);
-    if (!acquire(off, off + sz)) return false;
+    uint32_t start;
+    const uint32_t off = place(sz, start);
+    if (!acquire(start + sz)) return false;
     const uint32_t b = idx & (kRingBars - 1);
     const uint32_t full = sm_full_s(p) + 8 * b;
     dev::mbar_arrive_expect_tx(full, sz);
     dev::bulk_g2s(sm_ring_s(p) + off, src, sz, full, pol);
-    live_off[b] = off;
-    live_end[b] = off + sz;
+    sm_starts(p)[b] = start;
     src += sz;
     ++idx;
     return true;
@@ -391,14 +427,14 @@ struct Producer {
   // consumers fill the remaining rows.
   __device__ bool tile(const unsigned char* src, uint32_t bytes, uint32_t alloc) {
     if (sm_flags(p)[F_STOP]) return false;
-    const uint32_t off = ring_place(wend, alloc, (uint32_t)p.ring_bytes);
-    if (!acquire(off, off + alloc)) return false;
+    uint32_t start;
+    const uint32_t off = place(alloc, start);
+    if (!acquire(start + alloc)) return false;
     const uint32_t b = idx & (kRingBars - 1);
     const uint32_t full = sm_full_s(p) + 8 * b;
     dev::mbar_arrive_expect_tx(full, bytes);
     if (bytes > 0) dev::bulk_g2s(sm_ring_s(p) + off, src, bytes, full, pol);
-    live_off[b] = off;
-    live_end[b] = off + alloc;
+    sm_starts(p)[b] = start;
     ++idx;
     return true;
   }
@@ -582,28 +618,27 @@ struct AttnSmem {
   }
 };
 
+// Consumer state lives in registers and in the stack frame of the kernel
+// (the object's address is passed to the non-inlined stage functions), so it
+// is kept to the ring cursors and the (step, layer, stage) of error reports:
+// the parameter block is read from its shared-memory copy (kie_p), thread
+// indices come from threadIdx, and thread 0's cycle counters live in shared
+// memory (kie_ctr).  A large frame would be 128 bytes per 4-byte member and
+// warp in L1, where misses cost a round trip to L2 at every stage entry.
 struct Consumer {
-  const MonoParams& p;
-  int tid, warp, lane;
   uint32_t cidx;   // next chunk to wait for
   uint32_t crel;   // next chunk to release (stages release their chunks in order)
   uint32_t cend;   // ring read position (mirrors the producer's placement)
-  long long t_sync, t_stream;
-  long long w_stage;       // ns warp 0 waited for streamed chunks in the current stage (trace)
   int step, layer, stage;  // for error reports
 
-  __device__ explicit Consumer(const MonoParams& pp)
-      : p(pp), cidx(0), crel(0), cend(0), t_sync(0), t_stream(0), w_stage(0), step(0), layer(0),
-        stage(0) {
-    tid = threadIdx.x;
-    warp = tid >> 5;
-    lane = tid & 31;
-  }
+  __device__ Consumer() : cidx(0), crel(0), cend(0), step(0), layer(0), stage(0) {}
 
   // Stage trace (measurement, tid 0 only): per step kTracePerLayer slots
   // per layer (stage boundaries, attention sub-steps, stream waits; the
   // layout is documented with kie_set_trace) + 4 for the LM head.
   __device__ __forceinline__ void trace_put(int ev, unsigned long long v) const {
+    const MonoParams& p = kie_p;
+    const int tid = (int)threadIdx.x;
     if (p.trace && tid == 0 && (p.trace_cta < 0 || (int)blockIdx.x == p.trace_cta) &&
         step < p.trace_steps) {
       const int per = p.L * kTracePerLayer + 4;
@@ -613,14 +648,18 @@ struct Consumer {
     }
   }
   __device__ __forceinline__ void trace(int ev) const {
+    const MonoParams& p = kie_p;
     if (p.trace)
       trace_put(ev, p.trace_clock ? (unsigned long long)clock64()
                                   : (unsigned long long)dev::globaltimer());
   }
   // Stream wait of the stage just finished (slots 16 + stage), then reset.
   __device__ __forceinline__ void trace_stream_wait(int st) {
-    if (p.trace) trace_put(16 + st, (unsigned long long)w_stage);
-    w_stage = 0;
+    const MonoParams& p = kie_p;
+    if (threadIdx.x == 0) {
+      if (p.trace) trace_put(16 + st, (unsigned long long)kie_ctr[2]);
+      kie_ctr[2] = 0;
+    }
   }
   __device__ __forceinline__ void trace_loaded() const {
     switch (stage) {
@@ -633,12 +672,15 @@ struct Consumer {
   }
 
   __device__ __forceinline__ bool fault_here(int st) const {
+    const MonoParams& p = kie_p;
     return p.fault_cta == (int)blockIdx.x && p.fault_step == step && p.fault_layer == layer &&
            p.fault_stage == st;
   }
 
   // Slow path of a chunk wait: bounded spin on the full barrier.
   __device__ __noinline__ bool wait_slow(uint32_t bar, uint32_t par) {
+    const MonoParams& p = kie_p;
+    const int tid = (int)threadIdx.x;
     const long long c0 = clock64();
     const long long t0 = dev::globaltimer();
     bool ok = true;
@@ -658,14 +700,16 @@ struct Consumer {
       }
     }
     if (tid == 0) {
-      t_stream += clock64() - c0;
-      if (p.trace) w_stage += dev::globaltimer() - t0;
+      kie_ctr[1] += clock64() - c0;
+      if (p.trace) kie_ctr[2] += dev::globaltimer() - t0;
     }
     return ok;
   }
 
   // ---- ring: waits for the next chunk (sz bytes) and returns its offset
   __device__ __forceinline__ bool wait_chunk(uint32_t sz, uint32_t& off) {
+    const MonoParams& p = kie_p;
+    const int tid = (int)threadIdx.x;
     off = ring_place(cend, sz, (uint32_t)p.ring_bytes);
     const uint32_t bar = sm_full_s(p) + 8 * (cidx & (kRingBars - 1));
     const uint32_t par = (cidx / kRingBars) & 1u;
@@ -690,13 +734,15 @@ struct Consumer {
       }
     }
     if (tid == 0) {
-      t_stream += clock64() - c0;
-      if (p.trace) w_stage += dev::globaltimer() - t0;
+      kie_ctr[1] += clock64() - c0;
+      if (p.trace) kie_ctr[2] += dev::globaltimer() - t0;
     }
     return ok;
   }
   // Releases the oldest chunk this warp waited for and has not released.
   __device__ __forceinline__ void release_chunk() {
+    const MonoParams& p = kie_p;
+    const int lane = (int)(threadIdx.x & 31);
     __syncwarp();
     if (lane == 0) dev::mbar_arrive(sm_empty_s(p) + 8 * (crel & (kRingBars - 1)));
     ++crel;
@@ -711,6 +757,7 @@ struct Consumer {
   template <int NB>
   __device__ __forceinline__ bool poll_pairs(const u64* src, const int (&k2)[NB], int n2,
                                              unsigned tag, ulonglong2 (&v)[NB], int where) {
+    const MonoParams& p = kie_p;
     unsigned pend = 0;
 #pragma unroll
     for (int b = 0; b < NB; ++b)
@@ -758,6 +805,7 @@ struct Consumer {
   // ---- GEMV input vector in shared memory: fp16, natural order (lane l of
   // piece q reads elements 256q + 8l .. +8 with one 16-byte load).
   __device__ __forceinline__ __half2* xs16() const {
+    const MonoParams& p = kie_p;
     return reinterpret_cast<__half2*>(kie_smem + p.sm.xs_off);
   }
 
@@ -782,6 +830,8 @@ struct Consumer {
   // overlap.  Returns false (uniformly) on abort.
   __device__ __noinline__ bool load_vec(const u64* src, unsigned tag, const __half* emb, int K,
                            const __half* gain, float& ss, int where) {
+    const MonoParams& p = kie_p;
+    const int tid = (int)threadIdx.x, warp = (int)(threadIdx.x >> 5), lane = (int)(threadIdx.x & 31);
     constexpr int NB = 8;
     const long long c0 = clock64();
     float acc = 0.f;
@@ -817,7 +867,7 @@ struct Consumer {
 #pragma unroll
     for (int w = 0; w < kConsumerWarps; ++w) t += sm_red(p)[w];
     ss = t;
-    if (tid == 0) t_sync += clock64() - c0;
+    if (tid == 0) kie_ctr[0] += clock64() - c0;
     trace_loaded();
     return !bad;
   }
@@ -825,6 +875,7 @@ struct Consumer {
   // Polls n2 pairs of tagged words into dst[0 .. 2*n2) (times `scale`).
   __device__ __noinline__ bool load_pairs(const u64* src, unsigned tag, int n2, float* dst,
                                           float scale, int where) {
+    const int tid = (int)threadIdx.x;
     constexpr int NB = 4;
     for (int base = tid; base < n2; base += kConsumerThreads * NB) {
       ulonglong2 v[NB];
@@ -856,6 +907,8 @@ struct Consumer {
 
   // Fills the stage plans (threads 0..N_STAGES-1; the caller synchronises).
   __device__ void make_plans() {
+    const MonoParams& p = kie_p;
+    const int tid = (int)threadIdx.x;
     if (tid < N_STAGES) {
       const int st = tid;
       const int2 r = p.ranges[st * p.grid + blockIdx.x];
@@ -891,7 +944,7 @@ struct Consumer {
   // timing.  Ring positions and the parameter block are held in registers
   // for the whole stage; one barrier at the end.
   __device__ __noinline__ bool gemv(int st) {
-    const MonoParams& p = this->p;
+    const MonoParams& p = kie_p;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const StagePlan pl = sm_plan(p)[st];
     const unsigned char* ring = sm_ring(p);
@@ -1068,6 +1121,7 @@ struct Consumer {
 
   // Raw dot product of row k (0-based within the CTA's rows) of the last gemv.
   __device__ __forceinline__ float row_result(const StagePlan& pl, int k) const {
+    const MonoParams& p = kie_p;
     const int tb = pl.nfull * kGroupRows;
     if (pl.tail > 0 && pl.t_lw > 0 && k >= tb) {
       const int base = (k - tb) << pl.t_lw;
@@ -1086,6 +1140,8 @@ struct Consumer {
 
   // RMSNorm + QKV GEMV + RoPE + KV append.
   __device__ __noinline__ bool stage_qkv(const LayerW& w, int tok, int pos, unsigned tag) {
+    const MonoParams& p = kie_p;
+    const int tid = (int)threadIdx.x;
     stage = ST_QKV;
     const int2 r = p.ranges[ST_QKV * p.grid + blockIdx.x];
     float ss;
@@ -1154,6 +1210,8 @@ struct Consumer {
   // abort.
   template <int HD>
   __device__ __noinline__ bool attn_combine(const AttnItem& it, unsigned tag) {
+    const MonoParams& p = kie_p;
+    const int tid = (int)threadIdx.x;
     constexpr int ROW = 2 + HD / 2;          // tagged words per (item, head) row
     const int G = p.G, nsplit = it.nsplit, j = it.j;
     const int W = (((HD + nsplit - 1) / nsplit) + 3) & ~3;
@@ -1242,6 +1300,8 @@ struct Consumer {
   //           the V tile; warp w owns HD/8 dims.
   template <int HD>
   __device__ __noinline__ bool stage_attn(int pos, unsigned tag) {
+    const MonoParams& p = kie_p;
+    const int tid = (int)threadIdx.x, warp = (int)(threadIdx.x >> 5), lane = (int)(threadIdx.x & 31);
     stage = 5;
     const AttnItem it = attn_item(p, pos);
     if (!it.valid) return true;
@@ -1301,7 +1361,7 @@ struct Consumer {
       a.lrun[tid] = 0.f;
     }
     if (dev::consumer_sync_or(bad)) return false;
-    if (tid == 0) t_sync += clock64() - c0;
+    if (tid == 0) kie_ctr[0] += clock64() - c0;
     trace(10);
 
     const int gid = lane >> 2, tig = lane & 3;
@@ -1449,6 +1509,8 @@ struct Consumer {
 
   // O projection + residual -> x_ffn.
   __device__ bool stage_o(const LayerW& w, int tok, unsigned tag) {
+    const MonoParams& p = kie_p;
+    const int tid = (int)threadIdx.x;
     stage = ST_O;
     const int2 r = p.ranges[ST_O * p.grid + blockIdx.x];
     if (r.y <= r.x) return true;
@@ -1469,6 +1531,8 @@ struct Consumer {
 
   // RMSNorm + gate/up GEMV + SwiGLU -> h.
   __device__ bool stage_gu(const LayerW& w, unsigned tag) {
+    const MonoParams& p = kie_p;
+    const int tid = (int)threadIdx.x;
     stage = ST_GU;
     const int2 r = p.ranges[ST_GU * p.grid + blockIdx.x];
     if (r.y <= r.x) return true;
@@ -1489,6 +1553,8 @@ struct Consumer {
 
   // Down GEMV + residual -> x_attn (input of the next layer).
   __device__ bool stage_down(const LayerW& w, unsigned tag, unsigned tag_next) {
+    const MonoParams& p = kie_p;
+    const int tid = (int)threadIdx.x;
     stage = ST_DOWN;
     const int2 r = p.ranges[ST_DOWN * p.grid + blockIdx.x];
     if (r.y <= r.x) return true;
@@ -1527,6 +1593,7 @@ struct Consumer {
   // under key (seed, 0), mapped to the open interval (0, 1).  The argmax of
   // the noisy scores is a draw from softmax(logits / T).
   __device__ __forceinline__ float pick_score(float v, int u, int pos) const {
+    const MonoParams& p = kie_p;
     if (!p.sample) return v;
     const unsigned long long w =
         dev::philox4x64_10_word((unsigned long long)(u >> 2), (unsigned long long)pos, p.seed, u & 3);
@@ -1534,6 +1601,7 @@ struct Consumer {
     return (float)((double)v * p.inv_temp - log(-log(uu)));
   }
   __device__ __forceinline__ bool is_eos(int t) const {
+    const MonoParams& p = kie_p;
     for (int k = 0; k < p.n_eos; ++k)
       if (t == p.eos_ids[k]) return true;
     return false;
@@ -1544,6 +1612,8 @@ struct Consumer {
   // on abort; *tok_out gets the picked id (uniform across the grid).
   __device__ __noinline__ bool stage_lm(bool pick, int step_row, unsigned tag, int pos,
                                         int* tok_out) {
+    const MonoParams& p = kie_p;
+    const int tid = (int)threadIdx.x, warp = (int)(threadIdx.x >> 5), lane = (int)(threadIdx.x & 31);
     stage = ST_LM;
     float best = -INFINITY;
     int bi = INT_MAX;
@@ -1627,7 +1697,7 @@ struct Consumer {
       }
     *tok_out = ib;
     if (tid == 0) {
-      t_sync += clock64() - c0;
+      kie_ctr[0] += clock64() - c0;
       // this step's KV writes of every CTA are now visible to this CTA:
       // the producer may copy them for the next step
       dev::st_release_cta(sm_flags(p) + F_KVSTEP, step + 1);
@@ -1637,6 +1707,7 @@ struct Consumer {
 
   // Walks a stage's chunk sequence without computing (stream-only timing).
   __device__ __noinline__ bool skip_stage(int st, int ub, int ue) {
+    const MonoParams& p = kie_p;
     const int R = range_rows(p, st, ub, ue);
     const int kp = stage_k(p, st) / kPieceElems;
     bool bad = false;
@@ -1652,6 +1723,8 @@ struct Consumer {
   // Standalone GEMV engine run: y = W x over the LM-head stage's rows,
   // `iters` times (mode 0: stream the weights only, mode 1: full GEMV).
   __device__ void gemv_bench(int mode, const float* x, float* y, int iters) {
+    const MonoParams& p = kie_p;
+    const int tid = (int)threadIdx.x;
     make_plans();
     const int2 r = p.ranges[ST_LM * p.grid + blockIdx.x];
     const int K = p.d;
@@ -1669,12 +1742,14 @@ struct Consumer {
     if (tid == 0) {
       sm_flags(p)[F_STOP] = 1;
       u64* st = p.cta_stats + kStatsPerCta * blockIdx.x;
-      st[2] = (u64)t_stream;
+      st[2] = (u64)kie_ctr[1];
     }
   }
 
   template <int HD>
   __device__ void run() {
+    const MonoParams& p = kie_p;
+    const int tid = (int)threadIdx.x;
     make_plans();
     dev::consumer_sync();
     const long long c_begin = clock64();
@@ -1712,7 +1787,7 @@ struct Consumer {
       trace(0);
       const bool lm_ok = stage_lm(pick, i - p.lm_from, epoch_of(p, i, p.L), pos, &next);
       trace(3);
-      w_stage = 0;
+      if (tid == 0) kie_ctr[2] = 0;
       if (!lm_ok) {
         ok = false;
         break;
@@ -1728,17 +1803,20 @@ struct Consumer {
     if (tid == 0) {
       u64* st = p.cta_stats + kStatsPerCta * blockIdx.x;
       st[0] = (u64)(clock64() - c_begin);
-      st[1] = (u64)t_sync;
-      st[2] = (u64)t_stream;
+      st[1] = (u64)kie_ctr[0];
+      st[2] = (u64)kie_ctr[1];
       st[4] = (u64)done;
     }
   }
 };
 
-}  // namespace
-
-template <int HD>
-__global__ void __launch_bounds__(kThreads, 1) kie_monokernel(const __grid_constant__ MonoParams p) {
+// Common start of the persistent kernels: the parameter block's shared copy,
+// the ring barriers, the flags and thread 0's counters.
+__device__ __forceinline__ void kernel_setup(const MonoParams& p) {
+  static_assert(sizeof(MonoParams) % 4 == 0, "parameter block copy");
+  const unsigned* src = reinterpret_cast<const unsigned*>(&p);
+  unsigned* dst = reinterpret_cast<unsigned*>(&kie_p);
+  for (int i = threadIdx.x; i < (int)(sizeof(MonoParams) / 4); i += blockDim.x) dst[i] = src[i];
   if (threadIdx.x == 0) {
     for (int s = 0; s < kRingBars; ++s) {
       dev::mbar_init(sm_full_s(p) + 8 * s, 1);
@@ -1747,9 +1825,17 @@ __global__ void __launch_bounds__(kThreads, 1) kie_monokernel(const __grid_const
     sm_flags(p)[F_ABORT] = 0;
     sm_flags(p)[F_STOP] = 0;
     sm_flags(p)[F_KVSTEP] = 0;
+    kie_ctr[0] = kie_ctr[1] = kie_ctr[2] = 0;
     dev::mbar_fence_init();
   }
   __syncthreads();
+}
+
+}  // namespace
+
+template <int HD>
+__global__ void __launch_bounds__(kThreads, 1) kie_monokernel(const __grid_constant__ MonoParams p) {
+  kernel_setup(p);
   if (threadIdx.x >= kConsumerThreads) {
     dev::regs_dec<kRegsProducer>();
     if (threadIdx.x == kConsumerThreads) {
@@ -1759,24 +1845,14 @@ __global__ void __launch_bounds__(kThreads, 1) kie_monokernel(const __grid_const
     return;
   }
   dev::regs_inc<kRegsConsumer>();
-  Consumer c(p);
+  Consumer c;
   c.run<HD>();
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
     kie_gemv_kernel(const __grid_constant__ MonoParams p, int mode, const float* x, float* y,
                     int iters) {
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < kRingBars; ++s) {
-      dev::mbar_init(sm_full_s(p) + 8 * s, 1);
-      dev::mbar_init(sm_empty_s(p) + 8 * s, kConsumerWarps);
-    }
-    sm_flags(p)[F_ABORT] = 0;
-    sm_flags(p)[F_STOP] = 0;
-    sm_flags(p)[F_KVSTEP] = 0;
-    dev::mbar_fence_init();
-  }
-  __syncthreads();
+  kernel_setup(p);
   if (threadIdx.x >= kConsumerThreads) {
     dev::regs_dec<kRegsProducer>();
     if (threadIdx.x == kConsumerThreads) {
@@ -1792,7 +1868,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     return;
   }
   dev::regs_inc<kRegsConsumer>();
-  Consumer c(p);
+  Consumer c;
   c.gemv_bench(mode, x, y, iters);
 }
 
@@ -1814,18 +1890,33 @@ cudaError_t repack_launch(const MonoParams& p, unsigned char* packed, cudaStream
   return cudaGetLastError();
 }
 
-// Lets kie_gemv_kernel use up to the current device's opt-in maximum of
-// dynamic shared memory.  Always the same value, so calls from several host
-// threads (the allocating and the no-allocation GEMV entry points) cannot
-// undo each other's setting between configure and launch.
-cudaError_t gemv_configure() {
+cudaError_t dynamic_smem_limit(int* out) {
   int dev = 0, optin = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e == cudaSuccess)
     e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+  size_t stat = 0;
+  for (const void* fn : {(const void*)kie_monokernel<64>, (const void*)kie_monokernel<128>,
+                         (const void*)kie_gemv_kernel}) {
+    cudaFuncAttributes a{};
+    if (e == cudaSuccess) e = cudaFuncGetAttributes(&a, fn);
+    stat = a.sharedSizeBytes > stat ? a.sharedSizeBytes : stat;
+  }
+  if (e != cudaSuccess) return e;
+  *out = optin - (int)stat;
+  return cudaSuccess;
+}
+
+// Lets kie_gemv_kernel use all the dynamic shared memory it may have on the
+// current device.  Always the same value, so calls from several host
+// threads (the allocating and the no-allocation GEMV entry points) cannot
+// undo each other's setting between configure and launch.
+cudaError_t gemv_configure() {
+  int limit = 0;
+  cudaError_t e = dynamic_smem_limit(&limit);
   if (e != cudaSuccess) return e;
   return cudaFuncSetAttribute((const void*)kie_gemv_kernel,
-                              cudaFuncAttributeMaxDynamicSharedMemorySize, optin);
+                              cudaFuncAttributeMaxDynamicSharedMemorySize, limit);
 }
 
 cudaError_t gemv_launch(const MonoParams& p, int mode, const float* x, float* y, int iters,

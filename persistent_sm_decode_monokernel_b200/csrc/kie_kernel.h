@@ -7,6 +7,11 @@
 
 namespace kie {
 
+// Dynamic shared memory the persistent kernels may use per CTA on the
+// current device: the opt-in maximum per block minus their static shared
+// memory (the parameter block's shared copy).
+cudaError_t dynamic_smem_limit(int* out);
+
 // Sets the dynamic shared-memory limit of the kernel instance for head
 // dimension `hd` (64 or 128) and reports how many CTAs fit on one SM.
 cudaError_t mono_configure(int hd, int smem_bytes, int* blocks_per_sm);

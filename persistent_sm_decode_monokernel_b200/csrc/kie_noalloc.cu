@@ -140,8 +140,7 @@ kie_status kie_gemv_f16_noalloc(const void* W, const float* x, float* y, int32_t
     int dev = 0, n_sm = 0, smem_optin = 0;
     if (cudaGetDevice(&dev) != cudaSuccess ||
         cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
-        cudaDeviceGetAttribute(&smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) !=
-            cudaSuccess)
+        kie::dynamic_smem_limit(&smem_optin) != cudaSuccess)
       return KIE_ERR_CUDA;
     const int grid = std::min(std::min(n_sm, kMaxCtas), (int)N);
 

@@ -3,15 +3,24 @@ CPU.
 
 The producer lane places each chunk (a weight chunk or an attention tile)
 right after the previous one, or at 0 when it would run past the end of the
-ring, and before issuing the copy waits, oldest first, until fewer than 16
-chunks are live and no live chunk overlaps the new range (the kernel's
-`ring_place` and `Producer::acquire`).  The consumers walk the same chunk
-sequence and recompute every offset themselves.  Random interleavings of the
-two sides must never let a copy land on bytes a consumer has not released,
-never reuse one of the 16 barrier pairs while its chunk is live, and always
-give both sides the same offsets.  Checking only the oldest live chunk for
-overlap is a plausible simplification that is wrong when both the live
-region and the new chunk wrap; the model must catch it.
+ring (the kernel's `ring_place`).  Besides the ring offset it keeps a
+monotonic byte position that also counts the bytes skipped at each wrap, so
+chunk i occupies the monotonic range [s_i, e_i) and its ring bytes are that
+range modulo the ring size R.  The live chunks of a new chunk [s, e) lie in
+[s_oldest, s); once the oldest live chunk starts at or after e - R they all
+lie in [e - R, s), which together with [s, e) spans exactly R bytes, so none
+of them shares a ring byte with the new chunk.  Chunks are released in
+order, so the producer waits oldest first until the oldest live chunk starts
+at or after e - R and fewer than 16 chunks are live (`Producer::acquire`):
+one comparison per released chunk.  The
+consumers walk the same chunk sequence and recompute every offset
+themselves.  Random interleavings of the two sides must never let a copy
+land on bytes a consumer has not released, never reuse one of the 16
+barrier pairs while its chunk is live, and always give both sides the same
+offsets.  Two plausible slips must be caught: checking only the oldest live
+chunk for overlap in ring offsets (wrong when both the live region and the
+new chunk wrap), and comparing the oldest start against s - R instead of
+e - R.
 """
 import random
 
@@ -25,21 +34,32 @@ def place(wend: int, size: int, ring: int):
     return off, off + size
 
 
-def producer(sizes, ring, shared, check_all=True):
-    """Generator: one yield per step that may block on the consumers."""
+def producer(sizes, ring, shared, rule="monotonic"):
+    """Generator: one yield per step that may block on the consumers.
+
+    rule "monotonic": the kernel's rule (see the module docstring);
+    "oldest_offsets": overlap of the new range with the oldest live chunk's
+    ring offsets only; "start_minus_ring": the monotonic rule with s - R in
+    place of e - R."""
     idx = cons = 0
     wend = 0
+    head = 0                          # monotonic write position
     live = [(0, 0)] * N_BARS
+    starts = [0] * N_BARS
     for size in sizes:
+        prev = wend
         off, wend = place(wend, size, ring)
+        if off == 0 and prev != 0:
+            head += ring - prev       # bytes skipped at the wrap
+        s, e = head, head + size
+        head = e
         while cons < idx:
-            blocked = idx - cons >= N_BARS
-            span = range(cons, idx) if check_all else range(cons, cons + 1)
-            for j in span:
-                if blocked:
-                    break
-                lo, hi = live[j % N_BARS]
-                blocked = off < hi and lo < off + size
+            if rule == "oldest_offsets":
+                lo, hi = live[cons % N_BARS]
+                blocked = idx - cons >= N_BARS or (off < hi and lo < off + size)
+            else:
+                bound = e - ring if rule == "monotonic" else s - ring
+                blocked = idx - cons >= N_BARS or starts[cons % N_BARS] < bound
             if not blocked:
                 break
             while shared["consumed"] <= cons:      # wait until chunk `cons` is released
@@ -52,15 +72,16 @@ def producer(sizes, ring, shared, check_all=True):
         assert idx - shared["consumed"] < N_BARS, "barrier pair reused while live"
         shared["where"][idx] = (off, off + size)
         live[idx % N_BARS] = (off, off + size)
+        starts[idx % N_BARS] = s
         idx += 1
         shared["issued"] = idx
         yield
 
 
-def run(sizes, ring, seed, check_all=True):
+def run(sizes, ring, seed, rule="monotonic"):
     rnd = random.Random(seed)
     shared = {"consumed": 0, "issued": 0, "where": {}}
-    prod = producer(sizes, ring, shared, check_all)
+    prod = producer(sizes, ring, shared, rule)
     finished = False
     cend = 0
     for _ in range(10 ** 6):
@@ -93,9 +114,10 @@ def test_ring_protocol_random_interleavings():
         run(sizes, ring, seed)
 
 
-def test_checking_only_the_oldest_chunk_is_caught():
+@pytest.mark.parametrize("rule", ["oldest_offsets", "start_minus_ring"])
+def test_plausible_wrong_rules_are_caught(rule):
     with pytest.raises(AssertionError) as e:
         for seed in range(600):
             sizes, ring = _case(seed)
-            run(sizes, ring, seed, check_all=False)
+            run(sizes, ring, seed, rule=rule)
     assert "overlap" in str(e.value), str(e.value)
