@@ -63,6 +63,17 @@ __shared__ MonoParams kie_p;
 // cycles waiting for the weight stream, and the ns the current stage waited
 // for the stream (stage trace).
 __shared__ long long kie_ctr[3];
+// Ring cursors of the consumer warps, the same in every consumer thread:
+// next chunk to wait for, next chunk to release (chunks are released in
+// order), ring read position (mirrors the producer's placement).  Every
+// consumer thread reads them at the start of a stage, after a barrier;
+// consumer thread 0 writes them back after the stage's last barrier, and the
+// next stage reads them only after another barrier.
+__shared__ uint32_t kie_cur[3];
+// (step, layer, stage) of the consumer warps, written by consumer thread 0
+// only: exact for thread 0 (the stage trace), and for the other threads the
+// position an error report names (possibly one stage behind).
+__shared__ int kie_at[3];
 
 // Views of the dynamic shared memory, always derived from the __shared__
 // symbol so that every access compiles to a shared-memory instruction.
@@ -618,20 +629,16 @@ struct AttnSmem {
   }
 };
 
-// Consumer state lives in registers and in the stack frame of the kernel
-// (the object's address is passed to the non-inlined stage functions), so it
-// is kept to the ring cursors and the (step, layer, stage) of error reports:
-// the parameter block is read from its shared-memory copy (kie_p), thread
-// indices come from threadIdx, and thread 0's cycle counters live in shared
-// memory (kie_ctr).  A large frame would be 128 bytes per 4-byte member and
-// warp in L1, where misses cost a round trip to L2 at every stage entry.
+// The consumer warps' code.  It keeps no state in the object: a non-inlined
+// member function reaches members through a pointer to the stack, and stack
+// lines that miss the small L1 left beside the shared-memory carve-out cost
+// an L2 round trip at every stage entry.  The parameter block is read from
+// its shared-memory copy (kie_p), thread indices come from threadIdx, the
+// ring cursors, the (step, layer, stage) position and thread 0's counters
+// live in shared memory (kie_cur, kie_at, kie_ctr), and the stage functions
+// get the layer and the fault-hook decision as arguments.
 struct Consumer {
-  uint32_t cidx;   // next chunk to wait for
-  uint32_t crel;   // next chunk to release (stages release their chunks in order)
-  uint32_t cend;   // ring read position (mirrors the producer's placement)
-  int step, layer, stage;  // for error reports
-
-  __device__ Consumer() : cidx(0), crel(0), cend(0), step(0), layer(0), stage(0) {}
+  __device__ Consumer() {}
 
   // Stage trace (measurement, tid 0 only): per step kTracePerLayer slots
   // per layer (stage boundaries, attention sub-steps, stream waits; the
@@ -640,7 +647,8 @@ struct Consumer {
     const MonoParams& p = kie_p;
     const int tid = (int)threadIdx.x;
     if (p.trace && tid == 0 && (p.trace_cta < 0 || (int)blockIdx.x == p.trace_cta) &&
-        step < p.trace_steps) {
+        kie_at[0] < p.trace_steps) {
+      const int step = kie_at[0], layer = kie_at[1];
       const int per = p.L * kTracePerLayer + 4;
       const int row = p.trace_cta < 0 ? step * p.grid + (int)blockIdx.x : step;
       const int idx = row * per + (layer < p.L ? layer * kTracePerLayer : p.L * kTracePerLayer) + ev;
@@ -662,7 +670,7 @@ struct Consumer {
     }
   }
   __device__ __forceinline__ void trace_loaded() const {
-    switch (stage) {
+    switch (kie_at[2]) {
       case ST_QKV: trace(1); break;
       case ST_O: trace(4); break;
       case ST_GU: trace(6); break;
@@ -671,10 +679,17 @@ struct Consumer {
     }
   }
 
-  __device__ __forceinline__ bool fault_here(int st) const {
+  // Test hook: the stage whose publication this CTA withholds at (step i,
+  // layer l), or -1.
+  __device__ __forceinline__ static int fault_stage_at(int i, int l) {
     const MonoParams& p = kie_p;
-    return p.fault_cta == (int)blockIdx.x && p.fault_step == step && p.fault_layer == layer &&
-           p.fault_stage == st;
+    return (p.fault_cta == (int)blockIdx.x && p.fault_step == i && p.fault_layer == l)
+               ? p.fault_stage
+               : -1;
+  }
+  // Sets the stage of the position reported by errors and traces.
+  __device__ __forceinline__ static void at_stage(int st) {
+    if (threadIdx.x == 0) kie_at[2] = st;
   }
 
   // Slow path of a chunk wait: bounded spin on the full barrier.
@@ -692,7 +707,7 @@ struct Consumer {
           break;
         }
         if (dev::globaltimer() - t0 > p.timeout_ns) {
-          raise_error(p, DEV_TIMEOUT, step, layer, stage, 3);
+          raise_error(p, DEV_TIMEOUT, kie_at[0], kie_at[1], kie_at[2], 3);
           sm_flags(p)[F_ABORT] = 1;
           ok = false;
           break;
@@ -706,8 +721,10 @@ struct Consumer {
     return ok;
   }
 
-  // ---- ring: waits for the next chunk (sz bytes) and returns its offset
-  __device__ __forceinline__ bool wait_chunk(uint32_t sz, uint32_t& off) {
+  // ---- ring: waits for the next chunk (sz bytes) and returns its offset;
+  // cidx / cend: the caller's copies of the wait and read-position cursors
+  __device__ __forceinline__ bool wait_chunk(uint32_t sz, uint32_t& off, uint32_t& cidx,
+                                             uint32_t& cend) {
     const MonoParams& p = kie_p;
     const int tid = (int)threadIdx.x;
     off = ring_place(cend, sz, (uint32_t)p.ring_bytes);
@@ -726,7 +743,7 @@ struct Consumer {
           break;
         }
         if (dev::globaltimer() - t0 > p.timeout_ns) {
-          raise_error(p, DEV_TIMEOUT, step, layer, stage, 3);
+          raise_error(p, DEV_TIMEOUT, kie_at[0], kie_at[1], kie_at[2], 3);
           sm_flags(p)[F_ABORT] = 1;
           ok = false;
           break;
@@ -739,8 +756,9 @@ struct Consumer {
     }
     return ok;
   }
-  // Releases the oldest chunk this warp waited for and has not released.
-  __device__ __forceinline__ void release_chunk() {
+  // Releases the oldest chunk this warp waited for and has not released
+  // (crel: the caller's copy of the release cursor).
+  __device__ __forceinline__ void release_chunk(uint32_t& crel) {
     const MonoParams& p = kie_p;
     const int lane = (int)(threadIdx.x & 31);
     __syncwarp();
@@ -778,7 +796,7 @@ struct Consumer {
       }
       if (!pend) return true;
       if (newer) {
-        raise_error(p, DEV_PROTOCOL, step, layer, stage, where);
+        raise_error(p, DEV_PROTOCOL, kie_at[0], kie_at[1], kie_at[2], where);
         sm_flags(p)[F_ABORT] = 1;
         return false;
       }
@@ -790,7 +808,7 @@ struct Consumer {
           return false;
         }
         if (dev::globaltimer() - t0 > p.timeout_ns) {
-          raise_error(p, DEV_TIMEOUT, step, layer, stage, where);
+          raise_error(p, DEV_TIMEOUT, kie_at[0], kie_at[1], kie_at[2], where);
           sm_flags(p)[F_ABORT] = 1;
           return false;
         }
@@ -952,7 +970,7 @@ struct Consumer {
     float* rowacc = sm_rowacc(p);
     const uint32_t ring_bytes = (uint32_t)p.ring_bytes;
     const uint32_t full_s = sm_full_s(p), empty_s = sm_empty_s(p);
-    uint32_t ci = cidx, cr = crel, ce = cend;
+    uint32_t ci = kie_cur[0], cr = kie_cur[1], ce = kie_cur[2];
     bool bad = false;
     auto wait = [&](uint32_t sz, uint32_t& off) -> bool {
       off = ring_place(ce, sz, ring_bytes);
@@ -1113,10 +1131,13 @@ struct Consumer {
         }
       }
     }
-    cidx = ci;
-    crel = cr;
-    cend = ce;
-    return !dev::consumer_sync_or(bad);
+    const bool any_bad = dev::consumer_sync_or(bad);
+    if (threadIdx.x == 0) {
+      kie_cur[0] = ci;
+      kie_cur[1] = cr;
+      kie_cur[2] = ce;
+    }
+    return !any_bad;
   }
 
   // Raw dot product of row k (0-based within the CTA's rows) of the last gemv.
@@ -1139,10 +1160,11 @@ struct Consumer {
   // ---- stage bodies -------------------------------------------------------
 
   // RMSNorm + QKV GEMV + RoPE + KV append.
-  __device__ __noinline__ bool stage_qkv(const LayerW& w, int tok, int pos, unsigned tag) {
+  __device__ __noinline__ bool stage_qkv(const LayerW& w, int layer, int tok, int pos, unsigned tag,
+                                         bool skip) {
     const MonoParams& p = kie_p;
     const int tid = (int)threadIdx.x;
-    stage = ST_QKV;
+    at_stage(ST_QKV);
     const int2 r = p.ranges[ST_QKV * p.grid + blockIdx.x];
     float ss;
     const __half* emb = layer == 0 ? p.tok_emb + (size_t)tok * p.d : nullptr;
@@ -1162,7 +1184,6 @@ struct Consumer {
     const StagePlan pl = sm_plan(p)[ST_QKV];
     const float rs = 1.0f / sqrtf(ss / (float)p.d + p.eps);
     const int np = qkv_pairs_in(p, r.x, r.y);
-    const bool skip = fault_here(ST_QKV);
     const int kvs = p.hd + kKvPad;                    // padded cache row
     __half* kbase = p.kv + (size_t)layer * 2 * p.KV * p.max_seq * kvs;
     __half* vbase = kbase + (size_t)p.KV * p.max_seq * kvs;
@@ -1209,7 +1230,7 @@ struct Consumer {
   // o = sum_s w_s (o_s / l_s) for its dims.  Returns false (uniformly) on
   // abort.
   template <int HD>
-  __device__ __noinline__ bool attn_combine(const AttnItem& it, unsigned tag) {
+  __device__ __noinline__ bool attn_combine(const AttnItem it, unsigned tag, bool skip) {
     const MonoParams& p = kie_p;
     const int tid = (int)threadIdx.x;
     constexpr int ROW = 2 + HD / 2;          // tagged words per (item, head) row
@@ -1263,7 +1284,6 @@ struct Consumer {
       }
     }
     if (dev::consumer_sync_or(bad)) return false;
-    const bool skip = fault_here(1);
     const int wd = d1 - d0;
     for (int e = tid; e < G * wd; e += kConsumerThreads) {
       const int g = e / wd, dd = e - g * wd;
@@ -1299,10 +1319,10 @@ struct Consumer {
   //   P.V:    O[head][dims] += P V, B fragments by transposed ldmatrix from
   //           the V tile; warp w owns HD/8 dims.
   template <int HD>
-  __device__ __noinline__ bool stage_attn(int pos, unsigned tag) {
+  __device__ __noinline__ bool stage_attn(int pos, unsigned tag, bool skip_combine) {
     const MonoParams& p = kie_p;
     const int tid = (int)threadIdx.x, warp = (int)(threadIdx.x >> 5), lane = (int)(threadIdx.x & 31);
-    stage = 5;
+    at_stage(5);
     const AttnItem it = attn_item(p, pos);
     if (!it.valid) return true;
     constexpr int QS = HD + 8;                  // halfs per Q tile row
@@ -1363,6 +1383,9 @@ struct Consumer {
     if (dev::consumer_sync_or(bad)) return false;
     if (tid == 0) kie_ctr[0] += clock64() - c0;
     trace(10);
+    // ring cursors (read after the barrier above; written back after the last
+    // barrier below)
+    uint32_t ci = kie_cur[0], cr = kie_cur[1], ce = kie_cur[2];
 
     const int gid = lane >> 2, tig = lane & 3;
     // A fragments of q come from the hi / lo tiles (rows gid are heads,
@@ -1383,8 +1406,8 @@ struct Consumer {
       const int nbp = (nb + 15) & ~15;
       const uint32_t sz = (uint32_t)(nbp * RS);
       uint32_t offk = 0, offv = 0;
-      bool badc = !wait_chunk(sz, offk);
-      badc = !wait_chunk(sz, offv) || badc;
+      bool badc = !wait_chunk(sz, offk, ci, ce);
+      badc = !wait_chunk(sz, offv, ci, ce) || badc;
       if (b0 == it.t0) trace(14);
       __half* Kt = reinterpret_cast<__half*>(sm_ring_w(p) + offk);
       __half* Vt = reinterpret_cast<__half*>(sm_ring_w(p) + offv);
@@ -1473,8 +1496,8 @@ struct Consumer {
         }
       }
       dev::consumer_sync();
-      release_chunk();
-      release_chunk();
+      release_chunk(cr);
+      release_chunk(cr);
     }
     // running output of heads gid < G to shared memory
     if (gid < G && pv_warp) {
@@ -1486,6 +1509,11 @@ struct Consumer {
       }
     }
     dev::consumer_sync();
+    if (tid == 0) {
+      kie_cur[0] = ci;
+      kie_cur[1] = cr;
+      kie_cur[2] = ce;
+    }
     trace(11);
     // publish this item's partial as tagged words: per head [m, l, then
     // o / l as fp16 pairs]
@@ -1504,21 +1532,20 @@ struct Consumer {
       dev::st_relaxed_u64(part + tid * ROW + 1, dev::tag_word(tag, a.lrun[tid]));
     }
     trace(12);
-    return attn_combine<HD>(it, tag);
+    return attn_combine<HD>(it, tag, skip_combine);
   }
 
   // O projection + residual -> x_ffn.
-  __device__ bool stage_o(const LayerW& w, int tok, unsigned tag) {
+  __device__ bool stage_o(const LayerW& w, int layer, int tok, unsigned tag, bool skip) {
     const MonoParams& p = kie_p;
     const int tid = (int)threadIdx.x;
-    stage = ST_O;
+    at_stage(ST_O);
     const int2 r = p.ranges[ST_O * p.grid + blockIdx.x];
     if (r.y <= r.x) return true;
     float ss;
     if (!load_vec(p.obuf, tag, nullptr, p.H * p.hd, nullptr, ss, 30)) return false;
     if (!gemv(ST_O)) return false;
     const StagePlan pl = sm_plan(p)[ST_O];
-    const bool skip = fault_here(ST_O);
     for (int u = r.x + tid; u < r.y; u += kConsumerThreads) {
       const int k = u - r.x;
       const float res = layer == 0 ? __half2float(p.tok_emb[(size_t)tok * p.d + u]) : sm_res_attn(p)[k];
@@ -1530,10 +1557,10 @@ struct Consumer {
   }
 
   // RMSNorm + gate/up GEMV + SwiGLU -> h.
-  __device__ bool stage_gu(const LayerW& w, unsigned tag) {
+  __device__ bool stage_gu(const LayerW& w, unsigned tag, bool skip) {
     const MonoParams& p = kie_p;
     const int tid = (int)threadIdx.x;
-    stage = ST_GU;
+    at_stage(ST_GU);
     const int2 r = p.ranges[ST_GU * p.grid + blockIdx.x];
     if (r.y <= r.x) return true;
     float ss;
@@ -1541,7 +1568,6 @@ struct Consumer {
     if (!gemv(ST_GU)) return false;
     const StagePlan pl = sm_plan(p)[ST_GU];
     const float rs = 1.0f / sqrtf(ss / (float)p.d + p.eps);
-    const bool skip = fault_here(ST_GU);
     for (int u = r.x + tid; u < r.y; u += kConsumerThreads) {
       const int k = u - r.x;
       const float g = row_result(pl, 2 * k) * rs, up = row_result(pl, 2 * k + 1) * rs;
@@ -1552,17 +1578,16 @@ struct Consumer {
   }
 
   // Down GEMV + residual -> x_attn (input of the next layer).
-  __device__ bool stage_down(const LayerW& w, unsigned tag, unsigned tag_next) {
+  __device__ bool stage_down(const LayerW& w, unsigned tag, unsigned tag_next, bool skip) {
     const MonoParams& p = kie_p;
     const int tid = (int)threadIdx.x;
-    stage = ST_DOWN;
+    at_stage(ST_DOWN);
     const int2 r = p.ranges[ST_DOWN * p.grid + blockIdx.x];
     if (r.y <= r.x) return true;
     float ss;
     if (!load_vec(p.hbuf, tag, nullptr, p.F, nullptr, ss, 50)) return false;
     if (!gemv(ST_DOWN)) return false;
     const StagePlan pl = sm_plan(p)[ST_DOWN];
-    const bool skip = fault_here(ST_DOWN);
     for (int u = r.x + tid; u < r.y; u += kConsumerThreads) {
       const int k = u - r.x;
       const float v = sm_res_ffn(p)[k] + row_result(pl, k);
@@ -1608,20 +1633,20 @@ struct Consumer {
   }
 
   // Final RMSNorm + LM head + token pick (argmax of pick_score); or, on
-  // steps that pick no id, only the per-step fenced publish.  Returns false
-  // on abort; *tok_out gets the picked id (uniform across the grid).
-  __device__ __noinline__ bool stage_lm(bool pick, int step_row, unsigned tag, int pos,
-                                        int* tok_out) {
+  // steps that pick no id, only the per-step fenced publish.  Returns the
+  // picked id (uniform across the grid), or -1 on abort.
+  __device__ __noinline__ int stage_lm(bool pick, int step, int step_row, unsigned tag, int pos,
+                                       bool skip) {
     const MonoParams& p = kie_p;
     const int tid = (int)threadIdx.x, warp = (int)(threadIdx.x >> 5), lane = (int)(threadIdx.x & 31);
-    stage = ST_LM;
+    at_stage(ST_LM);
     float best = -INFINITY;
     int bi = INT_MAX;
     const int2 r = p.ranges[ST_LM * p.grid + blockIdx.x];
     if (pick && r.y > r.x) {
       float ss;
-      if (!load_vec(p.x_attn, tag, nullptr, p.d, p.final_norm, ss, 60)) return false;
-      if (!gemv(ST_LM)) return false;
+      if (!load_vec(p.x_attn, tag, nullptr, p.d, p.final_norm, ss, 60)) return -1;
+      if (!gemv(ST_LM)) return -1;
       const StagePlan pl = sm_plan(p)[ST_LM];
       trace(2);
       const float rs = 1.0f / sqrtf(ss / (float)p.d + p.eps);
@@ -1644,7 +1669,6 @@ struct Consumer {
       sm_redi(p)[warp] = bi;
     }
     dev::consumer_sync();
-    const bool skip = fault_here(ST_LM);
     if (tid == 0) {
       float b = sm_red(p)[0];
       int ib = sm_redi(p)[0];
@@ -1687,7 +1711,7 @@ struct Consumer {
       sm_red2(p)[warp] = gb;
       sm_redi2(p)[warp] = gi;
     }
-    if (dev::consumer_sync_or(bad)) return false;
+    if (dev::consumer_sync_or(bad)) return -1;
     float b = sm_red2(p)[0];
     int ib = sm_redi2(p)[0];
     for (int w = 1; w < kConsumerWarps; ++w)
@@ -1695,14 +1719,13 @@ struct Consumer {
         b = sm_red2(p)[w];
         ib = sm_redi2(p)[w];
       }
-    *tok_out = ib;
     if (tid == 0) {
       kie_ctr[0] += clock64() - c0;
       // this step's KV writes of every CTA are now visible to this CTA:
       // the producer may copy them for the next step
       dev::st_release_cta(sm_flags(p) + F_KVSTEP, step + 1);
     }
-    return true;
+    return ib;
   }
 
   // Walks a stage's chunk sequence without computing (stream-only timing).
@@ -1711,13 +1734,20 @@ struct Consumer {
     const int R = range_rows(p, st, ub, ue);
     const int kp = stage_k(p, st) / kPieceElems;
     bool bad = false;
+    uint32_t ci = kie_cur[0], cr = kie_cur[1], ce = kie_cur[2];
     for_each_chunk(R, kp, p.chunk_bytes, [&](int, int rg, int n, int) {
       uint32_t off;
-      if (!wait_chunk((uint32_t)(rg * n * kPieceBytes), off)) bad = true;
-      release_chunk();
+      if (!wait_chunk((uint32_t)(rg * n * kPieceBytes), off, ci, ce)) bad = true;
+      release_chunk(cr);
       return true;
     });
-    return !dev::consumer_sync_or(bad);
+    const bool any_bad = dev::consumer_sync_or(bad);
+    if (threadIdx.x == 0) {
+      kie_cur[0] = ci;
+      kie_cur[1] = cr;
+      kie_cur[2] = ce;
+    }
+    return !any_bad;
   }
 
   // Standalone GEMV engine run: y = W x over the LM-head stage's rows,
@@ -1735,8 +1765,10 @@ struct Consumer {
     }
     dev::consumer_sync();
     bool ok = true;
-    for (int it = 0; it < iters && ok; ++it)
+    for (int it = 0; it < iters && ok; ++it) {
+      dev::consumer_sync();   // the ring cursors thread 0 wrote back are visible
       ok = mode == 0 ? skip_stage(ST_LM, r.x, r.y) : gemv(ST_LM);
+    }
     if (ok && mode == 1)
       for (int u = r.x + tid; u < r.y; u += kConsumerThreads) y[u] = row_result(sm_plan(p)[ST_LM], u - r.x);
     if (tid == 0) {
@@ -1757,38 +1789,39 @@ struct Consumer {
     int done = 0;
     bool ok = true;
     for (int i = 0; i < p.n_steps && ok; ++i) {
-      step = i;
+      if (tid == 0) kie_at[0] = i;
       const int pos = p.pos0 + i;
       for (int l = 0; l < p.L && ok; ++l) {
-        layer = l;
+        if (tid == 0) kie_at[1] = l;
         const LayerW& w = p.layers[l];
         const unsigned tag = epoch_of(p, i, l);
+        const int fst = fault_stage_at(i, l);
         trace(0);
-        ok = stage_qkv(w, tok, pos, tag);
+        ok = stage_qkv(w, l, tok, pos, tag, fst == ST_QKV);
         trace(2);
         trace_stream_wait(ST_QKV);
-        ok = ok && stage_attn<HD>(pos, tag);
+        ok = ok && stage_attn<HD>(pos, tag, fst == ST_O);
         trace(3);
         trace_stream_wait(5);
-        ok = ok && stage_o(w, tok, tag);
+        ok = ok && stage_o(w, l, tok, tag, fst == ST_O);
         trace(5);
         trace_stream_wait(ST_O);
-        ok = ok && stage_gu(w, tag);
+        ok = ok && stage_gu(w, tag, fst == ST_GU);
         trace(7);
         trace_stream_wait(ST_GU);
-        ok = ok && stage_down(w, tag, tag + 1u);
+        ok = ok && stage_down(w, tag, tag + 1u, fst == ST_DOWN);
         trace(9);
         trace_stream_wait(ST_DOWN);
       }
       if (!ok) break;
-      layer = p.L;
+      if (tid == 0) kie_at[1] = p.L;
       const bool pick = i >= p.lm_from;
-      int next = 0;
       trace(0);
-      const bool lm_ok = stage_lm(pick, i - p.lm_from, epoch_of(p, i, p.L), pos, &next);
+      const int next = stage_lm(pick, i, i - p.lm_from, epoch_of(p, i, p.L), pos,
+                                fault_stage_at(i, p.L) == ST_LM);
       trace(3);
       if (tid == 0) kie_ctr[2] = 0;
-      if (!lm_ok) {
+      if (next < 0) {
         ok = false;
         break;
       }
@@ -1826,6 +1859,8 @@ __device__ __forceinline__ void kernel_setup(const MonoParams& p) {
     sm_flags(p)[F_STOP] = 0;
     sm_flags(p)[F_KVSTEP] = 0;
     kie_ctr[0] = kie_ctr[1] = kie_ctr[2] = 0;
+    kie_cur[0] = kie_cur[1] = kie_cur[2] = 0u;
+    kie_at[0] = kie_at[1] = kie_at[2] = 0;
     dev::mbar_fence_init();
   }
   __syncthreads();
