@@ -459,17 +459,35 @@ struct Producer {
     }
   }
 
+  // The stage's chunks in stream order (for_each_chunk's order; only their
+  // sizes matter here): full-group pairs (the two groups' chunks alternate
+  // per k-chunk), a leftover full group, the partial group.  One loop nest
+  // with a single issue site keeps the producer's code small: it shares the
+  // SM's instruction cache with the consumer warps.
   __device__ bool stage(int st, const unsigned char*& src) {
     const int2 r = p.ranges[st * p.grid + blockIdx.x];
     const int R = range_rows(p, st, r.x, r.y);
     const int kp = stage_k(p, st) / kPieceElems;
-    return for_each_chunk(R, kp, p.chunk_bytes, [&](int, int rg, int n, int) {
-      const uint32_t sz = (uint32_t)(rg * n * kPieceBytes);
-      if (p.l2_prefetch > 0) prefetch(sz);
-      if (!chunk(src, sz)) return false;
-      pf_ahead -= sz;
-      return true;
-    });
+    const int nfull = R / kGroupRows, tail = R - nfull * kGroupRows;
+    const Chunking cf = chunking(kGroupRows, kp, p.chunk_bytes);
+    const Chunking ct = chunking(tail > 0 ? tail : 1, kp, p.chunk_bytes);
+#pragma unroll 1
+    for (int sg = 0; sg < 3; ++sg) {
+      const int reps = sg == 0 ? nfull / 2 : (sg == 1 ? (nfull & 1) : (tail > 0 ? 1 : 0));
+      const int rows = sg < 2 ? kGroupRows : tail;
+      const int mult = sg == 0 ? 2 : 1;
+      const Chunking c = sg < 2 ? cf : ct;
+#pragma unroll 1
+      for (int rep = 0; rep < reps; ++rep)
+#pragma unroll 1
+        for (int j = 0; j < c.nk * mult; ++j) {
+          const uint32_t sz = (uint32_t)(rows * c.count(j / mult) * kPieceBytes);
+          if (p.l2_prefetch > 0) prefetch(sz);
+          if (!chunk(src, sz)) return false;
+          pf_ahead -= sz;
+        }
+    }
+    return true;
   }
 
   // K and V blocks of this CTA's attention item at step i, layer l, for the
@@ -559,16 +577,28 @@ struct Producer {
     len_lm = stage_len(ST_LM);
     for (int i = 0; i < p.n_steps && ok; ++i) {
       const unsigned char* src = base;
-      for (int l = 0; l < p.L && ok; ++l) {
-        prefetch_kv(i, l);
-        trace(i, l, 22);
-        ok = stage(ST_QKV, src);
-        trace(i, l, 23);
-        ok = ok && attn(i, l);
-        trace(i, l, 20);
-        ok = ok && stage(ST_O, src) && stage(ST_GU, src) && stage(ST_DOWN, src);
+      // layers, then the LM head as a last pseudo-layer on steps that pick
+      // an id; per layer QKV, the attention tiles, O, gate/up, down.  One
+      // call site per kind of work (see stage).
+      const int nl = p.L + (i >= p.lm_from ? 1 : 0);
+#pragma unroll 1
+      for (int l = 0; l < nl && ok; ++l) {
+        const bool lm = l == p.L;
+        if (!lm) {
+          prefetch_kv(i, l);
+          trace(i, l, 22);
+        }
+#pragma unroll 1
+        for (int k = lm ? 4 : 0; k < 5 && ok; ++k) {
+          if (k == 1) {
+            trace(i, l, 23);
+            ok = attn(i, l);
+            trace(i, l, 20);
+          } else {
+            ok = stage(lm ? ST_LM : (k == 0 ? ST_QKV : k - 1), src);
+          }
+        }
       }
-      if (ok && i >= p.lm_from) ok = stage(ST_LM, src);
     }
     drain();
     p.cta_stats[kStatsPerCta * blockIdx.x + 3] = (unsigned long long)t_wait;
