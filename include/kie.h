@@ -145,7 +145,7 @@ typedef struct {
 typedef enum {
   KIE_OPT_TIMEOUT_NS = 1,     /* bound of every device-side wait (default 2e9) */
   KIE_OPT_CHUNK_BYTES = 2,    /* largest weight chunk in bytes (>= 8192, multiple of 512;
-                                 default 65536, or 32768 where two 64 KB chunks do not
+                                 default 32768, or 16384 where two 32 KB chunks do not
                                  fit the ring); re-plans the ring and rebuilds the packed
                                  weight copy, so the caller's matrices must still be valid */
   KIE_OPT_MIN_SPLIT_LEN = 3,  /* minimum positions per attention split (default 64) */

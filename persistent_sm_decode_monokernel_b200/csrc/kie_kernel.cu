@@ -673,7 +673,7 @@ struct Consumer {
   // Stage trace (measurement, tid 0 only): per step kTracePerLayer slots
   // per layer (stage boundaries, attention sub-steps, stream waits; the
   // layout is documented with kie_set_trace) + 4 for the LM head.
-  __device__ __forceinline__ void trace_put(int ev, unsigned long long v) const {
+  __device__ __noinline__ void trace_put(int ev, unsigned long long v) const {
     const MonoParams& p = kie_p;
     const int tid = (int)threadIdx.x;
     if (p.trace && tid == 0 && (p.trace_cta < 0 || (int)blockIdx.x == p.trace_cta) &&
@@ -762,29 +762,7 @@ struct Consumer {
     const uint32_t par = (cidx / kRingBars) & 1u;
     ++cidx;
     if (dev::mbar_test_wait(bar, par)) return true;
-    const long long c0 = clock64();
-    const long long t0 = dev::globaltimer();
-    bool ok = true;
-    for (unsigned it = 1;; ++it) {
-      if (dev::mbar_try_wait(bar, par)) break;
-      if ((it & 15u) == 0u) {
-        if (sm_flags(p)[F_ABORT]) {
-          ok = false;
-          break;
-        }
-        if (dev::globaltimer() - t0 > p.timeout_ns) {
-          raise_error(p, DEV_TIMEOUT, kie_at[0], kie_at[1], kie_at[2], 3);
-          sm_flags(p)[F_ABORT] = 1;
-          ok = false;
-          break;
-        }
-      }
-    }
-    if (tid == 0) {
-      kie_ctr[1] += clock64() - c0;
-      if (p.trace) kie_ctr[2] += dev::globaltimer() - t0;
-    }
-    return ok;
+    return wait_slow(bar, par);
   }
   // Releases the oldest chunk this warp waited for and has not released
   // (crel: the caller's copy of the release cursor).

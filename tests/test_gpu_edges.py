@@ -82,7 +82,7 @@ def test_long_context_one_split_many_blocks(torch_cuda):
     assert rep.compared == 9
 
 
-@pytest.mark.parametrize("chunk", [8192, 12800, 32768, 98304])
+@pytest.mark.parametrize("chunk", [8192, 12800, 65536, 98304])
 def test_chunk_sizes(torch_cuda, chunk):
     from persistent_sm_decode_monokernel_b200 import _kie
     rep = _forced_parity(synth.WORKLOADS["l16-d1024"].shape, 40, 12,
