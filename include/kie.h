@@ -258,6 +258,25 @@ KIE_API kie_status kie_set_trace(kie_ctx *ctx, uint64_t *dev_buf, int32_t capaci
  * temperature that is negative, infinite or NaN.  Host only. */
 KIE_API kie_status kie_set_sampling(kie_ctx *ctx, float temperature, uint64_t seed);
 
+/* Restriction of the sampled draw (kie_set_sampling with temperature > 0;
+ * greedy picks ignore it).  The pages name LM-head sampling without a
+ * sampler (revietech.ru, "Kog выжимает максимум из GPU: 3000 токенов/с",
+ * section "Что такое monokernel"); top-k and nucleus (top-p) filtering are
+ * the readings taken.  top_k in 1 .. KIE_MAX_TOP_K keeps the top_k largest
+ * logits of the step (ties by the lower id); top_p in (0, 1) then keeps, of
+ * those, the shortest prefix ordered by probability under
+ * softmax(logits / temperature) restricted to them whose mass reaches top_p
+ * (computed in fp64 from the fp32 logits).  The draw is the Gumbel-max draw
+ * of kie_set_sampling over the kept ids, with the same noise.  top_k = 0
+ * and top_p = 1 switch the restriction off (the default).  Returns
+ * KIE_ERR_INVALID_ARG for a NULL ctx, top_k outside 0 .. KIE_MAX_TOP_K or
+ * top_p outside (0, 1], and KIE_ERR_UNSUPPORTED for top_p < 1 with
+ * top_k = 0 (the kernel bounds the nucleus by a top-k set).  Each picking
+ * step then exchanges every CTA's top_k candidates once more between the
+ * CTAs.  Host only. */
+#define KIE_MAX_TOP_K 64
+KIE_API kie_status kie_set_sampling_filter(kie_ctx *ctx, int32_t top_k, float top_p);
+
 /* Ids that end a decode: a step whose picked id is one of ids[0 .. n) is
  * the last one (it is written and counted in *n_out).  n = 0 goes back to
  * the model descriptor's eos_id (none if -1).  ids: HOST array, copied.

@@ -15,7 +15,8 @@ from . import _kie
 from ._kie import (KieError, kie_check_desc, kie_create, kie_decode, kie_decode_forced,  # noqa: F401
                    kie_destroy, kie_get_stats, kie_kv_cache_bytes, kie_last_error,
                    kie_plan_units, kie_prefill, kie_rewind, kie_set_eos_ids,
-                   kie_set_logits_capture, kie_set_option, kie_set_sampling, kie_set_trace,
+                   kie_set_logits_capture, kie_set_option, kie_set_sampling,
+                   kie_set_sampling_filter, kie_set_trace,
                    load_library, make_desc)
 
 TRACE_PER_LAYER = 24   # trace slots per layer (kie.h, kie_set_trace)
@@ -124,9 +125,13 @@ class Session:
                              "session has released (keep_matrices=False)")
         kie_set_option(self.ctx, opt, value)
 
-    def set_sampling(self, temperature: float, seed: int = 0) -> None:
-        """temperature 0 = greedy (default); > 0 samples in the kernel."""
+    def set_sampling(self, temperature: float, seed: int = 0, top_k: int = 0,
+                     top_p: float = 1.0) -> None:
+        """temperature 0 = greedy (default); > 0 samples in the kernel, from
+        the top_k largest logits (0 = all) and of those the top_p nucleus
+        (1 = all; top_p < 1 needs top_k >= 1)."""
         kie_set_sampling(self.ctx, temperature, seed)
+        kie_set_sampling_filter(self.ctx, top_k, top_p)
 
     def set_eos_ids(self, ids: Sequence[int]) -> None:
         """Ids that end a decode ([] = the descriptor's eos_id)."""

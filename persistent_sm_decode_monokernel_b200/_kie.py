@@ -30,6 +30,7 @@ KIE_ERR_HOST_MEMORY = 9
 
 KIE_NOALLOC_MAX_WEIGHT_BYTES = 16 * 1024 * 1024
 KIE_MAX_EOS_IDS = 8
+KIE_MAX_TOP_K = 64
 
 KIE_OPT_TIMEOUT_NS = 1
 KIE_OPT_CHUNK_BYTES = 2
@@ -103,6 +104,7 @@ SIGNATURES = {
                                     ctypes.POINTER(ctypes.c_float),
                                     ctypes.POINTER(ctypes.c_double)]),
     "kie_gemv_f16_noalloc": (ctypes.c_int, [_P, _P, _P, _I32, _I32, _P]),
+    "kie_set_sampling_filter": (ctypes.c_int, [_P, _I32, ctypes.c_float]),
 }
 
 _lib: Optional[ctypes.CDLL] = None
@@ -245,6 +247,13 @@ def kie_set_sampling(ctx, temperature: float, seed: int = 0) -> None:
     """temperature 0 = greedy; > 0 = in-kernel temperature sampling."""
     _check(load_library().kie_set_sampling(ctx, float(temperature), int(seed) & ((1 << 64) - 1)),
            "kie_set_sampling", ctx)
+
+
+def kie_set_sampling_filter(ctx, top_k: int = 0, top_p: float = 1.0) -> None:
+    """Restricts sampled draws to the top_k largest logits, then to the
+    top_p nucleus of those (0 and 1: off)."""
+    _check(load_library().kie_set_sampling_filter(ctx, int(top_k), float(top_p)),
+           "kie_set_sampling_filter", ctx)
 
 
 def kie_set_eos_ids(ctx, ids: Sequence[int]) -> None:

@@ -38,7 +38,7 @@ struct kie_ctx {
   unsigned long long* tagged = nullptr;
   size_t tagged_words = 0;
   unsigned long long *x_attn = nullptr, *x_ffn = nullptr, *hbuf = nullptr, *qbuf = nullptr,
-                     *kvnew = nullptr, *obuf = nullptr, *slots = nullptr;
+                     *kvnew = nullptr, *obuf = nullptr, *slots = nullptr, *cands = nullptr;
   unsigned long long* partials = nullptr;
   int* d_ids = nullptr;               // fed ids of a launch [max_seq]
   unsigned char* d_io = nullptr;      // DevStatus + out ids [max_seq]
@@ -73,6 +73,8 @@ struct kie_ctx {
   // the model descriptor's eos_id, if any)
   double temperature = 0.0;
   unsigned long long seed = 0;
+  int top_k = 0;          // 0: no top-k restriction of the draw
+  double top_p = 1.0;     // 1: no top-p restriction
   std::vector<int32_t> eos_ids;
   unsigned long long* trace = nullptr;
   int trace_cta = 0, trace_steps = 0, trace_clock = 0;
@@ -170,6 +172,9 @@ kie_status launch(kie_ctx* c, int n_steps, int pos0, const int32_t* host_ids, bo
   p.sample = c->temperature > 0.0 ? 1 : 0;
   p.inv_temp = c->temperature > 0.0 ? 1.0 / c->temperature : 0.0;
   p.seed = c->seed;
+  p.top_k = c->top_k;
+  p.top_p = c->top_p;
+  p.cands = c->cands;
   p.layers = c->dlayers;
   p.tok_emb = c->tok_emb;
   p.final_norm = c->final_norm;
@@ -401,7 +406,9 @@ kie_status kie_create(const kie_model_desc* d, const kie_weights* w, void* kv_ca
 
     const int G = d->n_heads / d->n_kv_heads;
     const size_t qd = (size_t)d->n_heads * d->head_dim, kvd = (size_t)d->n_kv_heads * d->head_dim;
-    c->tagged_words = 2 * (size_t)d->d_model + d->ffn_dim + qd + 2 * kvd + qd + 2 * (size_t)grid;
+    // activation vectors, argmax slots, top-k candidate lists
+    c->tagged_words = 2 * (size_t)d->d_model + d->ffn_dim + qd + 2 * kvd + qd + 2 * (size_t)grid +
+                      2 * (size_t)kie::kMaxTopK * grid;
     std::vector<int2> flat;
     for (auto& v : c->hranges) flat.insert(flat.end(), v.begin(), v.end());
     const size_t half = d->head_dim / 2;
@@ -431,7 +438,8 @@ kie_status kie_create(const kie_model_desc* d, const kie_weights* w, void* kv_ca
     c->qbuf = t;    t += qd;
     c->kvnew = t;   t += 2 * kvd;
     c->obuf = t;    t += qd;
-    c->slots = t;
+    c->slots = t;   t += 2 * (size_t)grid;
+    c->cands = t;
     if (cuda_bad(cudaMemcpyAsync(c->dlayers, c->hlayers.data(), sizeof(LayerW) * d->n_layers,
                                  cudaMemcpyHostToDevice, c->stream)) ||
         cuda_bad(cudaMemcpyAsync(c->rope, rope.data(), sizeof(float2) * rope.size(),
@@ -559,6 +567,22 @@ kie_status kie_set_sampling(kie_ctx* c, float temperature, uint64_t seed) {
   // compares in, and the draw is the greedy pick anyway (T -> 0 limit).
   c->temperature = temperature < 1e-20f ? 0.0 : (double)temperature;
   c->seed = seed;
+  return KIE_OK;
+}
+
+static_assert(KIE_MAX_TOP_K == kie::kMaxTopK, "top-k bound");
+
+kie_status kie_set_sampling_filter(kie_ctx* c, int32_t top_k, float top_p) {
+  if (!c) return KIE_ERR_INVALID_ARG;
+  if (top_k < 0 || top_k > KIE_MAX_TOP_K)
+    return set_err(c, KIE_ERR_INVALID_ARG, "top_k must be in 0 .. KIE_MAX_TOP_K");
+  if (!(top_p > 0.f && top_p <= 1.f))
+    return set_err(c, KIE_ERR_INVALID_ARG, "top_p must be in (0, 1]");
+  if (top_p < 1.f && top_k == 0)
+    return set_err(c, KIE_ERR_UNSUPPORTED,
+                   "top_p < 1 needs a top_k bound (1 .. KIE_MAX_TOP_K) in the kernel");
+  c->top_k = top_k;
+  c->top_p = (double)top_p;
   return KIE_OK;
 }
 

@@ -756,7 +756,6 @@ struct Consumer {
   __device__ __forceinline__ bool wait_chunk(uint32_t sz, uint32_t& off, uint32_t& cidx,
                                              uint32_t& cend) {
     const MonoParams& p = kie_p;
-    const int tid = (int)threadIdx.x;
     off = ring_place(cend, sz, (uint32_t)p.ring_bytes);
     const uint32_t bar = sm_full_s(p) + 8 * (cidx & (kRingBars - 1));
     const uint32_t par = (cidx / kRingBars) & 1u;
@@ -1640,6 +1639,174 @@ struct Consumer {
     return false;
   }
 
+  // ---- top-k / top-p restriction of the draw
+  // Sort key of vocabulary entry u with logit v: unsigned order is the
+  // order "larger logit first, then the lower index" (the fp32 bits made
+  // monotone in the high half, the complemented index in the low half).
+  // Keys are unique and never 0, so 0 marks "no entry".
+  __device__ __forceinline__ static u64 vocab_key(float v, int u) {
+    const unsigned b = __float_as_uint(v);
+    const unsigned ord = (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+    return (static_cast<u64>(ord) << 32) | (0xFFFFFFFFu - (unsigned)u);
+  }
+  __device__ __forceinline__ static float key_value(u64 k) {
+    const unsigned ord = (unsigned)(k >> 32);
+    return __uint_as_float((ord & 0x80000000u) ? (ord & 0x7FFFFFFFu) : ~ord);
+  }
+  __device__ __forceinline__ static u64 shfl_xor_u64(u64 v, int o) {
+    const unsigned lo = __shfl_xor_sync(0xffffffffu, (unsigned)v, o);
+    const unsigned hi = __shfl_xor_sync(0xffffffffu, (unsigned)(v >> 32), o);
+    return (static_cast<u64>(hi) << 32) | lo;
+  }
+
+  // The smallest key of the kept set: the top_k largest logits of the
+  // whole vocabulary (ties by the lower index), then of those the shortest
+  // prefix, largest probability first, whose mass under softmax(logits / T)
+  // restricted to them reaches top_p.  Every CTA ranks its own rows and
+  // publishes its sorted top_k keys as tagged words; every CTA then copies
+  // the first kFilterHeads keys of all the CTAs' lists and pops the global
+  // top_k with one warp (a lane holds the heads of grid / 32 lists; a list
+  // popped past its copied keys is read on from global memory), so every
+  // CTA finds the same threshold and no further exchange is needed.
+  // Called by all consumer threads; returns ~0 on abort.
+  __device__ __noinline__ u64 filter_threshold(int2 r, float rs, unsigned tag) {
+    const MonoParams& p = kie_p;
+    const StagePlan pl = sm_plan(p)[ST_LM];
+    const int tid = (int)threadIdx.x, warp = (int)(threadIdx.x >> 5), lane = (int)(threadIdx.x & 31);
+    constexpr u64 kAbort = ~0ull;
+    const int n = r.y - r.x, kf = p.top_k, m = min(kf, kFilterHeads);
+    u64* K = reinterpret_cast<u64*>(kie_smem + p.sm.xs_off);   // this CTA's keys [n]
+    u64* Ls = K + n;                                            // its top kf, sorted
+    u64* S = Ls + kMaxTopK;                                     // [grid][kFilterHeads]
+    u64* P = S + p.grid * kFilterHeads;                         // global top kf, popped
+    u64* tau_s = P + kMaxTopK;
+    for (int i = tid; i < n; i += kConsumerThreads)
+      K[i] = vocab_key(row_result(pl, i) * rs, r.x + i);
+    for (int i = tid; i < kf; i += kConsumerThreads) Ls[i] = 0ull;
+    dev::consumer_sync();
+    for (int i = tid; i < n; i += kConsumerThreads) {
+      const u64 k = K[i];
+      int rank = 0;
+      for (int j = 0; j < n; ++j) rank += K[j] > k ? 1 : 0;
+      if (rank < kf) Ls[rank] = k;
+    }
+    dev::consumer_sync();
+    // publish: pair (2i, 2i+1) = high and low half of key i, tagged
+    u64* mine = p.cands + (size_t)blockIdx.x * kMaxTopK * 2;
+    for (int i = tid; i < kf; i += kConsumerThreads) {
+      dev::st_relaxed_u64(mine + 2 * i, (static_cast<u64>(tag) << 32) | (unsigned)(Ls[i] >> 32));
+      dev::st_relaxed_u64(mine + 2 * i + 1, (static_cast<u64>(tag) << 32) | (unsigned)Ls[i]);
+    }
+    // gather the first m keys of every list
+    constexpr int NB = 4;
+    const int ntot = p.grid * m, n2 = p.grid * kMaxTopK;
+    bool bad = false;
+    for (int base = tid; base < ntot && !bad; base += kConsumerThreads * NB) {
+      int k2[NB];
+      ulonglong2 v[NB];
+#pragma unroll
+      for (int b = 0; b < NB; ++b) {
+        const int q = base + b * kConsumerThreads;
+        const int c = q / m, j = q - (q / m) * m;
+        k2[b] = q < ntot ? c * kMaxTopK + j : n2;
+      }
+      if (!poll_pairs<NB>(p.cands, k2, n2, tag, v, 62)) {
+        bad = true;
+        break;
+      }
+#pragma unroll
+      for (int b = 0; b < NB; ++b) {
+        const int q = base + b * kConsumerThreads;
+        if (q < ntot) {
+          const int c = q / m, j = q - (q / m) * m;
+          S[c * kFilterHeads + j] = (v[b].x << 32) | (v[b].y & 0xFFFFFFFFull);
+        }
+      }
+    }
+    if (dev::consumer_sync_or(bad)) return kAbort;
+    if (warp == 0) {
+      constexpr int Q = (160 + 31) / 32;   // lists per lane (grid <= 160)
+      int ptr[Q];
+      u64 h[Q];
+#pragma unroll
+      for (int q = 0; q < Q; ++q) {
+        const int c = lane + 32 * q;
+        ptr[q] = 0;
+        h[q] = c < p.grid ? S[c * kFilterHeads] : 0ull;
+      }
+      // (every lane runs every round: the shuffles need the whole warp)
+      for (int t = 0; t < kf; ++t) {
+        u64 best = 0ull;
+        int bq = 0;
+#pragma unroll
+        for (int q = 0; q < Q; ++q)
+          if (h[q] > best) {
+            best = h[q];
+            bq = q;
+          }
+        u64 wb = best;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+          const u64 x = shfl_xor_u64(wb, o);
+          wb = x > wb ? x : wb;
+        }
+        if (lane == 0) P[t] = wb;
+        if (wb != 0ull && best == wb) {
+#pragma unroll
+          for (int q = 0; q < Q; ++q)
+            if (q == bq) {
+              const int c = lane + 32 * q;
+              ++ptr[q];
+              if (ptr[q] >= kf) {
+                h[q] = 0ull;
+              } else if (ptr[q] < m) {
+                h[q] = S[c * kFilterHeads + ptr[q]];
+              } else {   // past the copied keys: read the list on
+                const int k2[1] = {c * kMaxTopK + ptr[q]};
+                ulonglong2 v[1];
+                if (!poll_pairs<1>(p.cands, k2, n2, tag, v, 63)) bad = true;
+                h[q] = bad ? 0ull : (v[0].x << 32) | (v[0].y & 0xFFFFFFFFull);
+              }
+            }
+        }
+      }
+      bad = __any_sync(0xffffffffu, bad);
+      __syncwarp();
+      // the kept prefix: all kf (or fewer if the vocabulary is smaller), cut
+      // at the first entry where the probability mass reaches top_p
+      int nk = 0;
+      for (int i = lane; i < kf; i += 32) nk += P[i] != 0ull ? 1 : 0;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) nk += __shfl_xor_sync(0xffffffffu, nk, o);
+      int cut = nk;   // entries kept
+      if (p.top_p < 1.0 && nk > 0) {
+        const double z0 = (double)key_value(P[0]) * p.inv_temp;
+        const double e0 = lane < nk ? exp((double)key_value(P[lane]) * p.inv_temp - z0) : 0.0;
+        const double e1 = lane + 32 < nk ? exp((double)key_value(P[lane + 32]) * p.inv_temp - z0) : 0.0;
+        // inclusive prefix sums of both halves
+        double c0 = e0, c1 = e1;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const double a0 = __shfl_up_sync(0xffffffffu, c0, o);
+          const double a1 = __shfl_up_sync(0xffffffffu, c1, o);
+          if (lane >= o) {
+            c0 += a0;
+            c1 += a1;
+          }
+        }
+        const double half0 = __shfl_sync(0xffffffffu, c0, 31);
+        c1 += half0;
+        const double total = __shfl_sync(0xffffffffu, c1, 31);
+        const unsigned b0 = __ballot_sync(0xffffffffu, lane < nk && c0 / total >= p.top_p);
+        const unsigned b1 = __ballot_sync(0xffffffffu, lane + 32 < nk && c1 / total >= p.top_p);
+        cut = b0 ? __ffs(b0) : (b1 ? 32 + __ffs(b1) : nk);
+      }
+      if (lane == 0) *tau_s = cut > 0 ? P[cut - 1] : 0ull;
+    }
+    if (dev::consumer_sync_or(bad)) return kAbort;
+    return *tau_s;
+  }
+
   // Final RMSNorm + LM head + token pick (argmax of pick_score); or, on
   // steps that pick no id, only the per-step fenced publish.  Returns the
   // picked id (uniform across the grid), or -1 on abort.
@@ -1661,9 +1828,16 @@ struct Consumer {
       float* cap = (p.capture && step_row < p.capture_rows)
                        ? p.capture + (size_t)step_row * p.V
                        : nullptr;
+      // rows below the top-k / top-p threshold key take no part in the draw
+      u64 tau = 0ull;
+      if (p.sample && p.top_k > 0) {
+        tau = filter_threshold(r, rs, tag);
+        if (tau == ~0ull) return -1;
+      }
       for (int u = r.x + tid; u < r.y; u += kConsumerThreads) {
         const float v = row_result(pl, u - r.x) * rs;
         if (cap) cap[u] = v;
+        if (vocab_key(v, u) < tau) continue;
         const float sc = pick_score(v, u, pos);
         if (better(sc, u, best, bi)) {
           best = sc;

@@ -54,6 +54,16 @@ constexpr int kMiscHead = 128;
 constexpr int kEngineMisc = 896;
 // Most ids of the set that ends a decode (end-of-sequence ids).
 constexpr int kMaxEosIds = 8;
+// Top-k / top-p sampling: largest k, and how many entries of every CTA's
+// local top-k list each CTA copies to shared memory for the merge (deeper
+// entries are fetched from global memory when a merge reaches them).
+constexpr int kMaxTopK = 64;
+constexpr int kFilterHeads = 8;
+// Shared-memory bytes of the top-k / top-p selection for a CTA with `rows`
+// vocabulary rows in a grid of `grid` CTAs (it reuses the GEMV input area).
+constexpr int filter_smem_bytes(int rows, int grid) {
+  return 8 * (rows + 2 * kMaxTopK + grid * kFilterHeads + 2);
+}
 
 // Device status word block (library scratch, zeroed before each launch).
 struct DevStatus {
@@ -86,6 +96,12 @@ struct MonoParams {
   int sample;
   double inv_temp;
   unsigned long long seed;
+  // restriction of the draw (sample != 0): the top_k largest logits (0 =
+  // none), then of those the shortest prefix by probability whose mass
+  // reaches top_p (1 = none; top_p < 1 needs top_k >= 1)
+  int top_k;
+  double top_p;
+  unsigned long long* cands;  // [grid][kMaxTopK][2] tagged words: every CTA's local top-k keys
   // weights (device)
   const LayerW* layers;
   const __half* tok_emb;

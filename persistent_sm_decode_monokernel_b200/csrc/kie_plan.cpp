@@ -99,11 +99,15 @@ bool plan_smem(const Shape& s, int grid, int chunk_bytes, int smem_limit,
   const int G = s.H / s.KV;
   const int kmax = std::max(std::max(s.d, s.H * s.hd), s.F);
   SmemLayout L{};
-  L.xs_bytes = align_up(std::max(kmax * 2, attn_smem_bytes(G, s.hd)), 128);  // fp16 input vector
   int maxrows = 0;
   for (int st = 0; st < N_STAGES; ++st)
     for (int c = 0; c < grid; ++c)
       maxrows = std::max(maxrows, rows_in_range(s, st, ranges[st][c].x, ranges[st][c].y));
+  // fp16 input vector; the area also holds the attention scratch and the
+  // top-k / top-p selection of the LM-head pick
+  L.xs_bytes = align_up(std::max(std::max(kmax * 2, attn_smem_bytes(G, s.hd)),
+                                 filter_smem_bytes(maxrows, grid)),
+                        128);
   L.rowacc_rows = maxrows;
   int maxres = 0;
   for (int c = 0; c < grid; ++c)

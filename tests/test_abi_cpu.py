@@ -135,6 +135,7 @@ def test_status_strings(lib):
 
 def test_selection_setters_reject_null_context(lib):
     assert lib.kie_set_sampling(None, 1.0, 5) == _kie.KIE_ERR_INVALID_ARG
+    assert lib.kie_set_sampling_filter(None, 5, 0.9) == _kie.KIE_ERR_INVALID_ARG
     ids = (ctypes.c_int32 * 2)(1, 2)
     assert lib.kie_set_eos_ids(None, ids, 2) == _kie.KIE_ERR_INVALID_ARG
     assert _kie.KIE_MAX_EOS_IDS == int(re.search(
