@@ -33,6 +33,9 @@ Pinned by tests/test_oracle_fp8.py.
 """
 from __future__ import annotations
 
+import os
+from concurrent.futures import ThreadPoolExecutor
+
 import numpy as np
 
 __all__ = ["E4M3_MAX", "FP8_MATRICES", "e4m3_value", "e4m3_encode", "row_scales",
@@ -59,13 +62,32 @@ def e4m3_value(codes) -> np.ndarray:
 
 # the 127 non-negative finite values, increasing with the code 0 .. 126
 _POS = e4m3_value(np.arange(127, dtype=np.uint8))
+# value of every code, looked up by dequantize_rows
+_VALUES = e4m3_value(np.arange(256, dtype=np.uint8))
 
 
 def e4m3_encode(x) -> np.ndarray:
     """E4M3 code (uint8) of each value: the nearest finite value, ties to the
     even code (mantissa LSB 0), magnitudes beyond 448 saturated to 448; the
     sign bit is the sign of x (so -0.0 and negatives that round to zero get
-    code 0x80)."""
+    code 0x80).  Large arrays go through in blocks (the same arithmetic)."""
+    x = np.asarray(x)
+    if x.size > _BLOCK:
+        flat = x.reshape(-1)
+        out = np.empty(flat.shape, dtype=np.uint8)
+
+        def block(i):
+            out[i:i + _BLOCK] = _encode_block(flat[i:i + _BLOCK])
+        with ThreadPoolExecutor(min(32, os.cpu_count() or 1)) as ex:
+            list(ex.map(block, range(0, flat.size, _BLOCK)))
+        return out.reshape(x.shape)
+    return _encode_block(x)
+
+
+_BLOCK = 1 << 20
+
+
+def _encode_block(x) -> np.ndarray:
     x = np.asarray(x, dtype=np.float64)
     a = np.minimum(np.abs(x), E4M3_MAX)
     hi = np.searchsorted(_POS, a, side="left")            # first value >= a
@@ -97,7 +119,7 @@ def quantize_rows(W):
 
 def dequantize_rows(codes, scales, dtype=np.float64) -> np.ndarray:
     """s_r * value(q_rc) in `dtype`."""
-    v = e4m3_value(codes).astype(dtype)
+    v = _VALUES.astype(dtype)[np.asarray(codes, dtype=np.uint8)]
     return v * np.asarray(scales, dtype=dtype)[:, None]
 
 

@@ -119,6 +119,7 @@ def test_quantized_matvec_bruteforce():
     x = rng.standard_normal(33)
     codes, s = fp8.quantize_rows(W)
     want = []
+    deq = np.empty((7, 33))
     for r in range(7):
         acc = 0.0
         for c in range(33):
@@ -126,9 +127,11 @@ def test_quantized_matvec_bruteforce():
             sign = -1.0 if b & 0x80 else 1.0
             e, m = (b >> 3) & 15, b & 7
             val = sign * (m / 8 * 2.0 ** -6 if e == 0 else (1 + m / 8) * 2.0 ** (e - 7))
+            deq[r, c] = float(s[r]) * val
             acc += val * x[c]
         want.append(float(s[r]) * acc)
     np.testing.assert_allclose(fp8.quantized_matvec(codes, s, x), want, rtol=1e-12, atol=1e-15)
+    np.testing.assert_array_equal(fp8.dequantize_rows(codes, s), deq)
 
 
 def test_fp8_model_replaces_only_the_matrices():
