@@ -89,16 +89,29 @@ def profiled_traffic(w: synth.Workload, n_steps: int):
     return per_step * n_steps, path
 
 
-def decode_bytes(w: synth.Workload, pos0: int, n_steps: int) -> float:
+def weight_bytes_per_token(s: synth.ModelShape, weights: str = "fp16") -> float:
+    """Bytes of the weights one decode step reads: every matrix (fp16, or
+    one byte per FP8 E4M3 code plus a 4-byte scale per row), the fp16 norm
+    gains and one fp16 embedding row."""
+    if weights == "fp16":
+        return float(s.matrix_bytes_per_token())
+    d, L = s.d_model, s.n_layers
+    rows = L * (s.q_dim + 2 * s.kv_dim + d + 2 * s.ffn_dim + d) + s.vocab
+    elems = L * (d * s.q_dim + 2 * d * s.kv_dim + s.q_dim * d + 3 * d * s.ffn_dim) + s.vocab * d
+    return float(elems + 4 * rows + 2 * (2 * L * d + d) + 2 * d)
+
+
+def decode_bytes(w: synth.Workload, pos0: int, n_steps: int, weights: str = "fp16") -> float:
     """Algorithmic HBM bytes of n_steps decode steps starting at position
     pos0: every weight matrix, the norm gains and one embedding row per
     step, plus K/V reads of positions 0..pos and the K/V write at pos."""
     s = w.shape
     per_pos = s.kv_bytes_per_position()
+    wb = weight_bytes_per_token(s, weights)
     total = 0.0
     for i in range(n_steps):
         pos = pos0 + i
-        total += s.matrix_bytes_per_token() + per_pos * (pos + 1) + per_pos
+        total += wb + per_pos * (pos + 1) + per_pos
     return total
 
 
@@ -292,11 +305,17 @@ def run_reference(args, w, rank, world):
 
 
 def run_config(w: synth.Workload, args):
-    """The workload plus the token-selection rule of this run."""
+    """The workload plus the token-selection rule and weight format of this run."""
     sel = "greedy" if args.temperature <= 0 else {
         "sampling": "temperature (Gumbel-max, Philox4x64-10)",
-        "temperature": args.temperature, "seed": args.seed}
-    return dict(workload_config(w), token_selection=sel)
+        "temperature": args.temperature, "seed": args.seed,
+        "top_k": args.top_k, "top_p": args.top_p}
+    cfg = dict(workload_config(w), token_selection=sel)
+    if getattr(args, "weights", "fp16") == "fp8":
+        cfg["weights"] = ("fp16 N(0,0.02), seed 0, streamed as FP8 E4M3 with one fp32 "
+                          "scale per row (quantised by the library)")
+        cfg["weight_bytes_per_token"] = weight_bytes_per_token(w.shape, "fp8")
+    return cfg
 
 
 def workload_config(w: synth.Workload):
@@ -326,9 +345,10 @@ def run_gpu(args, w, dist, rank, world):
     stream = torch.cuda.current_stream()
     # the session keeps its packed copy of the matrices; the bench's own
     # references go, so the fp16 matrices are not held twice in HBM
-    sess = Session(w.shape, dev, max_seq=w.max_seq, stream=stream, keep_matrices=False)
+    sess = Session(w.shape, dev, max_seq=w.max_seq, stream=stream, keep_matrices=False,
+                   weight_format=args.weights)
     del dev
-    sess.set_sampling(args.temperature, args.seed)
+    sess.set_sampling(args.temperature, args.seed, top_k=args.top_k, top_p=args.top_p)
     sess.prefill(prompt)
     P, S = w.prompt_len, w.decode_steps
     out = np.empty(S, dtype=np.int32)
@@ -386,7 +406,7 @@ def run_gpu(args, w, dist, rank, world):
         return 0
     peak, peak_kind = _peaks()
     avg_launch_s = (sum(launch_ms) / len(launch_ms)) / 1000.0
-    bytes_launch = decode_bytes(w, P, S)
+    bytes_launch = decode_bytes(w, P, S, args.weights)
     achieved = bytes_launch / avg_launch_s / 1e9
     traffic, traffic_src = profiled_traffic(w, S)
     if args.traffic is not None:
@@ -396,7 +416,9 @@ def run_gpu(args, w, dist, rank, world):
         "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1000.0 * t_max / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None,
-        "dtype": "f16 weights+KV, f16 GEMV inputs, f32 accumulate",
+        "dtype": ("f16 weights+KV, f16 GEMV inputs, f32 accumulate" if args.weights == "fp16"
+                  else "fp8 E4M3 weights (fp32 row scales), f16 KV, f16 GEMV inputs, "
+                       "f32 accumulate"),
         "data": "synthetic",
         "config": run_config(w, args),
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
@@ -439,6 +461,10 @@ def main(argv=None):
                     choices=sorted(synth.WORKLOADS) + sorted(synth.PROFILE_WORKLOADS))
     ap.add_argument("--decode-steps", type=int, default=None,
                     help="decode steps per launch (default: the workload's); for profiler runs")
+    ap.add_argument("--weights", default="fp16", choices=["fp16", "fp8"],
+                    help="weight stream format: fp16 (default) or FP8 E4M3 with row scales")
+    ap.add_argument("--top-k", type=int, default=0, help="sampling: top-k bound (0 = off)")
+    ap.add_argument("--top-p", type=float, default=1.0, help="sampling: nucleus (1 = off)")
     ap.add_argument("--temperature", type=float, default=0.0,
                     help="0 = greedy (default); > 0 = in-kernel temperature sampling")
     ap.add_argument("--seed", type=int, default=0, help="sampling seed")

@@ -155,9 +155,23 @@ typedef enum {
   KIE_OPT_FAULT_STAGE = 7,    /* test hook: 0 QKV, 1 O, 2 gate/up, 3 down, 4 LM */
   KIE_OPT_POLL_BACKOFF_NS = 8, /* sleep between re-polls of another CTA's data (default 0) */
   KIE_OPT_TRACE_CLOCK = 9,     /* stage trace in SM cycles (1) instead of ns (0, default) */
-  KIE_OPT_L2_PREFETCH_BYTES = 10 /* per CTA, weight-stream bytes requested into L2 ahead of
+  KIE_OPT_L2_PREFETCH_BYTES = 10, /* per CTA, weight-stream bytes requested into L2 ahead of
                                     the shared-memory ring (multiple of 512, <= 16 MiB;
                                     0 = off, the default) */
+  KIE_OPT_WEIGHT_FP8 = 11      /* 1: stream the weight matrices as FP8 E4M3 with one fp32
+                                  scale per row (the pages' roadmap FP8 quantisation,
+                                  revietech.ru, "Kog выжимает максимум из GPU: 3000
+                                  токенов/с", section "Ограничения подхода"): half the
+                                  bytes per token.  Each row r of Wq, Wk, Wv, Wo, W_gate,
+                                  W_up, W_down and the LM head becomes s_r = max|W_r| / 448
+                                  (fp32; 1 for a zero row) and the codes E4M3(W_rc / s_r)
+                                  (fp32 division, round to nearest even, saturated at 448;
+                                  the codes of kie_quantize_e4m3); the GEMVs multiply the
+                                  codes, as fp16, with the fp16 inputs, accumulate in fp32
+                                  and scale the row sums.  The embedding, norm gains, KV
+                                  cache and everything else stay as they are.  0: fp16
+                                  weights (the default).  Rebuilds the packed weight copy
+                                  from the caller's matrices, which must still be valid */
 } kie_option;
 
 /* Bytes of the caller-provided KV cache: 2*n_layers*n_kv_heads*max_seq*(head_dim+8)*2.
@@ -310,6 +324,17 @@ KIE_API kie_status kie_destroy(kie_ctx *ctx);
 KIE_API kie_status kie_gemv_f16(const void *W, const float *x, float *y, int32_t N, int32_t K,
                                 int32_t iters, int32_t mode, int32_t chunk_bytes,
                                 void *cuda_stream, float *ms_out, double *stats_out);
+
+/* The FP8 quantisation of KIE_OPT_WEIGHT_FP8 applied to one matrix, for
+ * tests and for callers that store FP8 weights: W[N][K] fp16 row-major
+ * (device, 16-byte aligned, K a multiple of 16) to codes[N][K] (device,
+ * E4M3, one byte each, 16-byte aligned) and scales[N] (device, fp32), with
+ * s_r = max_c |W_rc| / 448 (1 for a zero row) and codes E4M3(W_rc / s_r),
+ * round to nearest even, saturated.  The caller owns all three buffers.
+ * Synchronous on `cuda_stream`.  KIE_ERR_INVALID_ARG for NULL or misaligned
+ * pointers or bad sizes, KIE_ERR_CUDA for a failed launch. */
+KIE_API kie_status kie_quantize_e4m3(const void *W, int32_t N, int32_t K, void *codes,
+                                     float *scales, void *cuda_stream);
 
 /* Largest fp16 weight matrix (N*K*2 bytes) kie_gemv_f16_noalloc takes. */
 #define KIE_NOALLOC_MAX_WEIGHT_BYTES (16u * 1024u * 1024u)

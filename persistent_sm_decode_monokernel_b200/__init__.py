@@ -46,14 +46,19 @@ class Session:
     keep_matrices=False the session drops its references to the matrices
     right after kie_create (their memory is freed once the caller drops
     its own), which halves the weights' device footprint; re-planning the
-    chunk size (KIE_OPT_CHUNK_BYTES) then raises, since it re-reads them.
+    chunk size (KIE_OPT_CHUNK_BYTES) or the weight format then raises, since
+    it re-reads them.
+
+    weight_format: "fp16" (the caller's weights as they are) or "fp8" (the
+    packed stream holds FP8 E4M3 codes with one fp32 scale per row,
+    KIE_OPT_WEIGHT_FP8), set before the matrices are released.
     """
 
     # the tensors kie_create's packed copy does not replace
     _KEPT = ("tok_emb", "final_norm")
 
     def __init__(self, shape, weights: Mapping[str, object], max_seq: int, eos_id: int = -1,
-                 stream=None, keep_matrices: bool = True):
+                 stream=None, keep_matrices: bool = True, weight_format: str = "fp16"):
         import torch
         load_library()
         self.shape = shape
@@ -71,6 +76,10 @@ class Session:
         self.stream = stream
         self.ctx = kie_create(self.desc, weights, self.kv, stream.cuda_stream)
         self._capture = None
+        if weight_format not in ("fp16", "fp8"):
+            raise ValueError(f"weight_format {weight_format!r}: 'fp16' or 'fp8'")
+        if weight_format == "fp8":
+            kie_set_option(self.ctx, _kie.KIE_OPT_WEIGHT_FP8, 1)
         if not keep_matrices:
             self.release_matrices()
 
@@ -120,9 +129,10 @@ class Session:
         self._trace = None
 
     def set_option(self, opt: int, value: int) -> None:
-        if opt == _kie.KIE_OPT_CHUNK_BYTES and getattr(self, "_matrices_released", False):
-            raise ValueError("KIE_OPT_CHUNK_BYTES re-reads the weight matrices, which this "
-                             "session has released (keep_matrices=False)")
+        if (opt in (_kie.KIE_OPT_CHUNK_BYTES, _kie.KIE_OPT_WEIGHT_FP8)
+                and getattr(self, "_matrices_released", False)):
+            raise ValueError("this option re-reads the weight matrices, which this session "
+                             "has released (keep_matrices=False)")
         kie_set_option(self.ctx, opt, value)
 
     def set_sampling(self, temperature: float, seed: int = 0, top_k: int = 0,

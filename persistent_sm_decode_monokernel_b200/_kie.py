@@ -42,6 +42,7 @@ KIE_OPT_FAULT_STAGE = 7
 KIE_OPT_POLL_BACKOFF_NS = 8
 KIE_OPT_TRACE_CLOCK = 9
 KIE_OPT_L2_PREFETCH_BYTES = 10
+KIE_OPT_WEIGHT_FP8 = 11
 
 STAGE_QKV, STAGE_O, STAGE_GU, STAGE_DOWN, STAGE_LM = range(5)
 
@@ -105,6 +106,7 @@ SIGNATURES = {
                                     ctypes.POINTER(ctypes.c_double)]),
     "kie_gemv_f16_noalloc": (ctypes.c_int, [_P, _P, _P, _I32, _I32, _P]),
     "kie_set_sampling_filter": (ctypes.c_int, [_P, _I32, ctypes.c_float]),
+    "kie_quantize_e4m3": (ctypes.c_int, [_P, _I32, _I32, _P, _P, _P]),
 }
 
 _lib: Optional[ctypes.CDLL] = None
@@ -283,6 +285,14 @@ def kie_gemv_f16(W, x, y, iters: int = 1, mode: int = 1, chunk_bytes: int = 3276
            "kie_gemv_f16")
     return ms.value, {"stream_wait_cycles": st[0], "producer_wait_cycles": st[1],
                       "grid": int(st[2]), "ring_bytes": int(st[3])}
+
+
+def kie_quantize_e4m3(W, codes, scales, stream=None) -> None:
+    """FP8 E4M3 codes [N, K] (uint8 tensor) and row scales [N] (fp32) of
+    an fp16 matrix W [N, K]: the rule of KIE_OPT_WEIGHT_FP8 (see kie.h)."""
+    N, K = W.shape
+    _check(load_library().kie_quantize_e4m3(_ptr(W), N, K, _ptr(codes), _ptr(scales),
+                                            ctypes.c_void_p(stream or 0)), "kie_quantize_e4m3")
 
 
 def kie_gemv_f16_noalloc(W, x, y, stream=None) -> None:

@@ -172,6 +172,23 @@ __device__ __forceinline__ void fma_f16x2_f32(float& a0, float& a1, uint32_t w, 
       : "r"(w), "r"(x));
 }
 
+// Four fp32 values to four FP8 E4M3 codes (byte k = value k): round to
+// nearest even, magnitudes beyond 448 saturated (cvt ... satfinite; the
+// first source operand goes to the high byte of each pair).
+__device__ __forceinline__ uint32_t f32x4_to_e4m3x4(float a, float b, float c, float d) {
+  unsigned short lo, hi;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(lo) : "f"(b), "f"(a));
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(hi) : "f"(d), "f"(c));
+  return (uint32_t)lo | ((uint32_t)hi << 16);
+}
+// Two E4M3 codes (low byte = element 0) to an fp16 pair (low half =
+// element 0); every E4M3 value is exact in fp16.
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(unsigned short v) {
+  uint32_t r;
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(r) : "h"(v));
+  return r;
+}
+
 // D = A B + D for one m16n8k16 tile: A 16x16 fp16 (row), B 16x8 fp16 (col),
 // fp32 accumulators (the PTX fragment layouts of mma.sync.m16n8k16).
 __device__ __forceinline__ void mma_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,

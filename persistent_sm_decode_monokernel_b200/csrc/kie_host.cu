@@ -52,6 +52,9 @@ struct kie_ctx {
   unsigned char* packed = nullptr;            // weight matrices in per-CTA stream order
   unsigned long long* packed_off = nullptr;   // [grid]
   size_t packed_bytes = 0;
+  int w8 = 0;                                 // packed stream: 0 fp16, 1 fp8 E4M3 + row scales
+  float* wscale = nullptr;                    // fp8: row scales, each CTA's in stream order
+  unsigned long long* wscale_off = nullptr;   // fp8: [grid] offsets (floats) into wscale
   kie::SmemLayout sm{};
 
   // session
@@ -128,6 +131,8 @@ void free_all(kie_ctx* c) {
   cudaFree(c->cta_stats);
   cudaFree(c->packed);
   cudaFree(c->packed_off);
+  cudaFree(c->wscale);
+  cudaFree(c->wscale_off);
   if (c->h_io) cudaFreeHost(c->h_io);
   if (c->ev0) cudaEventDestroy(c->ev0);
   if (c->ev1) cudaEventDestroy(c->ev1);
@@ -187,6 +192,9 @@ kie_status launch(kie_ctx* c, int n_steps, int pos0, const int32_t* host_ids, bo
   p.chunk_bytes = c->chunk_bytes;
   p.packed = c->packed;
   p.packed_off = c->packed_off;
+  p.w8 = c->w8;
+  p.wscale = c->wscale;
+  p.wscale_off = c->wscale_off;
   p.max_split = c->max_split;
   p.min_split_len = c->min_split_len;
   p.sm = c->sm;
@@ -249,21 +257,34 @@ kie_status launch(kie_ctx* c, int n_steps, int pos0, const int32_t* host_ids, bo
 }
 
 // (Re)builds the library's stream-ordered copy of the weight matrices for
-// the current partition and chunk size.  Reads the caller's matrices.
+// the current partition, chunk size and weight format (fp16, or fp8 E4M3
+// with row scales computed on the device first).  Reads the caller's
+// matrices.
 kie_status repack(kie_ctx* c) {
-  std::vector<unsigned long long> off(c->grid);
-  size_t total = 0;
+  std::vector<unsigned long long> off(c->grid), soff(c->grid);
+  size_t total = 0, srows = 0;
   for (int i = 0; i < c->grid; ++i) {
     off[i] = total;
-    total += (kie::stream_bytes(c->shape, c->hranges, i) + 511) / 512 * 512;
+    total += (kie::stream_bytes(c->shape, c->hranges, i, c->w8 ? 1 : 2) + 511) / 512 * 512;
+    soff[i] = srows;
+    srows += kie::stream_rows(c->shape, c->hranges, i);
   }
   cudaFree(c->packed);
   c->packed = nullptr;
+  cudaFree(c->wscale);
+  c->wscale = nullptr;
   if (!c->packed_off) KIE_CUDA(c, cudaMalloc(&c->packed_off, sizeof(unsigned long long) * c->grid));
   KIE_CUDA(c, cudaMalloc(&c->packed, total));
   c->packed_bytes = total;
   KIE_CUDA(c, cudaMemcpyAsync(c->packed_off, off.data(), sizeof(unsigned long long) * c->grid,
                               cudaMemcpyHostToDevice, c->stream));
+  if (c->w8) {
+    if (!c->wscale_off)
+      KIE_CUDA(c, cudaMalloc(&c->wscale_off, sizeof(unsigned long long) * c->grid));
+    KIE_CUDA(c, cudaMalloc(&c->wscale, sizeof(float) * srows));
+    KIE_CUDA(c, cudaMemcpyAsync(c->wscale_off, soff.data(), sizeof(unsigned long long) * c->grid,
+                                cudaMemcpyHostToDevice, c->stream));
+  }
   MonoParams p{};
   p.L = c->desc.n_layers;
   p.d = c->desc.d_model;
@@ -278,6 +299,9 @@ kie_status repack(kie_ctx* c) {
   p.grid = c->grid;
   p.chunk_bytes = c->chunk_bytes;
   p.packed_off = c->packed_off;
+  p.w8 = c->w8;
+  p.wscale = c->wscale;
+  p.wscale_off = c->wscale_off;
   KIE_CUDA(c, kie::repack_launch(p, c->packed, c->stream));
   KIE_CUDA(c, cudaStreamSynchronize(c->stream));
   return KIE_OK;
@@ -599,6 +623,19 @@ kie_status kie_set_eos_ids(kie_ctx* c, const int32_t* ids, int32_t n) {
   });
 }
 
+kie_status kie_quantize_e4m3(const void* W, int32_t N, int32_t K, void* codes, float* scales,
+                            void* cuda_stream) {
+  if (!W || !codes || !scales || N < 1 || K < 16 || K % 16) return KIE_ERR_INVALID_ARG;
+  if (!aligned16(W) || !aligned16(codes) || (reinterpret_cast<uintptr_t>(scales) & 3u))
+    return KIE_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
+  if (kie::quantize_launch(static_cast<const __half*>(W), N, K, static_cast<unsigned char*>(codes),
+                           scales, st) != cudaSuccess ||
+      cudaStreamSynchronize(st) != cudaSuccess)
+    return KIE_ERR_CUDA;
+  return KIE_OK;
+}
+
 kie_status kie_gemv_f16(const void* W, const float* x, float* y, int32_t N, int32_t K,
                         int32_t iters, int32_t mode, int32_t chunk_bytes, void* stream,
                         float* ms_out, double* stats_out) {
@@ -782,6 +819,15 @@ kie_status kie_set_option(kie_ctx* c, kie_option opt, int64_t v) {
         if (v < 0 || v > 100000) return KIE_ERR_INVALID_ARG;
         c->poll_ns = (unsigned)v;
         return KIE_OK;
+      case KIE_OPT_WEIGHT_FP8: {
+        if (c->failed) return set_err(c, KIE_ERR_STATE, "context failed earlier; destroy it");
+        if (v != 0 && v != 1) return KIE_ERR_INVALID_ARG;
+        if ((int)v == c->w8) return KIE_OK;
+        c->w8 = (int)v;
+        const kie_status st = repack(c);
+        if (st != KIE_OK) c->failed = true;
+        return st;
+      }
       case KIE_OPT_L2_PREFETCH_BYTES:
         if (v < 0 || v % 512 || v > (16 << 20)) return KIE_ERR_INVALID_ARG;
         c->l2_prefetch = v;

@@ -37,6 +37,7 @@
 #include <cfloat>
 #include <climits>
 #include <cuda_runtime.h>
+#include <type_traits>
 
 #include "kie_device.cuh"
 #include "kie_kernel.h"
@@ -74,6 +75,8 @@ __shared__ uint32_t kie_cur[3];
 // only: exact for thread 0 (the stage trace), and for the other threads the
 // position an error report names (possibly one stage behind).
 __shared__ int kie_at[3];
+// This CTA's row scales of an fp8 weight stream (set by make_plans).
+__shared__ const float* kie_wsc;
 
 // Views of the dynamic shared memory, always derived from the __shared__
 // symbol so that every access compiles to a shared-memory instruction.
@@ -119,7 +122,10 @@ struct StagePlan {
   int f_nk, f_base, f_rem;  // chunking of a full group (see Chunking)
   int t_nk, t_base, t_rem;  // chunking of the partial group
   int t_lw;              // partial group of <= kConsumerWarps rows: log2 warps per row
-  int pad[5];
+  // fp8 streams: index of the stage's first row scale among the CTA's scales
+  // of one layer (LM head: of the whole stream), and the scales of a layer
+  int sbase, rows_layer;
+  int pad[3];
 };
 __device__ __forceinline__ StagePlan* sm_plan(const MonoParams& p) {
   return reinterpret_cast<StagePlan*>(sm_misc(p) + kMiscHead + 2 * p.sm.resid_rows);
@@ -208,8 +214,8 @@ struct Chunking {
   __device__ __forceinline__ int first(int kc) const { return kc * base + min(kc, rem); }
   __device__ __forceinline__ int count(int kc) const { return base + (kc < rem ? 1 : 0); }
 };
-__device__ __forceinline__ Chunking chunking(int rg, int kp, int chunk_bytes) {
-  int mp = chunk_bytes / (rg * kPieceBytes);
+__device__ __forceinline__ Chunking chunking(int rg, int kp, int chunk_bytes, int pb) {
+  int mp = chunk_bytes / (rg * pb);
   if (mp < 1) mp = 1;
   Chunking c;
   c.nk = (kp + mp - 1) / mp;
@@ -226,9 +232,9 @@ __device__ __forceinline__ Chunking chunking(int rg, int kp, int chunk_bytes) {
 // the CTA's rows), its row count, its piece count and its first piece;
 // returning false stops the walk.
 template <class F>
-__device__ __forceinline__ bool for_each_chunk(int R, int kp, int chunk_bytes, F&& f) {
+__device__ __forceinline__ bool for_each_chunk(int R, int kp, int chunk_bytes, int pb, F&& f) {
   const int nfull = R / kGroupRows, tail = R - nfull * kGroupRows;
-  const Chunking cf = chunking(kGroupRows, kp, chunk_bytes);
+  const Chunking cf = chunking(kGroupRows, kp, chunk_bytes, pb);
   int g = 0;
   for (; g + 1 < nfull; g += 2)
     for (int kc = 0; kc < cf.nk; ++kc)
@@ -238,7 +244,7 @@ __device__ __forceinline__ bool for_each_chunk(int R, int kp, int chunk_bytes, F
     for (int kc = 0; kc < cf.nk; ++kc)
       if (!f(g * kGroupRows, kGroupRows, cf.count(kc), cf.first(kc))) return false;
   if (tail > 0) {
-    const Chunking ct = chunking(tail, kp, chunk_bytes);
+    const Chunking ct = chunking(tail, kp, chunk_bytes, pb);
     for (int kc = 0; kc < ct.nk; ++kc)
       if (!f(nfull * kGroupRows, tail, ct.count(kc), ct.first(kc))) return false;
   }
@@ -469,8 +475,9 @@ struct Producer {
     const int R = range_rows(p, st, r.x, r.y);
     const int kp = stage_k(p, st) / kPieceElems;
     const int nfull = R / kGroupRows, tail = R - nfull * kGroupRows;
-    const Chunking cf = chunking(kGroupRows, kp, p.chunk_bytes);
-    const Chunking ct = chunking(tail > 0 ? tail : 1, kp, p.chunk_bytes);
+    const int pb = piece_bytes(p.w8);
+    const Chunking cf = chunking(kGroupRows, kp, p.chunk_bytes, pb);
+    const Chunking ct = chunking(tail > 0 ? tail : 1, kp, p.chunk_bytes, pb);
 #pragma unroll 1
     for (int sg = 0; sg < 3; ++sg) {
       const int reps = sg == 0 ? nfull / 2 : (sg == 1 ? (nfull & 1) : (tail > 0 ? 1 : 0));
@@ -481,7 +488,7 @@ struct Producer {
       for (int rep = 0; rep < reps; ++rep)
 #pragma unroll 1
         for (int j = 0; j < c.nk * mult; ++j) {
-          const uint32_t sz = (uint32_t)(rows * c.count(j / mult) * kPieceBytes);
+          const uint32_t sz = (uint32_t)(rows * c.count(j / mult) * pb);
           if (p.l2_prefetch > 0) prefetch(sz);
           if (!chunk(src, sz)) return false;
           pf_ahead -= sz;
@@ -605,25 +612,74 @@ struct Producer {
   }
 };
 
+// FP8 E4M3 weights with one fp32 scale per row: s = max |w| / 448 (1 for a
+// zero row), codes E4M3(w / s) with fp32 division, round to nearest even,
+// saturated at +-448.
+__device__ __forceinline__ float e4m3_row_scale(float amax) {
+  return amax > 0.f ? __fdiv_rn(amax, 448.0f) : 1.0f;
+}
+// 16 fp16 weights (two 16-byte loads) to 16 codes
+__device__ __forceinline__ uint4 quantize16(const uint4& a, const uint4& b, float s) {
+  const uint32_t hw[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+  uint32_t o[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const float2 f0 = __half22float2(*reinterpret_cast<const __half2*>(&hw[2 * k]));
+    const float2 f1 = __half22float2(*reinterpret_cast<const __half2*>(&hw[2 * k + 1]));
+    o[k] = dev::f32x4_to_e4m3x4(__fdiv_rn(f0.x, s), __fdiv_rn(f0.y, s), __fdiv_rn(f1.x, s),
+                                __fdiv_rn(f1.y, s));
+  }
+  return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
 // Lays out CTA blockIdx.x's one-token weight stream in the order Producer
 // streams it: per layer the QKV, O, gate/up and down chunks, then the LM
-// head, each chunk [row][piece][512 B].  Run once per model.
-__device__ void repack_stage(const MonoParams& p, int st, const LayerW& w, unsigned char*& dst) {
+// head, each chunk [row][piece][piece bytes].  fp16: a copy; fp8: every
+// weight w of row r becomes the E4M3 code of w / s_r (fp32 division, round
+// to nearest even, saturated at +-448), s_r the row's scale (rowscale_stage).
+// Run once per model (and per change of the weight format or chunk size).
+__device__ void repack_stage(const MonoParams& p, int st, const LayerW& w, unsigned char*& dst,
+                             const float* scales) {
   const int2 r = p.ranges[st * p.grid + blockIdx.x];
   const int R = range_rows(p, st, r.x, r.y);
   const int kp = stage_k(p, st) / kPieceElems;
-  for_each_chunk(R, kp, p.chunk_bytes, [&](int g0, int rg, int n, int p0) {
-    const int n16 = n * kPieceBytes / 16;
+  const int pb = piece_bytes(p.w8);
+  for_each_chunk(R, kp, p.chunk_bytes, pb, [&](int g0, int rg, int n, int p0) {
+    const int n16 = n * pb / 16;   // 16-byte units of a row's part of the chunk
     uint4* d = reinterpret_cast<uint4*>(dst);
     for (int e = threadIdx.x; e < rg * n16; e += blockDim.x) {
       const int j = e / n16, q = e - j * n16;
-      const uint4* src = reinterpret_cast<const uint4*>(row_ptr(p, st, w, r.x, r.y, g0 + j) +
-                                                        (size_t)p0 * kPieceElems);
-      d[e] = src[q];
+      const __half* row = row_ptr(p, st, w, r.x, r.y, g0 + j) + (size_t)p0 * kPieceElems;
+      if (!p.w8) {
+        d[e] = reinterpret_cast<const uint4*>(row)[q];
+      } else {   // 16 weights -> 16 codes
+        d[e] = quantize16(reinterpret_cast<const uint4*>(row)[2 * q],
+                          reinterpret_cast<const uint4*>(row)[2 * q + 1], scales[g0 + j]);
+      }
     }
-    dst += (size_t)rg * n * kPieceBytes;
+    dst += (size_t)rg * n * pb;
     return true;
   });
+}
+
+// Row scales of CTA blockIdx.x's rows of stage st, in stream order:
+// s_r = max_c |w_rc| / 448 in fp32 (1 for a zero row).  One warp per row.
+__device__ void rowscale_stage(const MonoParams& p, int st, const LayerW& w, float* out) {
+  const int2 r = p.ranges[st * p.grid + blockIdx.x];
+  const int R = range_rows(p, st, r.x, r.y);
+  const int K = stage_k(p, st);
+  const int lane = threadIdx.x & 31;
+  for (int j = threadIdx.x >> 5; j < R; j += blockDim.x >> 5) {
+    const __half2* row = reinterpret_cast<const __half2*>(row_ptr(p, st, w, r.x, r.y, j));
+    float m = 0.f;
+    for (int k = lane; k < K / 2; k += 32) {
+      const float2 v = __half22float2(row[k]);
+      m = fmaxf(m, fmaxf(fabsf(v.x), fabsf(v.y)));
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    if (lane == 0) out[j] = e4m3_row_scale(m);
+  }
 }
 
 // ----------------------------------------------------------------- consumer
@@ -926,6 +982,13 @@ struct Consumer {
     dev::fma_f16x2_f32(c[4], c[5], w.z, x.z);
     dev::fma_f16x2_f32(c[6], c[7], w.w, x.w);
   }
+  // fp8 weights: lane l's 8 E4M3 codes of a piece (elements 8l .. 8l+7)
+  __device__ __forceinline__ static void dot_piece(const uint2& w, const uint4& x, float (&c)[8]) {
+    dev::fma_f16x2_f32(c[0], c[1], dev::e4m3x2_to_f16x2((unsigned short)(w.x & 0xFFFFu)), x.x);
+    dev::fma_f16x2_f32(c[2], c[3], dev::e4m3x2_to_f16x2((unsigned short)(w.x >> 16)), x.y);
+    dev::fma_f16x2_f32(c[4], c[5], dev::e4m3x2_to_f16x2((unsigned short)(w.y & 0xFFFFu)), x.z);
+    dev::fma_f16x2_f32(c[6], c[7], dev::e4m3x2_to_f16x2((unsigned short)(w.y >> 16)), x.w);
+  }
   __device__ __forceinline__ static float sum8(const float (&c)[8]) {
     return ((c[0] + c[1]) + (c[2] + c[3])) + ((c[4] + c[5]) + (c[6] + c[7]));
   }
@@ -942,12 +1005,12 @@ struct Consumer {
       pl.kp = stage_k(p, st) / kPieceElems;
       pl.nfull = pl.rows / kGroupRows;
       pl.tail = pl.rows - pl.nfull * kGroupRows;
-      const Chunking f = chunking(kGroupRows, pl.kp, p.chunk_bytes);
+      const Chunking f = chunking(kGroupRows, pl.kp, p.chunk_bytes, piece_bytes(p.w8));
       pl.f_nk = f.nk;
       pl.f_base = f.base;
       pl.f_rem = f.rem;
       if (pl.tail > 0) {
-        const Chunking t = chunking(pl.tail, pl.kp, p.chunk_bytes);
+        const Chunking t = chunking(pl.tail, pl.kp, p.chunk_bytes, piece_bytes(p.w8));
         pl.t_nk = t.nk;
         pl.t_base = t.base;
         pl.t_rem = t.rem;
@@ -955,20 +1018,38 @@ struct Consumer {
         while ((pl.tail << (lw + 1)) <= kConsumerWarps) ++lw;
         pl.t_lw = lw;
       }
+      // row-scale positions of an fp8 stream (per layer: QKV, O, gate/up,
+      // down rows; then the LM head after all layers)
+      int before = 0, layer_rows = 0;
+      for (int s2 = ST_QKV; s2 <= ST_DOWN; ++s2) {
+        const int2 r2 = p.ranges[s2 * p.grid + blockIdx.x];
+        const int n2 = range_rows(p, s2, r2.x, r2.y);
+        if (s2 < st) before += n2;
+        layer_rows += n2;
+      }
+      pl.rows_layer = layer_rows;
+      pl.sbase = st == ST_LM ? p.L * layer_rows : before;
       sm_plan(p)[st] = pl;
     }
+    if (tid == 0) kie_wsc = p.w8 ? p.wscale + p.wscale_off[blockIdx.x] : nullptr;
   }
 
-  // GEMV of this CTA's rows of stage st: raw dot products, read back with
-  // row_result.  A group of up to 16 rows streams as k-chunks.  In a group
-  // of more than 8 rows warp w owns rows w and w+8 for all of the group's
-  // chunks (one activation load serves two rows) and keeps its partial sums
-  // in registers.  A last group of at most 8 rows gives each row 8/rg
-  // (power of two) warps that split its pieces; their partial sums are
-  // added in a fixed order by row_result, so results do not depend on
-  // timing.  Ring positions and the parameter block are held in registers
-  // for the whole stage; one barrier at the end.
-  __device__ __noinline__ bool gemv(int st) {
+  // GEMV of this CTA's rows of stage st: dot products (times the rows'
+  // scales when the stream is fp8), read back with row_result.  A group of
+  // up to 16 rows streams as k-chunks.  In a group of more than 8 rows warp
+  // w owns rows w and w+8 for all of the group's chunks (one activation load
+  // serves two rows) and keeps its partial sums in registers.  A last group
+  // of at most 8 rows gives each row 8/rg (power of two) warps that split
+  // its pieces; their partial sums are added in a fixed order by
+  // row_result, so results do not depend on timing.  Ring positions and the
+  // parameter block are held in registers for the whole stage; one barrier
+  // at the end.  W8: pieces of fp8 E4M3 weights (8 bytes a lane), converted
+  // to fp16 pairs and multiplied like fp16 weights; rsc: the row scales of
+  // this CTA's rows of the stage (unused for fp16).
+  template <bool W8>
+  __device__ __noinline__ bool gemv(int st, const float* rsc) {
+    using WT = typename std::conditional<W8, uint2, uint4>::type;   // a lane's weights of a piece
+    constexpr int PB = W8 ? kPieceElems : kPieceBytes;
     const MonoParams& p = kie_p;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const StagePlan pl = sm_plan(p)[st];
@@ -992,24 +1073,26 @@ struct Consumer {
       if (lane == 0) dev::mbar_arrive(empty_s + 8 * (cr & (kRingBars - 1)));
       ++cr;
     };
+    // scale of row k (1 for fp16); issued early, used when the row's sum is written
+    auto scale_of = [&](int k) -> float { return W8 ? __ldg(rsc + k) : 1.0f; };
     // groups of more than kConsumerWarps rows / full groups: warp w owns
     // rows w (and w + kConsumerWarps when two rows per warp; the second may
     // be missing)
     auto group2 = [&](int g0, int rg, int nk, int base, int rem) {
       const bool two = kRowsPerWarp == 2 && warp + kConsumerWarps < rg;
+      const float s0 = scale_of(g0 + warp), s1 = two ? scale_of(g0 + warp + kConsumerWarps) : 1.f;
       float c0[8], c1[8];
 #pragma unroll
       for (int i = 0; i < 8; ++i) c0[i] = c1[i] = 0.f;
       for (int kc = 0; kc < nk; ++kc) {
         const int n = base + (kc < rem ? 1 : 0), p0 = kc * base + min(kc, rem);
         uint32_t off;
-        if (!wait((uint32_t)(rg * n * kPieceBytes), off)) bad = true;
+        if (!wait((uint32_t)(rg * n * PB), off)) bad = true;
         if (!bad) {
-          const uint4* w0 =
-              reinterpret_cast<const uint4*>(ring + off + (size_t)warp * n * kPieceBytes) + lane;
+          const WT* w0 = reinterpret_cast<const WT*>(ring + off + (size_t)warp * n * PB) + lane;
           const uint4* x = xv + (size_t)p0 * 32;
           if (two) {
-            const uint4* w1 = w0 + (size_t)kConsumerWarps * n * 32;
+            const WT* w1 = w0 + (size_t)kConsumerWarps * n * 32;
 #pragma unroll 4
             for (int q = 0; q < n; ++q) {
               const uint4 a = x[q * 32];
@@ -1031,11 +1114,11 @@ struct Consumer {
         float t = (upper ? b : a) + __shfl_xor_sync(0xffffffffu, upper ? a : b, 16);
 #pragma unroll
         for (int o = 8; o > 0; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
-        if (lane == 0) rowacc[g0 + warp] = t;
-        if (two && lane == 16) rowacc[g0 + warp + kConsumerWarps] = t;
+        if (lane == 0) rowacc[g0 + warp] = t * s0;
+        if (two && lane == 16) rowacc[g0 + warp + kConsumerWarps] = t * s1;
       } else {
         const float t = dev::warp_sum(sum8(c0));
-        if (lane == 0) rowacc[g0 + warp] = t;
+        if (lane == 0) rowacc[g0 + warp] = t * s0;
       }
     };
     // pairs of full groups (their chunks interleave in the stream): warp w
@@ -1043,6 +1126,9 @@ struct Consumer {
     // of them
     auto group_pair = [&](int g0) {
       constexpr int RW = 2 * kRowsPerWarp;             // rows per warp
+      // the row this lane writes after the butterfly (lanes 0, 8, 16, 24)
+      const int my_row = (lane & 8 ? kGroupRows : 0) + (lane & 16 ? kConsumerWarps : 0) + warp;
+      const float s_me = (lane & 7) == 0 ? scale_of(g0 + (RW == 4 ? my_row : (lane & 16 ? kGroupRows : 0) + warp)) : 1.f;
       float c[RW][8];
 #pragma unroll
       for (int r = 0; r < RW; ++r)
@@ -1050,14 +1136,14 @@ struct Consumer {
         for (int i = 0; i < 8; ++i) c[r][i] = 0.f;
       for (int kc = 0; kc < pl.f_nk; ++kc) {
         const int n = pl.f_base + (kc < pl.f_rem ? 1 : 0), p0 = kc * pl.f_base + min(kc, pl.f_rem);
-        const uint32_t sz = (uint32_t)(kGroupRows * n * kPieceBytes);
+        const uint32_t sz = (uint32_t)(kGroupRows * n * PB);
         uint32_t offa, offb;
         if (!wait(sz, offa)) bad = true;
         if (!wait(sz, offb)) bad = true;
         if (!bad) {
           const uint4* x = xv + (size_t)p0 * 32;
-          const uint4* wa = reinterpret_cast<const uint4*>(ring + offa + (size_t)warp * n * kPieceBytes) + lane;
-          const uint4* wb = reinterpret_cast<const uint4*>(ring + offb + (size_t)warp * n * kPieceBytes) + lane;
+          const WT* wa = reinterpret_cast<const WT*>(ring + offa + (size_t)warp * n * PB) + lane;
+          const WT* wb = reinterpret_cast<const WT*>(ring + offb + (size_t)warp * n * PB) + lane;
           const size_t second = (size_t)kConsumerWarps * n * 32;   // row w + kConsumerWarps
 #pragma unroll 2
           for (int q = 0; q < n; ++q) {
@@ -1090,17 +1176,14 @@ struct Consumer {
 #pragma unroll
         for (int o = 4; o > 0; o >>= 1) u += __shfl_xor_sync(0xffffffffu, u, o);
         // lane 0: A w, 8: B w, 16: A w+K, 24: B w+K
-        if ((lane & 7) == 0) {
-          const int row = (lane & 8 ? kGroupRows : 0) + (lane & 16 ? kConsumerWarps : 0) + warp;
-          rowacc[g0 + row] = u;
-        }
+        if ((lane & 7) == 0) rowacc[g0 + my_row] = u * s_me;
       } else {
         // rows: 0 = A w, 1 = B w
         const bool up = (lane & 16) != 0;
         float u = (up ? v[1] : v[0]) + __shfl_xor_sync(0xffffffffu, up ? v[0] : v[1], 16);
 #pragma unroll
         for (int o = 8; o > 0; o >>= 1) u += __shfl_xor_sync(0xffffffffu, u, o);
-        if ((lane & 15) == 0) rowacc[g0 + (up ? kGroupRows : 0) + warp] = u;
+        if ((lane & 15) == 0) rowacc[g0 + (up ? kGroupRows : 0) + warp] = u * s_me;
       }
     };
     int g = 0;
@@ -1113,17 +1196,17 @@ struct Consumer {
       const int lw = pl.t_lw, rg = pl.tail;
       const int r = warp >> lw, part = warp & ((1 << lw) - 1);
       const bool active = r < rg;
+      const float s_r = active ? scale_of(tb + r) : 1.f;
       float c0[8];
 #pragma unroll
       for (int i = 0; i < 8; ++i) c0[i] = 0.f;
       for (int kc = 0; kc < pl.t_nk; ++kc) {
         const int n = pl.t_base + (kc < pl.t_rem ? 1 : 0), p0 = kc * pl.t_base + min(kc, pl.t_rem);
         uint32_t off;
-        if (!wait((uint32_t)(rg * n * kPieceBytes), off)) bad = true;
+        if (!wait((uint32_t)(rg * n * PB), off)) bad = true;
         if (active && !bad) {
           const int pa = (part * n) >> lw, pb = ((part + 1) * n) >> lw;
-          const uint4* wr =
-              reinterpret_cast<const uint4*>(ring + off + (size_t)r * n * kPieceBytes) + lane;
+          const WT* wr = reinterpret_cast<const WT*>(ring + off + (size_t)r * n * PB) + lane;
           const uint4* x = xv + (size_t)p0 * 32;
 #pragma unroll 4
           for (int q = pa; q < pb; ++q) dot_piece(wr[q * 32], x[q * 32], c0);
@@ -1131,7 +1214,7 @@ struct Consumer {
         release();
       }
       if (active) {
-        const float s = dev::warp_sum(sum8(c0));
+        const float s = dev::warp_sum(sum8(c0)) * s_r;
         if (lane == 0) {
           if (lw == 0) rowacc[tb + r] = s;
           else sm_part(p)[warp] = s;
@@ -1145,6 +1228,14 @@ struct Consumer {
       kie_cur[2] = ce;
     }
     return !any_bad;
+  }
+
+  // The GEMV of stage st of layer `layer` in the stream's weight format.
+  __device__ __forceinline__ bool gemv_stage(int st, int layer) {
+    const MonoParams& p = kie_p;
+    if (!p.w8) return gemv<false>(st, nullptr);
+    const StagePlan& pl = sm_plan(p)[st];
+    return gemv<true>(st, kie_wsc + (st == ST_LM ? 0 : (size_t)layer * pl.rows_layer) + pl.sbase);
   }
 
   // Raw dot product of row k (0-based within the CTA's rows) of the last gemv.
@@ -1187,7 +1278,7 @@ struct Consumer {
       if (u < r.y && u < np_all) cs0 = cs[(u < nqp ? u : u - nqp) % half];
     }
     if (!load_vec(p.x_attn, tag, emb, p.d, w.attn_norm, ss, 10)) return false;
-    if (!gemv(ST_QKV)) return false;
+    if (!gemv_stage(ST_QKV, layer)) return false;
     const StagePlan pl = sm_plan(p)[ST_QKV];
     const float rs = 1.0f / sqrtf(ss / (float)p.d + p.eps);
     const int np = qkv_pairs_in(p, r.x, r.y);
@@ -1551,7 +1642,7 @@ struct Consumer {
     if (r.y <= r.x) return true;
     float ss;
     if (!load_vec(p.obuf, tag, nullptr, p.H * p.hd, nullptr, ss, 30)) return false;
-    if (!gemv(ST_O)) return false;
+    if (!gemv_stage(ST_O, layer)) return false;
     const StagePlan pl = sm_plan(p)[ST_O];
     for (int u = r.x + tid; u < r.y; u += kConsumerThreads) {
       const int k = u - r.x;
@@ -1564,7 +1655,7 @@ struct Consumer {
   }
 
   // RMSNorm + gate/up GEMV + SwiGLU -> h.
-  __device__ bool stage_gu(const LayerW& w, unsigned tag, bool skip) {
+  __device__ bool stage_gu(const LayerW& w, int layer, unsigned tag, bool skip) {
     const MonoParams& p = kie_p;
     const int tid = (int)threadIdx.x;
     at_stage(ST_GU);
@@ -1572,7 +1663,7 @@ struct Consumer {
     if (r.y <= r.x) return true;
     float ss;
     if (!load_vec(p.x_ffn, tag, nullptr, p.d, w.ffn_norm, ss, 40)) return false;
-    if (!gemv(ST_GU)) return false;
+    if (!gemv_stage(ST_GU, layer)) return false;
     const StagePlan pl = sm_plan(p)[ST_GU];
     const float rs = 1.0f / sqrtf(ss / (float)p.d + p.eps);
     for (int u = r.x + tid; u < r.y; u += kConsumerThreads) {
@@ -1585,7 +1676,7 @@ struct Consumer {
   }
 
   // Down GEMV + residual -> x_attn (input of the next layer).
-  __device__ bool stage_down(const LayerW& w, unsigned tag, unsigned tag_next, bool skip) {
+  __device__ bool stage_down(const LayerW& w, int layer, unsigned tag, unsigned tag_next, bool skip) {
     const MonoParams& p = kie_p;
     const int tid = (int)threadIdx.x;
     at_stage(ST_DOWN);
@@ -1593,7 +1684,7 @@ struct Consumer {
     if (r.y <= r.x) return true;
     float ss;
     if (!load_vec(p.hbuf, tag, nullptr, p.F, nullptr, ss, 50)) return false;
-    if (!gemv(ST_DOWN)) return false;
+    if (!gemv_stage(ST_DOWN, layer)) return false;
     const StagePlan pl = sm_plan(p)[ST_DOWN];
     for (int u = r.x + tid; u < r.y; u += kConsumerThreads) {
       const int k = u - r.x;
@@ -1821,7 +1912,7 @@ struct Consumer {
     if (pick && r.y > r.x) {
       float ss;
       if (!load_vec(p.x_attn, tag, nullptr, p.d, p.final_norm, ss, 60)) return -1;
-      if (!gemv(ST_LM)) return -1;
+      if (!gemv_stage(ST_LM, 0)) return -1;
       const StagePlan pl = sm_plan(p)[ST_LM];
       trace(2);
       const float rs = 1.0f / sqrtf(ss / (float)p.d + p.eps);
@@ -1917,9 +2008,10 @@ struct Consumer {
     const int kp = stage_k(p, st) / kPieceElems;
     bool bad = false;
     uint32_t ci = kie_cur[0], cr = kie_cur[1], ce = kie_cur[2];
-    for_each_chunk(R, kp, p.chunk_bytes, [&](int, int rg, int n, int) {
+    const int pb = piece_bytes(p.w8);
+    for_each_chunk(R, kp, p.chunk_bytes, pb, [&](int, int rg, int n, int) {
       uint32_t off;
-      if (!wait_chunk((uint32_t)(rg * n * kPieceBytes), off, ci, ce)) bad = true;
+      if (!wait_chunk((uint32_t)(rg * n * pb), off, ci, ce)) bad = true;
       release_chunk(cr);
       return true;
     });
@@ -1949,7 +2041,7 @@ struct Consumer {
     bool ok = true;
     for (int it = 0; it < iters && ok; ++it) {
       dev::consumer_sync();   // the ring cursors thread 0 wrote back are visible
-      ok = mode == 0 ? skip_stage(ST_LM, r.x, r.y) : gemv(ST_LM);
+      ok = mode == 0 ? skip_stage(ST_LM, r.x, r.y) : gemv_stage(ST_LM, 0);
     }
     if (ok && mode == 1)
       for (int u = r.x + tid; u < r.y; u += kConsumerThreads) y[u] = row_result(sm_plan(p)[ST_LM], u - r.x);
@@ -1988,10 +2080,10 @@ struct Consumer {
         ok = ok && stage_o(w, l, tok, tag, fst == ST_O);
         trace(5);
         trace_stream_wait(ST_O);
-        ok = ok && stage_gu(w, tag, fst == ST_GU);
+        ok = ok && stage_gu(w, l, tag, fst == ST_GU);
         trace(7);
         trace_stream_wait(ST_GU);
-        ok = ok && stage_down(w, tag, tag + 1u, fst == ST_DOWN);
+        ok = ok && stage_down(w, l, tag, tag + 1u, fst == ST_DOWN);
         trace(9);
         trace_stream_wait(ST_DOWN);
       }
@@ -2089,20 +2181,75 @@ __global__ void __launch_bounds__(kThreads, 1)
   c.gemv_bench(mode, x, y, iters);
 }
 
+__global__ void __launch_bounds__(256) kie_rowscale_kernel(const __grid_constant__ MonoParams p) {
+  float* out = const_cast<float*>(p.wscale) + p.wscale_off[blockIdx.x];
+  for (int l = 0; l < p.L; ++l) {
+    const LayerW& w = p.layers[l];
+    for (int st = ST_QKV; st <= ST_DOWN; ++st) {
+      rowscale_stage(p, st, w, out);
+      const int2 r = p.ranges[st * p.grid + blockIdx.x];
+      out += range_rows(p, st, r.x, r.y);
+    }
+  }
+  rowscale_stage(p, ST_LM, p.layers[0], out);
+}
+
 __global__ void __launch_bounds__(256) kie_repack_kernel(const __grid_constant__ MonoParams p,
                                                          unsigned char* packed) {
   unsigned char* dst = packed + p.packed_off[blockIdx.x];
+  const float* sc = p.w8 ? p.wscale + p.wscale_off[blockIdx.x] : nullptr;
   for (int l = 0; l < p.L; ++l) {
     const LayerW& w = p.layers[l];
-    repack_stage(p, ST_QKV, w, dst);
-    repack_stage(p, ST_O, w, dst);
-    repack_stage(p, ST_GU, w, dst);
-    repack_stage(p, ST_DOWN, w, dst);
+    for (int st = ST_QKV; st <= ST_DOWN; ++st) {
+      repack_stage(p, st, w, dst, sc);
+      if (sc) {
+        const int2 r = p.ranges[st * p.grid + blockIdx.x];
+        sc += range_rows(p, st, r.x, r.y);
+      }
+    }
   }
-  repack_stage(p, ST_LM, p.layers[0], dst);
+  repack_stage(p, ST_LM, p.layers[0], dst, sc);
+}
+
+// One matrix W[N][K] (fp16, row-major) to E4M3 codes[N][K] and scales[N]:
+// a warp per row.
+__global__ void __launch_bounds__(256) kie_quantize_kernel(const __half* W, int N, int K,
+                                                           unsigned char* codes, float* scales) {
+  const int lane = threadIdx.x & 31;
+  for (int r = blockIdx.x * 8 + (int)(threadIdx.x >> 5); r < N; r += gridDim.x * 8) {
+    const uint4* row = reinterpret_cast<const uint4*>(W + (size_t)r * K);
+    float m = 0.f;
+    for (int k = lane; k < K / 8; k += 32) {
+      const uint4 v = row[k];
+      const uint32_t hw[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int h = 0; h < 4; ++h) {
+        const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&hw[h]));
+        m = fmaxf(m, fmaxf(fabsf(f.x), fabsf(f.y)));
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    const float sr = e4m3_row_scale(m);
+    if (lane == 0) scales[r] = sr;
+    uint4* out = reinterpret_cast<uint4*>(codes + (size_t)r * K);
+    for (int q = lane; q < K / 16; q += 32) out[q] = quantize16(row[2 * q], row[2 * q + 1], sr);
+  }
+}
+
+cudaError_t quantize_launch(const __half* W, int N, int K, unsigned char* codes, float* scales,
+                            cudaStream_t s) {
+  const int blocks = (N + 7) / 8 < 1184 ? (N + 7) / 8 : 1184;
+  kie_quantize_kernel<<<blocks, 256, 0, s>>>(W, N, K, codes, scales);
+  return cudaGetLastError();
 }
 
 cudaError_t repack_launch(const MonoParams& p, unsigned char* packed, cudaStream_t s) {
+  if (p.w8) {
+    kie_rowscale_kernel<<<p.grid, 256, 0, s>>>(p);
+    const cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
   kie_repack_kernel<<<p.grid, 256, 0, s>>>(p, packed);
   return cudaGetLastError();
 }

@@ -3,6 +3,8 @@
 
 #include <cuda_runtime.h>
 
+#include <cuda_fp16.h>
+
 #include "kie_params.h"
 
 namespace kie {
@@ -18,6 +20,11 @@ cudaError_t mono_configure(int hd, int smem_bytes, int* blocks_per_sm);
 
 // Cooperative launch (all CTAs co-resident) of `grid` persistent CTAs.
 cudaError_t mono_launch(const MonoParams& p, int hd, int grid, int smem_bytes, cudaStream_t s);
+
+// FP8 E4M3 quantisation of one fp16 matrix W[N][K] (row-major, K a multiple
+// of 16): codes[N][K] and one fp32 scale per row, the weight stream's rule.
+cudaError_t quantize_launch(const __half* W, int N, int K, unsigned char* codes, float* scales,
+                            cudaStream_t s);
 
 // Copies the weight matrices into `packed`, each CTA's one-token stream at
 // p.packed_off[cta], in the order the decode kernel streams them.

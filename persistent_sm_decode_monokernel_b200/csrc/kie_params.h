@@ -29,8 +29,11 @@ static_assert((kConsumerWarps + 4) * 32 * kRegsLaunch <= 65536, "launch register
 constexpr int kGroupRows = 16;              // rows streamed together
 constexpr int kRowsPerWarp = kGroupRows / kConsumerWarps;  // rows of a full group per warp
 static_assert(kRowsPerWarp == 1 || kRowsPerWarp == 2, "group mapping");
-constexpr int kPieceElems = 256;             // one warp pass: 32 lanes x 8 fp16
-constexpr int kPieceBytes = kPieceElems * 2;
+constexpr int kPieceElems = 256;             // one warp pass: 32 lanes x 8 weights
+constexpr int kPieceBytes = kPieceElems * 2;   // an fp16 piece (16 bytes a lane)
+// Bytes of a piece in the packed stream: fp16 weights, or fp8 E4M3 (8 bytes
+// a lane).
+__host__ __device__ constexpr int piece_bytes(int w8) { return w8 ? kPieceElems : kPieceBytes; }
 constexpr int kRingBars = 16;                // mbarrier pairs of the byte ring (power of 2)
 constexpr int kMaxGroup = 8;                 // heads per KV head handled by one CTA
 constexpr int kAttnBlock = 256;              // positions per attention block
@@ -102,6 +105,11 @@ struct MonoParams {
   int top_k;
   double top_p;
   unsigned long long* cands;  // [grid][kMaxTopK][2] tagged words: every CTA's local top-k keys
+  // weight format of the packed stream: 0 fp16; 1 fp8 E4M3 with one fp32
+  // scale per row (weight = scale * value(code))
+  int w8;
+  const float* wscale;                    // row scales, each CTA's in its stream order
+  const unsigned long long* wscale_off;   // [grid] offset (in floats) of each CTA's scales
   // weights (device)
   const LayerW* layers;
   const __half* tok_emb;

@@ -129,13 +129,23 @@ bool plan_smem(const Shape& s, int grid, int chunk_bytes, int smem_limit,
   return L.total <= smem_limit;
 }
 
-size_t stream_bytes(const Shape& s, const std::vector<std::vector<int2>>& ranges, int cta) {
+size_t stream_bytes(const Shape& s, const std::vector<std::vector<int2>>& ranges, int cta,
+                    int elem_bytes) {
   size_t layer = 0;
   for (int st = ST_QKV; st <= ST_DOWN; ++st)
-    layer += (size_t)rows_in_range(s, st, ranges[st][cta].x, ranges[st][cta].y) * stage_k(s, st) * 2;
+    layer += (size_t)rows_in_range(s, st, ranges[st][cta].x, ranges[st][cta].y) * stage_k(s, st) *
+             elem_bytes;
   const size_t lm =
-      (size_t)rows_in_range(s, ST_LM, ranges[ST_LM][cta].x, ranges[ST_LM][cta].y) * s.d * 2;
+      (size_t)rows_in_range(s, ST_LM, ranges[ST_LM][cta].x, ranges[ST_LM][cta].y) * s.d * elem_bytes;
   return (size_t)s.L * layer + lm;
+}
+
+size_t stream_rows(const Shape& s, const std::vector<std::vector<int2>>& ranges, int cta) {
+  size_t layer = 0;
+  for (int st = ST_QKV; st <= ST_DOWN; ++st)
+    layer += (size_t)rows_in_range(s, st, ranges[st][cta].x, ranges[st][cta].y);
+  return (size_t)s.L * layer +
+         (size_t)rows_in_range(s, ST_LM, ranges[ST_LM][cta].x, ranges[ST_LM][cta].y);
 }
 
 }  // namespace kie

@@ -38,7 +38,12 @@ int attn_smem_bytes(int G, int hd);
 bool plan_smem(const Shape& s, int grid, int chunk_bytes, int smem_limit,
                const std::vector<std::vector<int2>>& ranges, SmemLayout* out, int* ring_bytes);
 
-// Bytes of CTA `cta`'s one-token weight stream (all layers + LM head).
-size_t stream_bytes(const Shape& s, const std::vector<std::vector<int2>>& ranges, int cta);
+// Bytes of CTA `cta`'s one-token weight stream (all layers + LM head) with
+// `elem_bytes` bytes per weight (2: fp16, 1: fp8).
+size_t stream_bytes(const Shape& s, const std::vector<std::vector<int2>>& ranges, int cta,
+                    int elem_bytes = 2);
+// Rows of CTA `cta`'s one-token stream (all layers + LM head): the number of
+// row scales of an fp8 stream.
+size_t stream_rows(const Shape& s, const std::vector<std::vector<int2>>& ranges, int cta);
 
 }  // namespace kie
