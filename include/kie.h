@@ -46,7 +46,8 @@
  *     is one contiguous bulk copy; after kie_create the library reads only
  *     tok_emb and the norm gains from the caller (these must stay valid and
  *     unmodified until kie_destroy), and the caller's matrices are read
- *     again only by KIE_OPT_CHUNK_BYTES.  The KV cache must stay valid until
+ *     again by the batched prefill (KIE_OPT_BATCHED_PREFILL, on by default
+ *     for fp16 streams), KIE_OPT_CHUNK_BYTES and KIE_OPT_WEIGHT_FP8.  The KV cache must stay valid until
  *     kie_destroy.  The library owns the packed copy and its scratch
  *     (activation words, attention partials, the RoPE table, id buffers),
  *     allocated in kie_create and freed in kie_destroy.
@@ -140,6 +141,8 @@ typedef struct {
   double stream_wait_cycles;
   double producer_wait_cycles; /* producer cycles waiting for a free ring slot */
   double sync_wait_max_frac;   /* max over CTAs of sync_wait/loop */
+  double last_prefill_ms;      /* device time of the last kie_prefill (CUDA events) */
+  int32_t last_prefill_batched; /* 1: it ran the batched tensor-core path */
 } kie_stats;
 
 typedef enum {
@@ -158,7 +161,7 @@ typedef enum {
   KIE_OPT_L2_PREFETCH_BYTES = 10, /* per CTA, weight-stream bytes requested into L2 ahead of
                                     the shared-memory ring (multiple of 512, <= 16 MiB;
                                     0 = off, the default) */
-  KIE_OPT_WEIGHT_FP8 = 11      /* 1: stream the weight matrices as FP8 E4M3 with one fp32
+  KIE_OPT_WEIGHT_FP8 = 11,     /* 1: stream the weight matrices as FP8 E4M3 with one fp32
                                   scale per row (the pages' roadmap FP8 quantisation,
                                   revietech.ru, "Kog выжимает максимум из GPU: 3000
                                   токенов/с", section "Ограничения подхода"): half the
@@ -172,6 +175,15 @@ typedef enum {
                                   cache and everything else stay as they are.  0: fp16
                                   weights (the default).  Rebuilds the packed weight copy
                                   from the caller's matrices, which must still be valid */
+  KIE_OPT_BATCHED_PREFILL = 12  /* 1 (default): kie_prefill runs positions 0 .. n-2 of the
+                                  prompt through all layers at once -- the projections
+                                  as tcgen05 tensor-core GEMMs over the positions, causal
+                                  attention over the prompt, the K/V of every position
+                                  written to the cache -- and the last position as one
+                                  step of the decode kernel, which picks the first id.
+                                  It reads the caller's fp16 weight matrices, which must
+                                  then stay valid; contexts streaming FP8 weights, and
+                                  0, run every position as a decode step instead */
 } kie_option;
 
 /* Bytes of the caller-provided KV cache: 2*n_layers*n_kv_heads*max_seq*(head_dim+8)*2.

@@ -85,7 +85,10 @@ class Session:
 
     def release_matrices(self) -> None:
         """Drops this session's references to the weight matrices (kept:
-        the embedding and the norm gains, which the kernel still reads)."""
+        the embedding and the norm gains, which the kernel still reads).
+        The batched prefill reads the matrices, so prefill then runs every
+        position as a decode step."""
+        kie_set_option(self.ctx, _kie.KIE_OPT_BATCHED_PREFILL, 0)
         self.weights = {k: v for k, v in self.weights.items()
                         if k in self._KEPT or k.endswith("norm")}
         self._matrices_released = True
@@ -129,8 +132,9 @@ class Session:
         self._trace = None
 
     def set_option(self, opt: int, value: int) -> None:
-        if (opt in (_kie.KIE_OPT_CHUNK_BYTES, _kie.KIE_OPT_WEIGHT_FP8)
-                and getattr(self, "_matrices_released", False)):
+        rereads = opt in (_kie.KIE_OPT_CHUNK_BYTES, _kie.KIE_OPT_WEIGHT_FP8) or (
+            opt == _kie.KIE_OPT_BATCHED_PREFILL and value)
+        if rereads and getattr(self, "_matrices_released", False):
             raise ValueError("this option re-reads the weight matrices, which this session "
                              "has released (keep_matrices=False)")
         kie_set_option(self.ctx, opt, value)

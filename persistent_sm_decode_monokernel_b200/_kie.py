@@ -43,6 +43,7 @@ KIE_OPT_POLL_BACKOFF_NS = 8
 KIE_OPT_TRACE_CLOCK = 9
 KIE_OPT_L2_PREFETCH_BYTES = 10
 KIE_OPT_WEIGHT_FP8 = 11
+KIE_OPT_BATCHED_PREFILL = 12
 
 STAGE_QKV, STAGE_O, STAGE_GU, STAGE_DOWN, STAGE_LM = range(5)
 
@@ -73,7 +74,8 @@ class KieStats(ctypes.Structure):
                 ("last_device_ms", ctypes.c_float), ("launches", ctypes.c_uint64),
                 ("loop_cycles", ctypes.c_double), ("sync_wait_cycles", ctypes.c_double),
                 ("stream_wait_cycles", ctypes.c_double), ("producer_wait_cycles", ctypes.c_double),
-                ("sync_wait_max_frac", ctypes.c_double)]
+                ("sync_wait_max_frac", ctypes.c_double), ("last_prefill_ms", ctypes.c_double),
+                ("last_prefill_batched", ctypes.c_int32)]
 
 
 _P = ctypes.c_void_p

@@ -18,8 +18,8 @@ CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(HERE, "libkie.so")
 
-SOURCES = ["kie_host.cu", "kie_kernel.cu", "kie_plan.cpp", "kie_noalloc.cu"]
-HEADERS = ["kie_params.h", "kie_plan.h", "kie_kernel.h", "kie_device.cuh"]
+SOURCES = ["kie_host.cu", "kie_kernel.cu", "kie_plan.cpp", "kie_noalloc.cu", "kie_prefill.cu"]
+HEADERS = ["kie_params.h", "kie_plan.h", "kie_kernel.h", "kie_device.cuh", "kie_prefill.h"]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",

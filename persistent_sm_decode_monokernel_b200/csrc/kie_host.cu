@@ -1,6 +1,7 @@
 // Host side of the C ABI declared in include/kie.h: validation, planning,
 // scratch ownership, launches of the persistent decode kernel and session
 // state (position, fed ids).
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <algorithm>
@@ -15,6 +16,7 @@
 #include "kie_kernel.h"
 #include "kie_params.h"
 #include "kie_plan.h"
+#include "kie_prefill.h"
 
 using kie::DevStatus;
 using kie::LayerW;
@@ -53,6 +55,15 @@ struct kie_ctx {
   unsigned long long* packed_off = nullptr;   // [grid]
   size_t packed_bytes = 0;
   int w8 = 0;                                 // packed stream: 0 fp16, 1 fp8 E4M3 + row scales
+  // batched prefill (tensor-core GEMMs over the prompt) and its scratch,
+  // grown to the longest prompt seen
+  int batched_prefill = 1;
+  int pf_cap = 0;
+  int* pf_ids = nullptr;
+  float *pf_x = nullptr, *pf_qkv = nullptr, *pf_gu = nullptr;
+  __half *pf_a = nullptr, *pf_q = nullptr;
+  int* pf_err = nullptr;
+  cudaEvent_t pf_ev0 = nullptr, pf_ev1 = nullptr;
   float* wscale = nullptr;                    // fp8: row scales, each CTA's in stream order
   unsigned long long* wscale_off = nullptr;   // fp8: [grid] offsets (floats) into wscale
   kie::SmemLayout sm{};
@@ -133,6 +144,15 @@ void free_all(kie_ctx* c) {
   cudaFree(c->packed_off);
   cudaFree(c->wscale);
   cudaFree(c->wscale_off);
+  cudaFree(c->pf_ids);
+  cudaFree(c->pf_x);
+  cudaFree(c->pf_qkv);
+  cudaFree(c->pf_gu);
+  cudaFree(c->pf_a);
+  cudaFree(c->pf_q);
+  cudaFree(c->pf_err);
+  if (c->pf_ev0) cudaEventDestroy(c->pf_ev0);
+  if (c->pf_ev1) cudaEventDestroy(c->pf_ev1);
   if (c->h_io) cudaFreeHost(c->h_io);
   if (c->ev0) cudaEventDestroy(c->ev0);
   if (c->ev1) cudaEventDestroy(c->ev1);
@@ -304,6 +324,115 @@ kie_status repack(kie_ctx* c) {
   p.wscale_off = c->wscale_off;
   KIE_CUDA(c, kie::repack_launch(p, c->packed, c->stream));
   KIE_CUDA(c, cudaStreamSynchronize(c->stream));
+  return KIE_OK;
+}
+
+// ------------------------------------------------------- batched prefill
+
+using TmapEncodeFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+// The driver's tensor-map encoder, resolved through the runtime (the library
+// links no driver library); null if the driver does not offer it.
+TmapEncodeFn tmap_encoder() {
+  static const TmapEncodeFn fn = []() -> TmapEncodeFn {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q{};
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return nullptr;
+    return reinterpret_cast<TmapEncodeFn>(f);
+  }();
+  return fn;
+}
+
+// Tensor map of an fp16 row-major matrix [rows][cols] (cols a multiple of
+// 64, base 16-byte aligned): boxes of 64 columns x 128 rows, 128-byte
+// swizzle, rows past the end read as zeros.
+bool make_map(CUtensorMap* m, const void* base, int rows, int cols) {
+  const TmapEncodeFn enc = tmap_encoder();
+  if (!enc) return false;
+  const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
+  const cuuint32_t box[2] = {64, 128};
+  const cuuint32_t es[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool batched_prefill_possible(const kie_ctx* c, int n) {
+  return c->batched_prefill && !c->w8 && n >= 2 && tmap_encoder() != nullptr;
+}
+
+// Positions 0 .. T-1 of `ids` through every layer at once: K and V of each
+// position written to the cache (the decode kernel's layout), nothing else
+// kept.  Per layer: RMSNorm, Q / K / V GEMMs, RoPE + cache writes, causal
+// attention, O GEMM added to the residual, RMSNorm, gate and up GEMMs,
+// SwiGLU, down GEMM added to the residual.
+kie_status batched_prefill(kie_ctx* c, const int32_t* ids, int T) {
+  const kie_model_desc& d = c->desc;
+  const int D = d.d_model, F = d.ffn_dim, H = d.n_heads, KV = d.n_kv_heads, hd = d.head_dim;
+  const int nq = H * hd, nkv = KV * hd, nqkv = nq + 2 * nkv;
+  cudaStream_t st = c->stream;
+  if (T > c->pf_cap) {
+    cudaFree(c->pf_ids);
+    cudaFree(c->pf_x);
+    cudaFree(c->pf_qkv);
+    cudaFree(c->pf_gu);
+    cudaFree(c->pf_a);
+    cudaFree(c->pf_q);
+    c->pf_ids = nullptr;
+    c->pf_x = c->pf_qkv = c->pf_gu = nullptr;
+    c->pf_a = c->pf_q = nullptr;
+    c->pf_cap = 0;
+    const size_t wide = (size_t)std::max(std::max(D, F), nq);
+    KIE_CUDA(c, cudaMalloc(&c->pf_ids, sizeof(int) * T));
+    KIE_CUDA(c, cudaMalloc(&c->pf_x, sizeof(float) * T * (size_t)D));
+    KIE_CUDA(c, cudaMalloc(&c->pf_qkv, sizeof(float) * T * (size_t)nqkv));
+    KIE_CUDA(c, cudaMalloc(&c->pf_gu, sizeof(float) * T * 2 * (size_t)F));
+    KIE_CUDA(c, cudaMalloc(&c->pf_a, sizeof(__half) * T * wide));
+    KIE_CUDA(c, cudaMalloc(&c->pf_q, sizeof(__half) * T * (size_t)nq));
+    if (!c->pf_err) KIE_CUDA(c, cudaMalloc(&c->pf_err, sizeof(int)));
+    KIE_CUDA(c, kie::pf::gemm_configure());
+    c->pf_cap = T;
+  }
+  CUtensorMap a_d, a_nq, a_f;   // views of the fp16 activation buffer
+  if (!make_map(&a_d, c->pf_a, T, D) || !make_map(&a_nq, c->pf_a, T, nq) ||
+      !make_map(&a_f, c->pf_a, T, F))
+    return set_err(c, KIE_ERR_CUDA, "tensor map of the prefill activations");
+  KIE_CUDA(c, cudaMemcpyAsync(c->pf_ids, ids, sizeof(int) * T, cudaMemcpyHostToDevice, st));
+  KIE_CUDA(c, cudaMemsetAsync(c->pf_err, 0, sizeof(int), st));
+  KIE_CUDA(c, kie::pf::embed_rows(c->pf_ids, c->tok_emb, T, D, c->pf_x, st));
+  for (int l = 0; l < d.n_layers; ++l) {
+    const LayerW& w = c->hlayers[l];
+    CUtensorMap bq, bk, bv, bo, bg, bu, bd;
+    if (!make_map(&bq, w.wq, nq, D) || !make_map(&bk, w.wk, nkv, D) || !make_map(&bv, w.wv, nkv, D) ||
+        !make_map(&bo, w.wo, D, nq) || !make_map(&bg, w.wg, F, D) || !make_map(&bu, w.wu, F, D) ||
+        !make_map(&bd, w.wd, D, F))
+      return set_err(c, KIE_ERR_CUDA, "tensor map of a weight matrix");
+    KIE_CUDA(c, kie::pf::rmsnorm_rows(c->pf_x, w.attn_norm, T, D, d.rms_eps, c->pf_a, st));
+    KIE_CUDA(c, kie::pf::gemm_tn(a_d, bq, T, nq, D, c->pf_qkv, nqkv, 0, c->pf_err, st));
+    KIE_CUDA(c, kie::pf::gemm_tn(a_d, bk, T, nkv, D, c->pf_qkv + nq, nqkv, 0, c->pf_err, st));
+    KIE_CUDA(c, kie::pf::gemm_tn(a_d, bv, T, nkv, D, c->pf_qkv + nq + nkv, nqkv, 0, c->pf_err, st));
+    KIE_CUDA(c, kie::pf::rope_kv(c->pf_qkv, c->rope, T, H, KV, hd, d.max_seq, l, c->kv, c->pf_q, st));
+    KIE_CUDA(c, kie::pf::attention(c->pf_q, c->kv, T, H, KV, hd, d.max_seq, l, c->pf_a, st));
+    KIE_CUDA(c, kie::pf::gemm_tn(a_nq, bo, T, D, nq, c->pf_x, D, 1, c->pf_err, st));
+    KIE_CUDA(c, kie::pf::rmsnorm_rows(c->pf_x, w.ffn_norm, T, D, d.rms_eps, c->pf_a, st));
+    KIE_CUDA(c, kie::pf::gemm_tn(a_d, bg, T, F, D, c->pf_gu, 2 * F, 0, c->pf_err, st));
+    KIE_CUDA(c, kie::pf::gemm_tn(a_d, bu, T, F, D, c->pf_gu + F, 2 * F, 0, c->pf_err, st));
+    KIE_CUDA(c, kie::pf::swiglu(c->pf_gu, T, F, c->pf_a, st));
+    KIE_CUDA(c, kie::pf::gemm_tn(a_f, bd, T, D, F, c->pf_x, D, 1, c->pf_err, st));
+  }
+  int err = 0;
+  KIE_CUDA(c, cudaMemcpyAsync(&err, c->pf_err, sizeof(int), cudaMemcpyDeviceToHost, st));
+  KIE_CUDA(c, cudaStreamSynchronize(st));
+  if (err != 0) {
+    c->failed = true;
+    return set_err(c, KIE_ERR_TIMEOUT, "a bounded wait of the prefill GEMM gave up");
+  }
   return KIE_OK;
 }
 
@@ -498,9 +627,32 @@ kie_status kie_prefill(kie_ctx* c, const int32_t* ids, int32_t n, int32_t* first
         return set_err(c, KIE_ERR_INVALID_ARG, "prompt id out of range");
     c->primed = false;
     int done = 0;
-    s = launch(c, n, 0, ids, true, 0, n - 1, &done);
-    if (s != KIE_OK) return s;
-    const int32_t g0 = reinterpret_cast<const int32_t*>(c->h_io + kStatusBytes)[n - 1];
+    if (!c->pf_ev0) {
+      KIE_CUDA(c, cudaEventCreate(&c->pf_ev0));
+      KIE_CUDA(c, cudaEventCreate(&c->pf_ev1));
+    }
+    KIE_CUDA(c, cudaEventRecord(c->pf_ev0, c->stream));
+    const bool batched = batched_prefill_possible(c, n);
+    int32_t g0 = 0;
+    if (batched) {
+      // positions 0 .. n-2 at once, then the last one as a decode step that
+      // picks the first id
+      s = batched_prefill(c, ids, n - 1);
+      if (s != KIE_OK) return s;
+      s = launch(c, 1, n - 1, ids + n - 1, true, 0, 0, &done);
+      if (s != KIE_OK) return s;
+      g0 = reinterpret_cast<const int32_t*>(c->h_io + kStatusBytes)[0];
+    } else {
+      s = launch(c, n, 0, ids, true, 0, n - 1, &done);
+      if (s != KIE_OK) return s;
+      g0 = reinterpret_cast<const int32_t*>(c->h_io + kStatusBytes)[n - 1];
+    }
+    KIE_CUDA(c, cudaEventRecord(c->pf_ev1, c->stream));
+    KIE_CUDA(c, cudaEventSynchronize(c->pf_ev1));
+    float pms = 0.f;
+    cudaEventElapsedTime(&pms, c->pf_ev0, c->pf_ev1);
+    c->stats.last_prefill_ms = pms;
+    c->stats.last_prefill_batched = batched ? 1 : 0;
     c->fed.assign(ids, ids + n);
     c->pos = n;
     c->next_tok = g0;
@@ -818,6 +970,10 @@ kie_status kie_set_option(kie_ctx* c, kie_option opt, int64_t v) {
       case KIE_OPT_POLL_BACKOFF_NS:
         if (v < 0 || v > 100000) return KIE_ERR_INVALID_ARG;
         c->poll_ns = (unsigned)v;
+        return KIE_OK;
+      case KIE_OPT_BATCHED_PREFILL:
+        if (v != 0 && v != 1) return KIE_ERR_INVALID_ARG;
+        c->batched_prefill = (int)v;
         return KIE_OK;
       case KIE_OPT_WEIGHT_FP8: {
         if (c->failed) return set_err(c, KIE_ERR_STATE, "context failed earlier; destroy it");
