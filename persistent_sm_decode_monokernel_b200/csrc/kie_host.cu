@@ -318,6 +318,7 @@ kie_status repack(kie_ctx* c) {
   p.ranges = c->ranges;
   p.grid = c->grid;
   p.chunk_bytes = c->chunk_bytes;
+  p.sm = c->sm;   // the unit plan reads the result-slot count
   p.packed_off = c->packed_off;
   p.w8 = c->w8;
   p.wscale = c->wscale;
@@ -819,16 +820,18 @@ kie_status kie_gemv_f16(const void* W, const float* x, float* y, int32_t N, int3
     }
     kie::SmemLayout L{};
     L.xs_bytes = (K * 4 + 127) / 128 * 128;
-    L.rowacc_rows = maxrows;
+    L.rowacc_rows = kie::result_slots(maxrows, K / kie::kPieceElems, chunk_bytes);
     L.resid_rows = 0;
-    const int fixed = 256 + L.xs_bytes + (maxrows * 4 + 127) / 128 * 128 + kie::kEngineMisc;
+    const int rowacc_bytes = (L.rowacc_rows * 4 + 127) / 128 * 128;
+    const int bars = 2 * kie::kRingBars * 8;
+    const int fixed = bars + L.xs_bytes + rowacc_bytes + kie::kEngineMisc;
     const int ring = (smem_optin - fixed) / 512 * 512;
     if (ring < 2 * chunk_bytes) return KIE_ERR_UNSUPPORTED;
     L.ring_off = 0;
     L.bar_off = ring;
-    L.xs_off = L.bar_off + 256;
+    L.xs_off = L.bar_off + bars;
     L.rowacc_off = L.xs_off + L.xs_bytes;
-    L.misc_off = L.rowacc_off + (maxrows * 4 + 127) / 128 * 128;
+    L.misc_off = L.rowacc_off + rowacc_bytes;
     L.total = L.misc_off + kie::kEngineMisc;
 
     int2* d_ranges = nullptr;

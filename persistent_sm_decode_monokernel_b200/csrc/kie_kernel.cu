@@ -75,7 +75,7 @@ __shared__ uint32_t kie_cur[3];
 // only: exact for thread 0 (the stage trace), and for the other threads the
 // position an error report names (possibly one stage behind).
 __shared__ int kie_at[3];
-// This CTA's row scales of an fp8 weight stream (set by make_plans).
+// This CTA's row scales of an fp8 weight stream (set by setup_plans).
 __shared__ const float* kie_wsc;
 
 // Views of the dynamic shared memory, always derived from the __shared__
@@ -114,19 +114,27 @@ __device__ __forceinline__ float* sm_res_ffn(const MonoParams& p) {
   return sm_misc(p) + kMiscHead + p.sm.resid_rows;
 }
 
-// This CTA's GEMV work in one stage, computed once per launch: kGroupRows
-// row groups and the k-chunking of a full group and of the last group.
+// This CTA's GEMV work in one stage, computed once per launch (plan_units).
+// The rows are cut into blocks of nr rows (the last block may be shorter)
+// and the kp pieces of a block's rows into S parts (part s: count(s)
+// pieces from piece first(s)).  Unit u = (block u / S, part u % S) is one
+// ring chunk, stored [row][piece][piece bytes], and warp u % kConsumerWarps
+// alone computes it.  With S > 1 a row's S partial sums go to S result
+// slots, which row_result adds in part order.
 struct StagePlan {
-  int rows, kp;          // rows of the CTA in the stage, 512-byte pieces per row
-  int nfull, tail;       // full groups; rows of the last, partial group (0: none)
-  int f_nk, f_base, f_rem;  // chunking of a full group (see Chunking)
-  int t_nk, t_base, t_rem;  // chunking of the partial group
-  int t_lw;              // partial group of <= kConsumerWarps rows: log2 warps per row
+  int rows, kp;          // rows of the CTA in the stage, pieces per row
+  int nr, S;             // rows per block, parts per row
+  int base, rem;         // part s has base + (s < rem ? 1 : 0) pieces
+  int nb;                // blocks: ceil(rows / nr)
   // fp8 streams: index of the stage's first row scale among the CTA's scales
   // of one layer (LM head: of the whole stream), and the scales of a layer
   int sbase, rows_layer;
-  int pad[3];
+  int pad[7];
+  __device__ __forceinline__ int first(int s) const { return s * base + min(s, rem); }
+  __device__ __forceinline__ int count(int s) const { return base + (s < rem ? 1 : 0); }
+  __device__ __forceinline__ int block_rows(int b) const { return min(nr, rows - b * nr); }
 };
+static_assert(sizeof(StagePlan) == 64, "stage plan slot");
 __device__ __forceinline__ StagePlan* sm_plan(const MonoParams& p) {
   return reinterpret_cast<StagePlan*>(sm_misc(p) + kMiscHead + 2 * p.sm.resid_rows);
 }
@@ -206,49 +214,85 @@ __device__ __forceinline__ const __half* row_ptr(const MonoParams& p, int st, co
   }
 }
 
-// k-chunking of one group of rg (<= kGroupRows) rows with kp pieces per row into nk
-// chunks of at most chunk_bytes: chunk kc holds count(kc) pieces of every
-// row of the group, starting at piece first(kc).  Stored [row][piece][512 B].
-struct Chunking {
-  int nk, base, rem;
-  __device__ __forceinline__ int first(int kc) const { return kc * base + min(kc, rem); }
-  __device__ __forceinline__ int count(int kc) const { return base + (kc < rem ? 1 : 0); }
-};
-__device__ __forceinline__ Chunking chunking(int rg, int kp, int chunk_bytes, int pb) {
-  int mp = chunk_bytes / (rg * pb);
-  if (mp < 1) mp = 1;
-  Chunking c;
-  c.nk = (kp + mp - 1) / mp;
-  c.base = kp / c.nk;
-  c.rem = kp - c.base * c.nk;
-  return c;
+// Unit shape of a stage plan's rows x kp pieces: the (rows per block,
+// parts) pair with the least estimated time of the busiest warp among those
+// whose units fit a chunk of chunk_bytes and whose partial sums fit `slots`
+// result words.  A warp runs its units one after another; a unit costs
+// (rows x pieces) piece-rows of weights, 0.3 piece-rows per piece for the
+// activation load its rows share and 6 for its wait, release and row
+// reductions.  Units of one row and one piece always fit (the host keeps
+// chunk_bytes >= pb and slots >= rows x ceil(kp / (chunk_bytes / pb))).
+__device__ __forceinline__ void plan_units(StagePlan& pl, int chunk_bytes, int pb, int slots) {
+  const int R = pl.rows, kp = pl.kp, m = chunk_bytes / pb;
+  int best = 0x7fffffff;
+  pl.nr = 1;
+  pl.S = (kp + m - 1) / m;
+  for (int nr = 1; nr <= 4 && (nr == 1 || nr <= R); ++nr) {
+    const int nb = (R + nr - 1) / nr;
+    for (int S = 1; S <= min(kp, 16); ++S) {
+      const int nmax = (kp + S - 1) / S;
+      if (nr * nmax > m) continue;
+      if (S > 1 && R * S > slots) break;
+      const int per_warp = (nb * S + kConsumerWarps - 1) / kConsumerWarps;
+      const int cost = per_warp * (10 * nr * nmax + 3 * nmax + 60);
+      if (cost < best) {
+        best = cost;
+        pl.nr = nr;
+        pl.S = S;
+      }
+    }
+  }
+  pl.base = kp / pl.S;
+  pl.rem = kp - pl.base * pl.S;
+  pl.nb = (R + pl.nr - 1) / pl.nr;
 }
 
-// The stream order of a stage's chunks (shared by the weight repack, the
-// producer and the consumers): full row groups in pairs whose k-chunks
-// interleave (A0, B0, A1, B1, ...) so that a consumer warp works on the
-// rows of both groups at once, then a leftover full group, then the last,
-// partial group.  f(g0, rg, n, p0) receives each chunk's first row (within
-// the CTA's rows), its row count, its piece count and its first piece;
-// returning false stops the walk.
+// The rows and unit shape of CTA blockIdx.x's share of stage st.
+__device__ __forceinline__ StagePlan stage_plan(const MonoParams& p, int st) {
+  const int2 r = p.ranges[st * p.grid + blockIdx.x];
+  StagePlan pl{};
+  pl.rows = range_rows(p, st, r.x, r.y);
+  pl.kp = stage_k(p, st) / kPieceElems;
+  plan_units(pl, p.chunk_bytes, piece_bytes(p.w8), p.sm.rowacc_rows);
+  return pl;
+}
+
+// The stream order of a stage's units (shared by the weight repack, the
+// producer and the consumers): f(u, b, s, rows, n) receives each unit's
+// index, block, part, row count and piece count; returning false stops the
+// walk.
 template <class F>
-__device__ __forceinline__ bool for_each_chunk(int R, int kp, int chunk_bytes, int pb, F&& f) {
-  const int nfull = R / kGroupRows, tail = R - nfull * kGroupRows;
-  const Chunking cf = chunking(kGroupRows, kp, chunk_bytes, pb);
-  int g = 0;
-  for (; g + 1 < nfull; g += 2)
-    for (int kc = 0; kc < cf.nk; ++kc)
-      for (int h = 0; h < 2; ++h)
-        if (!f((g + h) * kGroupRows, kGroupRows, cf.count(kc), cf.first(kc))) return false;
-  if (g < nfull)
-    for (int kc = 0; kc < cf.nk; ++kc)
-      if (!f(g * kGroupRows, kGroupRows, cf.count(kc), cf.first(kc))) return false;
-  if (tail > 0) {
-    const Chunking ct = chunking(tail, kp, chunk_bytes, pb);
-    for (int kc = 0; kc < ct.nk; ++kc)
-      if (!f(nfull * kGroupRows, tail, ct.count(kc), ct.first(kc))) return false;
+__device__ __forceinline__ bool for_each_unit(const StagePlan& pl, F&& f) {
+  int u = 0;
+  for (int b = 0; b < pl.nb; ++b) {
+    const int rows = pl.block_rows(b);
+    for (int s = 0; s < pl.S; ++s, ++u)
+      if (!f(u, b, s, rows, pl.count(s))) return false;
   }
   return true;
+}
+
+// Fills the stage plans in shared memory (threads 0..N_STAGES-1; the caller
+// synchronises) and thread 0 the fp8 row-scale pointer.
+__device__ __forceinline__ void setup_plans(const MonoParams& p) {
+  const int tid = (int)threadIdx.x;
+  if (tid < N_STAGES) {
+    const int st = tid;
+    StagePlan pl = stage_plan(p, st);
+    // row-scale positions of an fp8 stream (per layer: QKV, O, gate/up,
+    // down rows; then the LM head after all layers)
+    int before = 0, layer_rows = 0;
+    for (int s2 = ST_QKV; s2 <= ST_DOWN; ++s2) {
+      const int2 r2 = p.ranges[s2 * p.grid + blockIdx.x];
+      const int n2 = range_rows(p, s2, r2.x, r2.y);
+      if (s2 < st) before += n2;
+      layer_rows += n2;
+    }
+    pl.rows_layer = layer_rows;
+    pl.sbase = st == ST_LM ? p.L * layer_rows : before;
+    sm_plan(p)[st] = pl;
+  }
+  if (tid == 0) kie_wsc = p.w8 ? p.wscale + p.wscale_off[blockIdx.x] : nullptr;
 }
 
 // Byte ring placement shared by producer and consumers: a chunk goes right
@@ -345,7 +389,7 @@ struct Producer {
 
   __device__ long long stage_len(int st) const {
     const int2 r = p.ranges[st * p.grid + blockIdx.x];
-    return (long long)range_rows(p, st, r.x, r.y) * stage_k(p, st) * 2;
+    return (long long)range_rows(p, st, r.x, r.y) * stage_k(p, st) * piece_bytes(p.w8) / kPieceElems;
   }
 
   // Tops the prefetch up to `next` + p.l2_prefetch bytes beyond the copy cursor.
@@ -465,34 +509,24 @@ struct Producer {
     }
   }
 
-  // The stage's chunks in stream order (for_each_chunk's order; only their
-  // sizes matter here): full-group pairs (the two groups' chunks alternate
-  // per k-chunk), a leftover full group, the partial group.  One loop nest
-  // with a single issue site keeps the producer's code small: it shares the
-  // SM's instruction cache with the consumer warps.
+  // The stage's units in stream order, one chunk each (the plan is in
+  // shared memory from the kernel's start).  One loop with a single issue
+  // site keeps the producer's code small: it shares the SM's instruction
+  // cache with the consumer warps.
   __device__ bool stage(int st, const unsigned char*& src) {
-    const int2 r = p.ranges[st * p.grid + blockIdx.x];
-    const int R = range_rows(p, st, r.x, r.y);
-    const int kp = stage_k(p, st) / kPieceElems;
-    const int nfull = R / kGroupRows, tail = R - nfull * kGroupRows;
+    const StagePlan& pl = sm_plan(p)[st];
     const int pb = piece_bytes(p.w8);
-    const Chunking cf = chunking(kGroupRows, kp, p.chunk_bytes, pb);
-    const Chunking ct = chunking(tail > 0 ? tail : 1, kp, p.chunk_bytes, pb);
+    const int nb = pl.nb, S = pl.S;
 #pragma unroll 1
-    for (int sg = 0; sg < 3; ++sg) {
-      const int reps = sg == 0 ? nfull / 2 : (sg == 1 ? (nfull & 1) : (tail > 0 ? 1 : 0));
-      const int rows = sg < 2 ? kGroupRows : tail;
-      const int mult = sg == 0 ? 2 : 1;
-      const Chunking c = sg < 2 ? cf : ct;
+    for (int b = 0; b < nb; ++b) {
+      const int rows = pl.block_rows(b);
 #pragma unroll 1
-      for (int rep = 0; rep < reps; ++rep)
-#pragma unroll 1
-        for (int j = 0; j < c.nk * mult; ++j) {
-          const uint32_t sz = (uint32_t)(rows * c.count(j / mult) * pb);
-          if (p.l2_prefetch > 0) prefetch(sz);
-          if (!chunk(src, sz)) return false;
-          pf_ahead -= sz;
-        }
+      for (int s = 0; s < S; ++s) {
+        const uint32_t sz = (uint32_t)(rows * pl.count(s) * pb);
+        if (p.l2_prefetch > 0) prefetch(sz);
+        if (!chunk(src, sz)) return false;
+        pf_ahead -= sz;
+      }
     }
     return true;
   }
@@ -633,31 +667,32 @@ __device__ __forceinline__ uint4 quantize16(const uint4& a, const uint4& b, floa
 }
 
 // Lays out CTA blockIdx.x's one-token weight stream in the order Producer
-// streams it: per layer the QKV, O, gate/up and down chunks, then the LM
-// head, each chunk [row][piece][piece bytes].  fp16: a copy; fp8: every
+// streams it: per layer the QKV, O, gate/up and down units, then the LM
+// head, each unit [row][piece][piece bytes].  fp16: a copy; fp8: every
 // weight w of row r becomes the E4M3 code of w / s_r (fp32 division, round
 // to nearest even, saturated at +-448), s_r the row's scale (rowscale_stage).
 // Run once per model (and per change of the weight format or chunk size).
 __device__ void repack_stage(const MonoParams& p, int st, const LayerW& w, unsigned char*& dst,
                              const float* scales) {
   const int2 r = p.ranges[st * p.grid + blockIdx.x];
-  const int R = range_rows(p, st, r.x, r.y);
-  const int kp = stage_k(p, st) / kPieceElems;
   const int pb = piece_bytes(p.w8);
-  for_each_chunk(R, kp, p.chunk_bytes, pb, [&](int g0, int rg, int n, int p0) {
-    const int n16 = n * pb / 16;   // 16-byte units of a row's part of the chunk
+  const StagePlan pl = stage_plan(p, st);
+  for_each_unit(pl, [&](int, int b, int s, int rows, int n) {
+    const int n16 = n * pb / 16;   // 16-byte units of a row's part of the unit
+    const int p0 = pl.first(s);
     uint4* d = reinterpret_cast<uint4*>(dst);
-    for (int e = threadIdx.x; e < rg * n16; e += blockDim.x) {
+    for (int e = threadIdx.x; e < rows * n16; e += blockDim.x) {
       const int j = e / n16, q = e - j * n16;
-      const __half* row = row_ptr(p, st, w, r.x, r.y, g0 + j) + (size_t)p0 * kPieceElems;
+      const int k = b * pl.nr + j;
+      const __half* row = row_ptr(p, st, w, r.x, r.y, k) + (size_t)p0 * kPieceElems;
       if (!p.w8) {
         d[e] = reinterpret_cast<const uint4*>(row)[q];
       } else {   // 16 weights -> 16 codes
         d[e] = quantize16(reinterpret_cast<const uint4*>(row)[2 * q],
-                          reinterpret_cast<const uint4*>(row)[2 * q + 1], scales[g0 + j]);
+                          reinterpret_cast<const uint4*>(row)[2 * q + 1], scales[k]);
       }
     }
-    dst += (size_t)rg * n * pb;
+    dst += (size_t)rows * n * pb;
     return true;
   });
 }
@@ -993,238 +1028,130 @@ struct Consumer {
     return ((c[0] + c[1]) + (c[2] + c[3])) + ((c[4] + c[5]) + (c[6] + c[7]));
   }
 
-  // Fills the stage plans (threads 0..N_STAGES-1; the caller synchronises).
-  __device__ void make_plans() {
-    const MonoParams& p = kie_p;
-    const int tid = (int)threadIdx.x;
-    if (tid < N_STAGES) {
-      const int st = tid;
-      const int2 r = p.ranges[st * p.grid + blockIdx.x];
-      StagePlan pl{};
-      pl.rows = range_rows(p, st, r.x, r.y);
-      pl.kp = stage_k(p, st) / kPieceElems;
-      pl.nfull = pl.rows / kGroupRows;
-      pl.tail = pl.rows - pl.nfull * kGroupRows;
-      const Chunking f = chunking(kGroupRows, pl.kp, p.chunk_bytes, piece_bytes(p.w8));
-      pl.f_nk = f.nk;
-      pl.f_base = f.base;
-      pl.f_rem = f.rem;
-      if (pl.tail > 0) {
-        const Chunking t = chunking(pl.tail, pl.kp, p.chunk_bytes, piece_bytes(p.w8));
-        pl.t_nk = t.nk;
-        pl.t_base = t.base;
-        pl.t_rem = t.rem;
-        int lw = 0;
-        while ((pl.tail << (lw + 1)) <= kConsumerWarps) ++lw;
-        pl.t_lw = lw;
-      }
-      // row-scale positions of an fp8 stream (per layer: QKV, O, gate/up,
-      // down rows; then the LM head after all layers)
-      int before = 0, layer_rows = 0;
-      for (int s2 = ST_QKV; s2 <= ST_DOWN; ++s2) {
-        const int2 r2 = p.ranges[s2 * p.grid + blockIdx.x];
-        const int n2 = range_rows(p, s2, r2.x, r2.y);
-        if (s2 < st) before += n2;
-        layer_rows += n2;
-      }
-      pl.rows_layer = layer_rows;
-      pl.sbase = st == ST_LM ? p.L * layer_rows : before;
-      sm_plan(p)[st] = pl;
+  // Sums of NR rows' per-lane partial sums c[i][0..7] over the warp.  On
+  // return lane l holds the sum of row l / (32 / NR') (NR' = NR rounded up
+  // to a power of two; a fourth row of NR = 3 is zero): butterflies that
+  // hand half of the rows to the other half-warp first need 4 + log2 NR'
+  // exchanges for all rows instead of 5 per row.
+  template <int NR>
+  __device__ __forceinline__ static float reduce_rows(const float (&c)[NR][8], int lane) {
+    if constexpr (NR == 1) {
+      return dev::warp_sum(sum8(c[0]));
+    } else if constexpr (NR == 2) {
+      const bool up = (lane & 16) != 0;
+      const float a = sum8(c[0]), b = sum8(c[1]);
+      float t = (up ? b : a) + __shfl_xor_sync(0xffffffffu, up ? a : b, 16);
+#pragma unroll
+      for (int o = 8; o > 0; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
+      return t;
+    } else {
+      const float v0 = sum8(c[0]), v1 = sum8(c[1]), v2 = sum8(c[2]);
+      float v3 = 0.f;
+      if constexpr (NR == 4) v3 = sum8(c[3]);
+      // lanes 16-31 keep rows 2 and 3, lanes 0-15 rows 0 and 1
+      const bool up = (lane & 16) != 0;
+      const float t0 = (up ? v2 : v0) + __shfl_xor_sync(0xffffffffu, up ? v0 : v2, 16);
+      const float t1 = (up ? v3 : v1) + __shfl_xor_sync(0xffffffffu, up ? v1 : v3, 16);
+      // lanes with bit 3 set keep the odd row of their pair
+      const bool mid = (lane & 8) != 0;
+      float t = (mid ? t1 : t0) + __shfl_xor_sync(0xffffffffu, mid ? t0 : t1, 8);
+#pragma unroll
+      for (int o = 4; o > 0; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
+      return t;
     }
-    if (tid == 0) kie_wsc = p.w8 ? p.wscale + p.wscale_off[blockIdx.x] : nullptr;
   }
 
-  // GEMV of this CTA's rows of stage st: dot products (times the rows'
-  // scales when the stream is fp8), read back with row_result.  A group of
-  // up to 16 rows streams as k-chunks.  In a group of more than 8 rows warp
-  // w owns rows w and w+8 for all of the group's chunks (one activation load
-  // serves two rows) and keeps its partial sums in registers.  A last group
-  // of at most 8 rows gives each row 8/rg (power of two) warps that split
-  // its pieces; their partial sums are added in a fixed order by
-  // row_result, so results do not depend on timing.  Ring positions and the
-  // parameter block are held in registers for the whole stage; one barrier
-  // at the end.  W8: pieces of fp8 E4M3 weights (8 bytes a lane), converted
-  // to fp16 pairs and multiplied like fp16 weights; rsc: the row scales of
-  // this CTA's rows of the stage (unused for fp16).
-  template <bool W8>
-  __device__ __noinline__ bool gemv(int st, const float* rsc) {
+  // This warp's units of a stage whose blocks have NR rows (see StagePlan):
+  // every warp walks all units in stream order to follow the ring placement
+  // and computes its own, unit u belonging to warp u % kConsumerWarps.  For
+  // a unit it waits for the chunk, multiplies the rows' pieces by the
+  // activation pieces (one activation load serves all rows of the unit),
+  // releases the chunk with one arrival worth all consumer warps, reduces
+  // the rows across the lanes and writes each row's sum (part s of the row
+  // when the rows are split in parts) times the row's scale.
+  template <bool W8, int NR>
+  __device__ __forceinline__ void gemv_units(const StagePlan& pl, const float* rsc, uint32_t& ci,
+                                             uint32_t& ce, bool& bad) {
     using WT = typename std::conditional<W8, uint2, uint4>::type;   // a lane's weights of a piece
     constexpr int PB = W8 ? kPieceElems : kPieceBytes;
+    constexpr int kLanesPerRow = NR == 1 ? 32 : (NR == 2 ? 16 : 8);
     const MonoParams& p = kie_p;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const StagePlan pl = sm_plan(p)[st];
     const unsigned char* ring = sm_ring(p);
     const uint4* xv = reinterpret_cast<const uint4*>(kie_smem + p.sm.xs_off) + lane;
     float* rowacc = sm_rowacc(p);
     const uint32_t ring_bytes = (uint32_t)p.ring_bytes;
     const uint32_t full_s = sm_full_s(p), empty_s = sm_empty_s(p);
-    uint32_t ci = kie_cur[0], cr = kie_cur[1], ce = kie_cur[2];
-    bool bad = false;
-    auto wait = [&](uint32_t sz, uint32_t& off) -> bool {
-      off = ring_place(ce, sz, ring_bytes);
-      const uint32_t bar = full_s + 8 * (ci & (kRingBars - 1));
-      const uint32_t par = (ci / kRingBars) & 1u;
-      ++ci;
-      if (dev::mbar_test_wait(bar, par)) return true;
-      return wait_slow(bar, par);
-    };
-    auto release = [&]() {
-      __syncwarp();
-      if (lane == 0) dev::mbar_arrive(empty_s + 8 * (cr & (kRingBars - 1)));
-      ++cr;
-    };
-    // scale of row k (1 for fp16); issued early, used when the row's sum is written
-    auto scale_of = [&](int k) -> float { return W8 ? __ldg(rsc + k) : 1.0f; };
-    // groups of more than kConsumerWarps rows / full groups: warp w owns
-    // rows w (and w + kConsumerWarps when two rows per warp; the second may
-    // be missing)
-    auto group2 = [&](int g0, int rg, int nk, int base, int rem) {
-      const bool two = kRowsPerWarp == 2 && warp + kConsumerWarps < rg;
-      const float s0 = scale_of(g0 + warp), s1 = two ? scale_of(g0 + warp + kConsumerWarps) : 1.f;
-      float c0[8], c1[8];
+    const int my_i = lane / kLanesPerRow;          // the unit row whose sum this lane writes
+    const bool writer = (lane & (kLanesPerRow - 1)) == 0;
+    const int S = pl.S;
+    int u = 0;
+#pragma unroll 1
+    for (int b = 0; b < pl.nb; ++b) {
+      const int rows = pl.block_rows(b);
+#pragma unroll 1
+      for (int s = 0; s < S; ++s, ++u) {
+        const int n = pl.count(s);
+        const uint32_t off = ring_place(ce, (uint32_t)(rows * n * PB), ring_bytes);
+        const uint32_t chunk = ci++;
+        if ((u & (kConsumerWarps - 1)) != warp) continue;
+        const int k = b * NR + my_i;
+        const bool mine = writer && my_i < rows;
+        const float sc = (W8 && mine) ? __ldg(rsc + k) : 1.f;
+        const uint32_t bar = full_s + 8 * (chunk & (kRingBars - 1));
+        const uint32_t par = (chunk / kRingBars) & 1u;
+        if (!dev::mbar_test_wait(bar, par) && !wait_slow(bar, par)) bad = true;
+        float c[NR][8];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) c0[i] = c1[i] = 0.f;
-      for (int kc = 0; kc < nk; ++kc) {
-        const int n = base + (kc < rem ? 1 : 0), p0 = kc * base + min(kc, rem);
-        uint32_t off;
-        if (!wait((uint32_t)(rg * n * PB), off)) bad = true;
+        for (int i = 0; i < NR; ++i)
+#pragma unroll
+          for (int j = 0; j < 8; ++j) c[i][j] = 0.f;
         if (!bad) {
-          const WT* w0 = reinterpret_cast<const WT*>(ring + off + (size_t)warp * n * PB) + lane;
-          const uint4* x = xv + (size_t)p0 * 32;
-          if (two) {
-            const WT* w1 = w0 + (size_t)kConsumerWarps * n * 32;
-#pragma unroll 4
-            for (int q = 0; q < n; ++q) {
-              const uint4 a = x[q * 32];
-              dot_piece(w0[q * 32], a, c0);
-              dot_piece(w1[q * 32], a, c1);
-            }
-          } else {
-#pragma unroll 4
-            for (int q = 0; q < n; ++q) dot_piece(w0[q * 32], x[q * 32], c0);
-          }
-        }
-        release();
-      }
-      if constexpr (kRowsPerWarp == 2) {
-        // both rows' sums with one butterfly: after the exchange across the
-        // half-warps, lanes 0-15 reduce row w and lanes 16-31 row w+8
-        const bool upper = (lane & 16) != 0;
-        const float a = sum8(c0), b = sum8(c1);
-        float t = (upper ? b : a) + __shfl_xor_sync(0xffffffffu, upper ? a : b, 16);
+          // rows past the end of a short last block read the block's last
+          // row again (their sums are not written), so that every load is
+          // unconditional
+          const WT* w[NR];
 #pragma unroll
-        for (int o = 8; o > 0; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
-        if (lane == 0) rowacc[g0 + warp] = t * s0;
-        if (two && lane == 16) rowacc[g0 + warp + kConsumerWarps] = t * s1;
-      } else {
-        const float t = dev::warp_sum(sum8(c0));
-        if (lane == 0) rowacc[g0 + warp] = t * s0;
-      }
-    };
-    // pairs of full groups (their chunks interleave in the stream): warp w
-    // owns its rows of both groups, one activation load per piece serves all
-    // of them
-    auto group_pair = [&](int g0) {
-      constexpr int RW = 2 * kRowsPerWarp;             // rows per warp
-      // the row this lane writes after the butterfly (lanes 0, 8, 16, 24)
-      const int my_row = (lane & 8 ? kGroupRows : 0) + (lane & 16 ? kConsumerWarps : 0) + warp;
-      const float s_me = (lane & 7) == 0 ? scale_of(g0 + (RW == 4 ? my_row : (lane & 16 ? kGroupRows : 0) + warp)) : 1.f;
-      float c[RW][8];
-#pragma unroll
-      for (int r = 0; r < RW; ++r)
-#pragma unroll
-        for (int i = 0; i < 8; ++i) c[r][i] = 0.f;
-      for (int kc = 0; kc < pl.f_nk; ++kc) {
-        const int n = pl.f_base + (kc < pl.f_rem ? 1 : 0), p0 = kc * pl.f_base + min(kc, pl.f_rem);
-        const uint32_t sz = (uint32_t)(kGroupRows * n * PB);
-        uint32_t offa, offb;
-        if (!wait(sz, offa)) bad = true;
-        if (!wait(sz, offb)) bad = true;
-        if (!bad) {
-          const uint4* x = xv + (size_t)p0 * 32;
-          const WT* wa = reinterpret_cast<const WT*>(ring + offa + (size_t)warp * n * PB) + lane;
-          const WT* wb = reinterpret_cast<const WT*>(ring + offb + (size_t)warp * n * PB) + lane;
-          const size_t second = (size_t)kConsumerWarps * n * 32;   // row w + kConsumerWarps
+          for (int i = 0; i < NR; ++i)
+            w[i] = reinterpret_cast<const WT*>(ring + off) + (size_t)min(i, rows - 1) * n * 32 + lane;
+          const uint4* x = xv + (size_t)pl.first(s) * 32;
 #pragma unroll 2
           for (int q = 0; q < n; ++q) {
-            const uint4 xa = x[q * 32];
-            dot_piece(wa[q * 32], xa, c[0]);
-            dot_piece(wb[q * 32], xa, c[1]);
-            if constexpr (kRowsPerWarp == 2) {
-              dot_piece(wa[second + q * 32], xa, c[2]);
-              dot_piece(wb[second + q * 32], xa, c[3]);
-            }
+            const uint4 a = x[q * 32];
+#pragma unroll
+            for (int i = 0; i < NR; ++i) dot_piece(w[i][q * 32], a, c[i]);
           }
         }
-        release();
-        release();
+        __syncwarp();
+        if (lane == 0) dev::mbar_arrive_n(empty_s + 8 * (chunk & (kRingBars - 1)), kConsumerWarps);
+        const float t = reduce_rows<NR>(c, lane);
+        if (mine) rowacc[S == 1 ? k : k * S + s] = t * sc;
       }
-      // butterfly over the warp's rows: after the exchanges each group of
-      // 32 / RW lanes holds one row's partial sums
-      float v[RW];
-#pragma unroll
-      for (int r = 0; r < RW; ++r) v[r] = sum8(c[r]);
-      if constexpr (RW == 4) {
-        // rows: 0 = A w, 1 = B w, 2 = A w+K, 3 = B w+K (K = kConsumerWarps)
-        const bool up = (lane & 16) != 0;
-        const float k0 = up ? v[2] : v[0], s0 = up ? v[0] : v[2];
-        const float k1 = up ? v[3] : v[1], s1 = up ? v[1] : v[3];
-        const float t0 = k0 + __shfl_xor_sync(0xffffffffu, s0, 16);
-        const float t1 = k1 + __shfl_xor_sync(0xffffffffu, s1, 16);
-        const bool mid = (lane & 8) != 0;
-        float u = (mid ? t1 : t0) + __shfl_xor_sync(0xffffffffu, mid ? t0 : t1, 8);
-#pragma unroll
-        for (int o = 4; o > 0; o >>= 1) u += __shfl_xor_sync(0xffffffffu, u, o);
-        // lane 0: A w, 8: B w, 16: A w+K, 24: B w+K
-        if ((lane & 7) == 0) rowacc[g0 + my_row] = u * s_me;
-      } else {
-        // rows: 0 = A w, 1 = B w
-        const bool up = (lane & 16) != 0;
-        float u = (up ? v[1] : v[0]) + __shfl_xor_sync(0xffffffffu, up ? v[0] : v[1], 16);
-#pragma unroll
-        for (int o = 8; o > 0; o >>= 1) u += __shfl_xor_sync(0xffffffffu, u, o);
-        if ((lane & 15) == 0) rowacc[g0 + (up ? kGroupRows : 0) + warp] = u * s_me;
-      }
-    };
-    int g = 0;
-    for (; g + 1 < pl.nfull; g += 2) group_pair(g * kGroupRows);
-    if (g < pl.nfull) group2(g * kGroupRows, kGroupRows, pl.f_nk, pl.f_base, pl.f_rem);
-    const int tb = pl.nfull * kGroupRows;
-    if (pl.tail > kConsumerWarps) {
-      group2(tb, pl.tail, pl.t_nk, pl.t_base, pl.t_rem);
-    } else if (pl.tail > 0) {
-      const int lw = pl.t_lw, rg = pl.tail;
-      const int r = warp >> lw, part = warp & ((1 << lw) - 1);
-      const bool active = r < rg;
-      const float s_r = active ? scale_of(tb + r) : 1.f;
-      float c0[8];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) c0[i] = 0.f;
-      for (int kc = 0; kc < pl.t_nk; ++kc) {
-        const int n = pl.t_base + (kc < pl.t_rem ? 1 : 0), p0 = kc * pl.t_base + min(kc, pl.t_rem);
-        uint32_t off;
-        if (!wait((uint32_t)(rg * n * PB), off)) bad = true;
-        if (active && !bad) {
-          const int pa = (part * n) >> lw, pb = ((part + 1) * n) >> lw;
-          const WT* wr = reinterpret_cast<const WT*>(ring + off + (size_t)r * n * PB) + lane;
-          const uint4* x = xv + (size_t)p0 * 32;
-#pragma unroll 4
-          for (int q = pa; q < pb; ++q) dot_piece(wr[q * 32], x[q * 32], c0);
-        }
-        release();
-      }
-      if (active) {
-        const float s = dev::warp_sum(sum8(c0)) * s_r;
-        if (lane == 0) {
-          if (lw == 0) rowacc[tb + r] = s;
-          else sm_part(p)[warp] = s;
-        }
-      }
+    }
+  }
+
+  // GEMV of this CTA's rows of stage st: dot products (times the rows'
+  // scales when the stream is fp8), read back with row_result.  Ring
+  // positions are held in registers for the whole stage; one barrier at the
+  // end.  W8: pieces of fp8 E4M3 weights (8 bytes a lane), converted to fp16
+  // pairs and multiplied like fp16 weights; rsc: the row scales of this
+  // CTA's rows of the stage (unused for fp16).
+  template <bool W8>
+  __device__ __noinline__ bool gemv(int st, const float* rsc) {
+    const StagePlan pl = sm_plan(kie_p)[st];
+    uint32_t ci = kie_cur[0], ce = kie_cur[2];
+    bool bad = false;
+    switch (pl.nr) {
+      case 1: gemv_units<W8, 1>(pl, rsc, ci, ce, bad); break;
+      case 2: gemv_units<W8, 2>(pl, rsc, ci, ce, bad); break;
+      case 3: gemv_units<W8, 3>(pl, rsc, ci, ce, bad); break;
+      default: gemv_units<W8, 4>(pl, rsc, ci, ce, bad); break;
     }
     const bool any_bad = dev::consumer_sync_or(bad);
     if (threadIdx.x == 0) {
+      // every chunk of the stage was released by the warp that computed it
       kie_cur[0] = ci;
-      kie_cur[1] = cr;
+      kie_cur[1] = ci;
       kie_cur[2] = ce;
     }
     return !any_bad;
@@ -1238,17 +1165,14 @@ struct Consumer {
     return gemv<true>(st, kie_wsc + (st == ST_LM ? 0 : (size_t)layer * pl.rows_layer) + pl.sbase);
   }
 
-  // Raw dot product of row k (0-based within the CTA's rows) of the last gemv.
+  // Raw dot product of row k (0-based within the CTA's rows) of the last
+  // gemv: the row's sum, or its parts' sums added in part order.
   __device__ __forceinline__ float row_result(const StagePlan& pl, int k) const {
-    const MonoParams& p = kie_p;
-    const int tb = pl.nfull * kGroupRows;
-    if (pl.tail > 0 && pl.t_lw > 0 && k >= tb) {
-      const int base = (k - tb) << pl.t_lw;
-      float s = 0.f;
-      for (int q = 0; q < (1 << pl.t_lw); ++q) s += sm_part(p)[base + q];
-      return s;
-    }
-    return sm_rowacc(p)[k];
+    const float* a = sm_rowacc(kie_p);
+    if (pl.S == 1) return a[k];
+    float s = 0.f;
+    for (int q = 0; q < pl.S; ++q) s += a[k * pl.S + q];
+    return s;
   }
 
   __device__ __forceinline__ void put(u64* dst, unsigned tag, float v, bool skip) {
@@ -2002,16 +1926,15 @@ struct Consumer {
   }
 
   // Walks a stage's chunk sequence without computing (stream-only timing).
-  __device__ __noinline__ bool skip_stage(int st, int ub, int ue) {
+  __device__ __noinline__ bool skip_stage(int st) {
     const MonoParams& p = kie_p;
-    const int R = range_rows(p, st, ub, ue);
-    const int kp = stage_k(p, st) / kPieceElems;
+    const StagePlan pl = sm_plan(p)[st];
     bool bad = false;
     uint32_t ci = kie_cur[0], cr = kie_cur[1], ce = kie_cur[2];
     const int pb = piece_bytes(p.w8);
-    for_each_chunk(R, kp, p.chunk_bytes, pb, [&](int, int rg, int n, int) {
+    for_each_unit(pl, [&](int, int, int, int rows, int n) {
       uint32_t off;
-      if (!wait_chunk((uint32_t)(rg * n * pb), off, ci, ce)) bad = true;
+      if (!wait_chunk((uint32_t)(rows * n * pb), off, ci, ce)) bad = true;
       release_chunk(cr);
       return true;
     });
@@ -2029,7 +1952,6 @@ struct Consumer {
   __device__ void gemv_bench(int mode, const float* x, float* y, int iters) {
     const MonoParams& p = kie_p;
     const int tid = (int)threadIdx.x;
-    make_plans();
     const int2 r = p.ranges[ST_LM * p.grid + blockIdx.x];
     const int K = p.d;
     float acc = 0.f;
@@ -2041,7 +1963,7 @@ struct Consumer {
     bool ok = true;
     for (int it = 0; it < iters && ok; ++it) {
       dev::consumer_sync();   // the ring cursors thread 0 wrote back are visible
-      ok = mode == 0 ? skip_stage(ST_LM, r.x, r.y) : gemv_stage(ST_LM, 0);
+      ok = mode == 0 ? skip_stage(ST_LM) : gemv_stage(ST_LM, 0);
     }
     if (ok && mode == 1)
       for (int u = r.x + tid; u < r.y; u += kConsumerThreads) y[u] = row_result(sm_plan(p)[ST_LM], u - r.x);
@@ -2056,7 +1978,6 @@ struct Consumer {
   __device__ void run() {
     const MonoParams& p = kie_p;
     const int tid = (int)threadIdx.x;
-    make_plans();
     dev::consumer_sync();
     const long long c_begin = clock64();
     int tok = p.forced ? p.forced[0] : p.first_tok;
@@ -2137,6 +2058,7 @@ __device__ __forceinline__ void kernel_setup(const MonoParams& p) {
     kie_at[0] = kie_at[1] = kie_at[2] = 0;
     dev::mbar_fence_init();
   }
+  setup_plans(p);
   __syncthreads();
 }
 

@@ -161,15 +161,16 @@ kie_status kie_gemv_f16_noalloc(const void* W, const float* x, float* y, int32_t
 
     kie::SmemLayout L{};
     L.xs_bytes = (K * 4 + 127) / 128 * 128;
-    L.rowacc_rows = maxrows;
+    L.rowacc_rows = kie::result_slots(maxrows, K / kie::kPieceElems, kChunkBytes);
     L.resid_rows = 0;
-    const int rowacc_bytes = (maxrows * 4 + 127) / 128 * 128;
-    const int fixed = 256 + L.xs_bytes + rowacc_bytes + kie::kEngineMisc;
+    const int rowacc_bytes = (L.rowacc_rows * 4 + 127) / 128 * 128;
+    const int bars = 2 * kie::kRingBars * 8;
+    const int fixed = bars + L.xs_bytes + rowacc_bytes + kie::kEngineMisc;
     const int ring = (smem_optin - fixed) / 512 * 512;
     if (ring < 2 * kChunkBytes) return KIE_ERR_UNSUPPORTED;
     L.ring_off = 0;
     L.bar_off = ring;
-    L.xs_off = L.bar_off + 256;
+    L.xs_off = L.bar_off + bars;
     L.rowacc_off = L.xs_off + L.xs_bytes;
     L.misc_off = L.rowacc_off + rowacc_bytes;
     L.total = L.misc_off + kie::kEngineMisc;

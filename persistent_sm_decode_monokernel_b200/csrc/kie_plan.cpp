@@ -94,35 +94,44 @@ int attn_smem_bytes(int G, int hd) {
 
 static int align_up(int x, int a) { return (x + a - 1) / a * a; }
 
+int result_slots(int rows, int kp, int chunk_bytes) {
+  const int per_chunk = std::max(1, chunk_bytes / kPieceBytes);
+  const int parts = (kp + per_chunk - 1) / per_chunk;
+  return std::max(256, rows * parts);
+}
+
 bool plan_smem(const Shape& s, int grid, int chunk_bytes, int smem_limit,
                const std::vector<std::vector<int2>>& ranges, SmemLayout* out, int* ring_bytes) {
   const int G = s.H / s.KV;
   const int kmax = std::max(std::max(s.d, s.H * s.hd), s.F);
   SmemLayout L{};
-  int maxrows = 0;
+  int maxrows = 0, slots = 0;
   for (int st = 0; st < N_STAGES; ++st)
-    for (int c = 0; c < grid; ++c)
-      maxrows = std::max(maxrows, rows_in_range(s, st, ranges[st][c].x, ranges[st][c].y));
+    for (int c = 0; c < grid; ++c) {
+      const int rows = rows_in_range(s, st, ranges[st][c].x, ranges[st][c].y);
+      maxrows = std::max(maxrows, rows);
+      slots = std::max(slots, result_slots(rows, stage_k(s, st) / kPieceElems, chunk_bytes));
+    }
   // fp16 input vector; the area also holds the attention scratch and the
   // top-k / top-p selection of the LM-head pick
   L.xs_bytes = align_up(std::max(std::max(kmax * 2, attn_smem_bytes(G, s.hd)),
                                  filter_smem_bytes(maxrows, grid)),
                         128);
-  L.rowacc_rows = maxrows;
+  L.rowacc_rows = slots;
   int maxres = 0;
   for (int c = 0; c < grid; ++c)
     maxres = std::max(maxres, rows_in_range(s, ST_O, ranges[ST_O][c].x, ranges[ST_O][c].y));
   L.resid_rows = maxres;
   const int bars = 2 * kRingBars * 8;
   const int misc = align_up(kMiscHead * 4 + 2 * maxres * 4 + N_STAGES * 64, 128);  // + stage plans
-  const int fixed = align_up(bars, 128) + L.xs_bytes + align_up(maxrows * 4, 128) + misc;
+  const int fixed = align_up(bars, 128) + L.xs_bytes + align_up(slots * 4, 128) + misc;
   const int ring = (smem_limit - fixed) / 512 * 512;
   if (ring < 2 * chunk_bytes) return false;
   L.ring_off = 0;
   L.bar_off = ring;
   L.xs_off = L.bar_off + align_up(bars, 128);
   L.rowacc_off = L.xs_off + L.xs_bytes;
-  L.misc_off = L.rowacc_off + align_up(maxrows * 4, 128);
+  L.misc_off = L.rowacc_off + align_up(slots * 4, 128);
   L.total = L.misc_off + misc;
   *out = L;
   *ring_bytes = ring;

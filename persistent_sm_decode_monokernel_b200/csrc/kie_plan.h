@@ -32,6 +32,12 @@ std::vector<int2> partition(const Shape& s, int grid, int stage);
 // Attention shared-memory bytes for group size G and head_dim hd.
 int attn_smem_bytes(int G, int hd);
 
+// GEMV result words a CTA with `rows` rows of `kp` pieces needs: one per
+// row, and one per row and part when chunks of `chunk_bytes` hold less than
+// a row (a row then spans several work units); at least 256, so that the
+// kernel's unit planner may split the rows of small shares into parts.
+int result_slots(int rows, int kp, int chunk_bytes);
+
 // Shared memory carve-up: fixed regions first, the rest (rounded down to
 // 512 B) is the weight ring.  Returns false if the ring would be smaller
 // than two chunks of `chunk_bytes`.
