@@ -75,6 +75,9 @@ __shared__ uint32_t kie_cur[3];
 // only: exact for thread 0 (the stage trace), and for the other threads the
 // position an error report names (possibly one stage behind).
 __shared__ int kie_at[3];
+// Ring read position after the last GEMV unit of a stage (written by the
+// warp that computed that unit, read by thread 0 after the stage's barrier).
+__shared__ uint32_t kie_ring_end;
 // This CTA's row scales of an fp8 weight stream (set by setup_plans).
 __shared__ const float* kie_wsc;
 
@@ -107,7 +110,14 @@ __device__ __forceinline__ volatile int* sm_flags(const MonoParams& p) {
 __device__ __forceinline__ uint32_t* sm_starts(const MonoParams& p) {
   return reinterpret_cast<uint32_t*>(sm_misc(p) + 96);
 }
-static_assert(kConsumerWarps <= 16 && 96 + kRingBars <= kMiscHead, "scratch words");
+// ring offset of the chunk on each barrier pair, written by the producer
+// before it arms the chunk's full barrier, so that a consumer that waited
+// for the chunk reads it without following the placement of the chunks
+// before it
+__device__ __forceinline__ volatile uint32_t* sm_offs(const MonoParams& p) {
+  return reinterpret_cast<volatile uint32_t*>(sm_misc(p) + 96 + kRingBars);
+}
+static_assert(kConsumerWarps <= 16 && 96 + 2 * kRingBars <= kMiscHead, "scratch words");
 // residual stream rows this CTA owns (O / down stages)
 __device__ __forceinline__ float* sm_res_attn(const MonoParams& p) { return sm_misc(p) + kMiscHead; }
 __device__ __forceinline__ float* sm_res_ffn(const MonoParams& p) {
@@ -475,6 +485,7 @@ struct Producer {
     if (!acquire(start + sz)) return false;
     const uint32_t b = idx & (kRingBars - 1);
     const uint32_t full = sm_full_s(p) + 8 * b;
+    sm_offs(p)[b] = off;
     dev::mbar_arrive_expect_tx(full, sz);
     dev::bulk_g2s(sm_ring_s(p) + off, src, sz, full, pol);
     sm_starts(p)[b] = start;
@@ -1062,16 +1073,18 @@ struct Consumer {
   }
 
   // This warp's units of a stage whose blocks have NR rows (see StagePlan):
-  // every warp walks all units in stream order to follow the ring placement
-  // and computes its own, unit u belonging to warp u % kConsumerWarps.  For
-  // a unit it waits for the chunk, multiplies the rows' pieces by the
-  // activation pieces (one activation load serves all rows of the unit),
-  // releases the chunk with one arrival worth all consumer warps, reduces
-  // the rows across the lanes and writes each row's sum (part s of the row
-  // when the rows are split in parts) times the row's scale.
+  // unit u belongs to warp u % kConsumerWarps and is the stage's chunk
+  // ci0 + u.  For each of its units the warp waits for the chunk, reads its
+  // ring offset (published by the producer before it armed the chunk's
+  // barrier), multiplies the rows' pieces by the activation pieces (one
+  // activation load serves all rows of the unit), releases the chunk with
+  // one arrival worth all consumer warps, reduces the rows across the lanes
+  // and writes each row's sum (part s of the row when the rows are split in
+  // parts) times the row's scale.  The owner of the last unit records the
+  // ring position after it.
   template <bool W8, int NR>
-  __device__ __forceinline__ void gemv_units(const StagePlan& pl, const float* rsc, uint32_t& ci,
-                                             uint32_t& ce, bool& bad) {
+  __device__ __forceinline__ void gemv_units(const StagePlan& pl, const float* rsc, uint32_t ci0,
+                                             bool& bad) {
     using WT = typename std::conditional<W8, uint2, uint4>::type;   // a lane's weights of a piece
     constexpr int PB = W8 ? kPieceElems : kPieceBytes;
     constexpr int kLanesPerRow = NR == 1 ? 32 : (NR == 2 ? 16 : 8);
@@ -1080,79 +1093,82 @@ struct Consumer {
     const unsigned char* ring = sm_ring(p);
     const uint4* xv = reinterpret_cast<const uint4*>(kie_smem + p.sm.xs_off) + lane;
     float* rowacc = sm_rowacc(p);
-    const uint32_t ring_bytes = (uint32_t)p.ring_bytes;
     const uint32_t full_s = sm_full_s(p), empty_s = sm_empty_s(p);
+    const volatile uint32_t* offs = sm_offs(p);
     const int my_i = lane / kLanesPerRow;          // the unit row whose sum this lane writes
     const bool writer = (lane & (kLanesPerRow - 1)) == 0;
-    const int S = pl.S;
-    int u = 0;
+    const int S = pl.S, nu = pl.nb * S;
+    int b = warp / S, s = warp - (warp / S) * S;   // block and part of unit u
 #pragma unroll 1
-    for (int b = 0; b < pl.nb; ++b) {
-      const int rows = pl.block_rows(b);
-#pragma unroll 1
-      for (int s = 0; s < S; ++s, ++u) {
-        const int n = pl.count(s);
-        const uint32_t off = ring_place(ce, (uint32_t)(rows * n * PB), ring_bytes);
-        const uint32_t chunk = ci++;
-        if ((u & (kConsumerWarps - 1)) != warp) continue;
-        const int k = b * NR + my_i;
-        const bool mine = writer && my_i < rows;
-        const float sc = (W8 && mine) ? __ldg(rsc + k) : 1.f;
-        const uint32_t bar = full_s + 8 * (chunk & (kRingBars - 1));
-        const uint32_t par = (chunk / kRingBars) & 1u;
-        if (!dev::mbar_test_wait(bar, par) && !wait_slow(bar, par)) bad = true;
-        float c[NR][8];
+    for (int u = warp; u < nu; u += kConsumerWarps) {
+      const int rows = pl.block_rows(b), n = pl.count(s);
+      const uint32_t chunk = ci0 + (uint32_t)u;
+      const int k = b * NR + my_i;
+      const bool mine = writer && my_i < rows;
+      const float sc = (W8 && mine) ? __ldg(rsc + k) : 1.f;
+      const uint32_t bar = full_s + 8 * (chunk & (kRingBars - 1));
+      const uint32_t par = (chunk / kRingBars) & 1u;
+      if (!dev::mbar_test_wait(bar, par) && !wait_slow(bar, par)) bad = true;
+      const uint32_t off = offs[chunk & (kRingBars - 1)];
+      if (u == nu - 1 && lane == 0) kie_ring_end = off + (uint32_t)(rows * n * PB);
+      float c[NR][8];
+#pragma unroll
+      for (int i = 0; i < NR; ++i)
+#pragma unroll
+        for (int j = 0; j < 8; ++j) c[i][j] = 0.f;
+      if (!bad) {
+        // rows past the end of a short last block read the block's last
+        // row again (their sums are not written), so that every load is
+        // unconditional
+        const WT* w[NR];
 #pragma unroll
         for (int i = 0; i < NR; ++i)
-#pragma unroll
-          for (int j = 0; j < 8; ++j) c[i][j] = 0.f;
-        if (!bad) {
-          // rows past the end of a short last block read the block's last
-          // row again (their sums are not written), so that every load is
-          // unconditional
-          const WT* w[NR];
-#pragma unroll
-          for (int i = 0; i < NR; ++i)
-            w[i] = reinterpret_cast<const WT*>(ring + off) + (size_t)min(i, rows - 1) * n * 32 + lane;
-          const uint4* x = xv + (size_t)pl.first(s) * 32;
+          w[i] = reinterpret_cast<const WT*>(ring + off) + (size_t)min(i, rows - 1) * n * 32 + lane;
+        const uint4* x = xv + (size_t)pl.first(s) * 32;
 #pragma unroll 2
-          for (int q = 0; q < n; ++q) {
-            const uint4 a = x[q * 32];
+        for (int q = 0; q < n; ++q) {
+          const uint4 a = x[q * 32];
 #pragma unroll
-            for (int i = 0; i < NR; ++i) dot_piece(w[i][q * 32], a, c[i]);
-          }
+          for (int i = 0; i < NR; ++i) dot_piece(w[i][q * 32], a, c[i]);
         }
-        __syncwarp();
-        if (lane == 0) dev::mbar_arrive_n(empty_s + 8 * (chunk & (kRingBars - 1)), kConsumerWarps);
-        const float t = reduce_rows<NR>(c, lane);
-        if (mine) rowacc[S == 1 ? k : k * S + s] = t * sc;
+      }
+      __syncwarp();
+      if (lane == 0) dev::mbar_arrive_n(empty_s + 8 * (chunk & (kRingBars - 1)), kConsumerWarps);
+      const float t = reduce_rows<NR>(c, lane);
+      if (mine) rowacc[S == 1 ? k : k * S + s] = t * sc;
+      // the unit kConsumerWarps further on
+      s += kConsumerWarps;
+      while (s >= S) {
+        s -= S;
+        ++b;
       }
     }
   }
 
   // GEMV of this CTA's rows of stage st: dot products (times the rows'
-  // scales when the stream is fp8), read back with row_result.  Ring
-  // positions are held in registers for the whole stage; one barrier at the
-  // end.  W8: pieces of fp8 E4M3 weights (8 bytes a lane), converted to fp16
+  // scales when the stream is fp8), read back with row_result.  The stage's
+  // chunks are the next nb * S of the ring; one barrier at the end, after
+  // which thread 0 moves the ring cursors past them.  W8: pieces of fp8 E4M3 weights (8 bytes a lane), converted to fp16
   // pairs and multiplied like fp16 weights; rsc: the row scales of this
   // CTA's rows of the stage (unused for fp16).
   template <bool W8>
   __device__ __noinline__ bool gemv(int st, const float* rsc) {
     const StagePlan pl = sm_plan(kie_p)[st];
-    uint32_t ci = kie_cur[0], ce = kie_cur[2];
+    const uint32_t ci0 = kie_cur[0];
     bool bad = false;
     switch (pl.nr) {
-      case 1: gemv_units<W8, 1>(pl, rsc, ci, ce, bad); break;
-      case 2: gemv_units<W8, 2>(pl, rsc, ci, ce, bad); break;
-      case 3: gemv_units<W8, 3>(pl, rsc, ci, ce, bad); break;
-      default: gemv_units<W8, 4>(pl, rsc, ci, ce, bad); break;
+      case 1: gemv_units<W8, 1>(pl, rsc, ci0, bad); break;
+      case 2: gemv_units<W8, 2>(pl, rsc, ci0, bad); break;
+      case 3: gemv_units<W8, 3>(pl, rsc, ci0, bad); break;
+      default: gemv_units<W8, 4>(pl, rsc, ci0, bad); break;
     }
     const bool any_bad = dev::consumer_sync_or(bad);
-    if (threadIdx.x == 0) {
+    if (threadIdx.x == 0 && pl.nb > 0) {
       // every chunk of the stage was released by the warp that computed it
+      const uint32_t ci = ci0 + (uint32_t)(pl.nb * pl.S);
       kie_cur[0] = ci;
       kie_cur[1] = ci;
-      kie_cur[2] = ce;
+      kie_cur[2] = kie_ring_end;
     }
     return !any_bad;
   }
