@@ -34,7 +34,7 @@ constexpr int kPieceBytes = kPieceElems * 2;   // an fp16 piece (16 bytes a lane
 // Bytes of a piece in the packed stream: fp16 weights, or fp8 E4M3 (8 bytes
 // a lane).
 __host__ __device__ constexpr int piece_bytes(int w8) { return w8 ? kPieceElems : kPieceBytes; }
-constexpr int kRingBars = 16;                // mbarrier pairs of the byte ring (power of 2)
+constexpr int kRingBars = 32;                // mbarrier pairs of the byte ring (power of 2)
 constexpr int kMaxGroup = 8;                 // heads per KV head handled by one CTA
 constexpr int kAttnBlock = 256;              // positions per attention block
 constexpr int kMaxSplitCombine = 96;         // most attention splits of one KV head
@@ -53,8 +53,8 @@ constexpr int kCombineBytesPerHead = 2304;
 // Shared-memory scratch words before the residual rows: per-warp partial
 // sums and reductions, flags (kMiscHead floats).  The standalone GEMV
 // engine's scratch (no residual rows) adds the per-stage GEMV plans.
-constexpr int kMiscHead = 128;
-constexpr int kEngineMisc = 896;
+constexpr int kMiscHead = 192;
+constexpr int kEngineMisc = 1152;
 // Most ids of the set that ends a decode (end-of-sequence ids).
 constexpr int kMaxEosIds = 8;
 // Top-k / top-p sampling: largest k, and how many entries of every CTA's

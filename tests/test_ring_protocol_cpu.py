@@ -9,24 +9,28 @@ chunk i occupies the monotonic range [s_i, e_i) and its ring bytes are that
 range modulo the ring size R.  The live chunks of a new chunk [s, e) lie in
 [s_oldest, s); once the oldest live chunk starts at or after e - R they all
 lie in [e - R, s), which together with [s, e) spans exactly R bytes, so none
-of them shares a ring byte with the new chunk.  Chunks are released in
-order, so the producer waits oldest first until the oldest live chunk starts
-at or after e - R and fewer than 16 chunks are live (`Producer::acquire`):
-one comparison per released chunk.  The
-consumers walk the same chunk sequence and recompute every offset
-themselves.  Random interleavings of the two sides must never let a copy
-land on bytes a consumer has not released, never reuse one of the 16
-barrier pairs while its chunk is live, and always give both sides the same
-offsets.  Two plausible slips must be caught: checking only the oldest live
-chunk for overlap in ring offsets (wrong when both the live region and the
-new chunk wrap), and comparing the oldest start against s - R instead of
+of them shares a ring byte with the new chunk.  The producer counts chunks
+as released oldest first: it waits for the oldest live chunk's release until
+that chunk starts at or after e - R and fewer than 32 chunks are live
+(`Producer::acquire`); one comparison per released chunk.  A GEMV stage's
+chunks are released out of order -- each belongs to one consumer warp
+(chunk u of the stage to warp u % 8), which computes its own chunks in
+order -- and a warp learns a chunk's offset from the table the producer
+writes (one slot per barrier pair) before it arms the chunk's barrier.
+Random interleavings of the producer and eight warps must never let a copy
+land on bytes a warp has not released, never reuse one of the 32 barrier
+pairs while its chunk is live, and always hand a warp the offset its chunk
+was copied to.  Two plausible slips must be caught: checking only the oldest
+live chunk for overlap in ring offsets (wrong when both the live region and
+the new chunk wrap), and comparing the oldest start against s - R instead of
 e - R.
 """
 import random
 
 import pytest
 
-N_BARS = 16
+N_BARS = 32
+N_WARPS = 8
 
 
 def place(wend: int, size: int, ring: int):
@@ -62,15 +66,17 @@ def producer(sizes, ring, shared, rule="monotonic"):
                 blocked = idx - cons >= N_BARS or starts[cons % N_BARS] < bound
             if not blocked:
                 break
-            while shared["consumed"] <= cons:      # wait until chunk `cons` is released
+            while cons not in shared["released"]:   # wait until chunk `cons` is released
                 yield
             cons += 1
         # the copy is issued now: it must not touch any unreleased chunk
-        for j in range(shared["consumed"], idx):
+        unreleased = [j for j in range(idx) if j not in shared["released"]]
+        for j in unreleased:
             lo, hi = shared["where"][j]
             assert not (off < hi and lo < off + size), ("overlap", idx, j)
-        assert idx - shared["consumed"] < N_BARS, "barrier pair reused while live"
+        assert not unreleased or idx - unreleased[0] < N_BARS, "barrier pair reused while live"
         shared["where"][idx] = (off, off + size)
+        shared["table"][idx % N_BARS] = off      # published before the barrier is armed
         live[idx % N_BARS] = (off, off + size)
         starts[idx % N_BARS] = s
         idx += 1
@@ -80,23 +86,26 @@ def producer(sizes, ring, shared, rule="monotonic"):
 
 def run(sizes, ring, seed, rule="monotonic"):
     rnd = random.Random(seed)
-    shared = {"consumed": 0, "issued": 0, "where": {}}
+    shared = {"released": set(), "issued": 0, "where": {}, "table": [None] * N_BARS}
     prod = producer(sizes, ring, shared, rule)
     finished = False
-    cend = 0
+    nxt = list(range(N_WARPS))          # next chunk of each warp: w, w + 8, ...
     for _ in range(10 ** 6):
-        if shared["consumed"] == len(sizes):
+        if len(shared["released"]) == len(sizes):
             return
         if not finished and rnd.random() < 0.5:
             try:
                 next(prod)
             except StopIteration:
                 finished = True
-        elif shared["consumed"] < shared["issued"]:
-            i = shared["consumed"]
-            off, cend = place(cend, sizes[i], ring)
-            assert (off, off + sizes[i]) == shared["where"][i], "consumer offset differs"
-            shared["consumed"] += 1
+        else:
+            w = rnd.randrange(N_WARPS)
+            i = nxt[w]
+            if i < shared["issued"]:
+                off = shared["table"][i % N_BARS]
+                assert (off, off + sizes[i]) == shared["where"][i], "consumer offset differs"
+                shared["released"].add(i)
+                nxt[w] += N_WARPS
     raise AssertionError("no progress")
 
 
