@@ -175,7 +175,7 @@ typedef enum {
                                   cache and everything else stay as they are.  0: fp16
                                   weights (the default).  Rebuilds the packed weight copy
                                   from the caller's matrices, which must still be valid */
-  KIE_OPT_BATCHED_PREFILL = 12  /* 1 (default): kie_prefill runs positions 0 .. n-2 of the
+  KIE_OPT_BATCHED_PREFILL = 12, /* 1 (default): kie_prefill runs positions 0 .. n-2 of the
                                   prompt through all layers at once -- the projections
                                   as tcgen05 tensor-core GEMMs over the positions, causal
                                   attention over the prompt, the K/V of every position
@@ -184,6 +184,12 @@ typedef enum {
                                   It reads the caller's fp16 weight matrices, which must
                                   then stay valid; contexts streaming FP8 weights, and
                                   0, run every position as a decode step instead */
+  KIE_OPT_TMEM_PARK = 13       /* 1 (default): while a CTA's consumer warps wait for the
+                                  other CTAs' outputs, each moves the weight chunks of the
+                                  next GEMV that have already reached its shared-memory
+                                  ring into its own 32 KB of tensor memory and frees their
+                                  ring space, so the weight stream runs further ahead
+                                  (fp16 streams only); 0: off */
 } kie_option;
 
 /* Bytes of the caller-provided KV cache: 2*n_layers*n_kv_heads*max_seq*(head_dim+8)*2.

@@ -44,6 +44,7 @@ KIE_OPT_TRACE_CLOCK = 9
 KIE_OPT_L2_PREFETCH_BYTES = 10
 KIE_OPT_WEIGHT_FP8 = 11
 KIE_OPT_BATCHED_PREFILL = 12
+KIE_OPT_TMEM_PARK = 13
 
 STAGE_QKV, STAGE_O, STAGE_GU, STAGE_DOWN, STAGE_LM = range(5)
 

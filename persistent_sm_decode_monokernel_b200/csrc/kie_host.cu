@@ -58,6 +58,7 @@ struct kie_ctx {
   // batched prefill (tensor-core GEMMs over the prompt) and its scratch,
   // grown to the longest prompt seen
   int batched_prefill = 1;
+  int tmem_park = 1;
   int pf_cap = 0;
   int* pf_ids = nullptr;
   float *pf_x = nullptr, *pf_qkv = nullptr, *pf_gu = nullptr;
@@ -240,6 +241,7 @@ kie_status launch(kie_ctx* c, int n_steps, int pos0, const int32_t* host_ids, bo
   p.timeout_ns = c->timeout_ns;
   p.poll_ns = c->poll_ns;
   p.l2_prefetch = c->l2_prefetch;
+  p.tmem_park = c->tmem_park;
   p.trace = c->trace;
   p.trace_cta = c->trace_cta;
   p.trace_steps = c->trace_steps;
@@ -977,6 +979,10 @@ kie_status kie_set_option(kie_ctx* c, kie_option opt, int64_t v) {
       case KIE_OPT_BATCHED_PREFILL:
         if (v != 0 && v != 1) return KIE_ERR_INVALID_ARG;
         c->batched_prefill = (int)v;
+        return KIE_OK;
+      case KIE_OPT_TMEM_PARK:
+        if (v != 0 && v != 1) return KIE_ERR_INVALID_ARG;
+        c->tmem_park = (int)v;
         return KIE_OK;
       case KIE_OPT_WEIGHT_FP8: {
         if (c->failed) return set_err(c, KIE_ERR_STATE, "context failed earlier; destroy it");

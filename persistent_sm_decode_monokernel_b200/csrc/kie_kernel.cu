@@ -78,6 +78,12 @@ __shared__ int kie_at[3];
 // Ring read position after the last GEMV unit of a stage (written by the
 // warp that computed that unit, read by thread 0 after the stage's barrier).
 __shared__ uint32_t kie_ring_end;
+// Tensor memory of the consumer warps (all 512 columns, allocated by warp 0
+// when parking is on) and, per warp, how many of its units of the stage
+// whose first chunk is kie_park_ci[w] it has parked there.
+__shared__ uint32_t kie_tmem;
+__shared__ int kie_park_n[kConsumerWarps];
+__shared__ uint32_t kie_park_ci[kConsumerWarps];
 // This CTA's row scales of an fp8 weight stream (set by setup_plans).
 __shared__ const float* kie_wsc;
 
@@ -304,6 +310,9 @@ __device__ __forceinline__ void setup_plans(const MonoParams& p) {
   }
   if (tid == 0) kie_wsc = p.w8 ? p.wscale + p.wscale_off[blockIdx.x] : nullptr;
 }
+
+// Whether waiting consumer warps park GEMV chunks in tensor memory.
+__device__ __forceinline__ bool parking(const MonoParams& p) { return p.tmem_park && !p.w8; }
 
 // Byte ring placement shared by producer and consumers: a chunk goes right
 // after the previous one, or back to offset 0 when it would not fit.
@@ -952,15 +961,22 @@ struct Consumer {
 
   // Loads a K-vector into xs (times `gain` if given) and returns in `ss` the
   // sum of squares of the raw values.  Source: tagged words, or an fp16
-  // embedding row.  The polls of one thread are issued in batches of up to
-  // 16 16-byte loads (one batch for K <= 8192) so that their L2 round trips
-  // overlap.  Returns false (uniformly) on abort.
+  // embedding row.  The polls of one thread are issued in batches of 8
+  // 16-byte loads (one batch for K <= 4096) so that their L2 round trips
+  // overlap.  With parking on, each warp first parks the landed chunks of
+  // stage park_st (the GEMV that reads this vector).  Returns false
+  // (uniformly) on abort.
   __device__ __noinline__ bool load_vec(const u64* src, unsigned tag, const __half* emb, int K,
-                           const __half* gain, float& ss, int where) {
+                           const __half* gain, float& ss, int where, int park_st) {
     const MonoParams& p = kie_p;
     const int tid = (int)threadIdx.x, warp = (int)(threadIdx.x >> 5), lane = (int)(threadIdx.x & 31);
     constexpr int NB = 8;
     const long long c0 = clock64();
+    if (parking(p)) {
+      // the previous stage's ring cursors are visible after this barrier
+      dev::consumer_sync();
+      park(park_st);
+    }
     float acc = 0.f;
     bool bad = false;
     const int K2 = K >> 1;
@@ -1072,6 +1088,74 @@ struct Consumer {
     }
   }
 
+  // Tensor-memory address of column 0 of warp w's parking columns: its own
+  // 32 lanes, columns kParkCols * (w / 4) onward.
+  __device__ __forceinline__ static uint32_t park_base(int w) {
+    return kie_tmem + ((uint32_t)(32 * (w & 3)) << 16) + (uint32_t)(kParkCols * (w >> 2));
+  }
+
+  // Moves this warp's next units of stage st that have already landed in
+  // the ring (in unit order, while they fit its kParkCols columns) into its
+  // tensor memory, lane l keeping its 16 bytes of every piece of every row,
+  // and releases their ring chunks, so that the producer streams further
+  // ahead while the warp waits for other CTAs.  Called after a consumer
+  // barrier that follows the previous stage (the ring cursors are current).
+  // fp16 streams only.
+  __device__ __noinline__ void park(int st) {
+    const MonoParams& p = kie_p;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const StagePlan pl = sm_plan(p)[st];
+    const uint32_t ci0 = kie_cur[0];
+    const int S = pl.S, nu = pl.nb * S;
+    const unsigned char* ring = sm_ring(p);
+    const uint32_t full_s = sm_full_s(p), empty_s = sm_empty_s(p);
+    const volatile uint32_t* offs = sm_offs(p);
+    const uint32_t tb = park_base(warp);
+    int b = warp / S, s = warp - (warp / S) * S;
+    uint32_t col = 0;
+    int parked = 0;
+#pragma unroll 1
+    for (int u = warp; u < nu; u += kConsumerWarps) {
+      const int rows = pl.block_rows(b), n = pl.count(s);
+      const int np = rows * n;   // piece rows: 16 bytes of each per lane, 4 columns
+      if (col + 4u * (uint32_t)np > (uint32_t)kParkCols) break;
+      const uint32_t chunk = ci0 + (uint32_t)u;
+      const uint32_t bar = full_s + 8 * (chunk & (kRingBars - 1));
+      // every lane must have seen the chunk land before reading it
+      if (!__all_sync(0xffffffffu, dev::mbar_test_wait(bar, (chunk / kRingBars) & 1u))) break;
+      const uint32_t off = offs[chunk & (kRingBars - 1)];
+      if (u == nu - 1 && lane == 0) kie_ring_end = off + (uint32_t)(np * kPieceBytes);
+      const uint4* src = reinterpret_cast<const uint4*>(ring + off) + lane;
+      int j = 0;
+#pragma unroll 1
+      for (; j + 4 <= np; j += 4) {
+        const uint4 v0 = src[(j + 0) * 32], v1 = src[(j + 1) * 32];
+        const uint4 v2 = src[(j + 2) * 32], v3 = src[(j + 3) * 32];
+        dev::tmem_st4(tb + col + 4 * j, v0);
+        dev::tmem_st4(tb + col + 4 * j + 4, v1);
+        dev::tmem_st4(tb + col + 4 * j + 8, v2);
+        dev::tmem_st4(tb + col + 4 * j + 12, v3);
+      }
+#pragma unroll 1
+      for (; j < np; ++j) dev::tmem_st4(tb + col + 4 * j, src[j * 32]);
+      dev::tmem_wait_st();
+      __syncwarp();
+      if (lane == 0) dev::mbar_arrive_n(empty_s + 8 * (chunk & (kRingBars - 1)), kConsumerWarps);
+      col += 4u * (uint32_t)np;
+      ++parked;
+      s += kConsumerWarps;
+      while (s >= S) {
+        s -= S;
+        ++b;
+      }
+    }
+    if (lane == 0) {
+      kie_park_n[warp] = parked;
+      kie_park_ci[warp] = ci0;
+    }
+    __syncwarp();
+  }
+
   // This warp's units of a stage whose blocks have NR rows (see StagePlan):
   // unit u belongs to warp u % kConsumerWarps and is the stage's chunk
   // ci0 + u.  For each of its units the warp waits for the chunk, reads its
@@ -1099,23 +1183,58 @@ struct Consumer {
     const bool writer = (lane & (kLanesPerRow - 1)) == 0;
     const int S = pl.S, nu = pl.nb * S;
     int b = warp / S, s = warp - (warp / S) * S;   // block and part of unit u
+    // this warp's first units of the stage may be parked in tensor memory
+    const int npark = (!W8 && kie_park_ci[warp] == ci0) ? kie_park_n[warp] : 0;
+    const uint32_t tb = W8 ? 0u : park_base(warp);
+    uint32_t pcol = 0;
+    int kown = 0;
 #pragma unroll 1
-    for (int u = warp; u < nu; u += kConsumerWarps) {
+    for (int u = warp; u < nu; u += kConsumerWarps, ++kown) {
       const int rows = pl.block_rows(b), n = pl.count(s);
       const uint32_t chunk = ci0 + (uint32_t)u;
       const int k = b * NR + my_i;
       const bool mine = writer && my_i < rows;
       const float sc = (W8 && mine) ? __ldg(rsc + k) : 1.f;
-      const uint32_t bar = full_s + 8 * (chunk & (kRingBars - 1));
-      const uint32_t par = (chunk / kRingBars) & 1u;
-      if (!dev::mbar_test_wait(bar, par) && !wait_slow(bar, par)) bad = true;
-      const uint32_t off = offs[chunk & (kRingBars - 1)];
-      if (u == nu - 1 && lane == 0) kie_ring_end = off + (uint32_t)(rows * n * PB);
       float c[NR][8];
 #pragma unroll
       for (int i = 0; i < NR; ++i)
 #pragma unroll
         for (int j = 0; j < 8; ++j) c[i][j] = 0.f;
+      if constexpr (!W8) {
+        if (kown < npark) {
+          // parked: the chunk was released when it was parked; rows past
+          // the end of a short block read the block's last row again
+          if (!bad) {
+            const uint32_t rs = 4u * (uint32_t)n;   // columns per row
+            const uint32_t a0 = tb + pcol, a1 = a0 + rs * (uint32_t)min(1, rows - 1);
+            const uint32_t a2 = a0 + rs * (uint32_t)min(2, rows - 1);
+            const uint32_t a3 = a0 + rs * (uint32_t)min(3, rows - 1);
+            const uint4* x = xv + (size_t)pl.first(s) * 32;
+#pragma unroll 1
+            for (int q = 0; q < n; ++q) {
+              uint4 wv[4];
+              dev::tmem_ld4x4_wait(a0 + 4 * q, a1 + 4 * q, a2 + 4 * q, a3 + 4 * q, wv);
+              const uint4 a = x[q * 32];
+#pragma unroll
+              for (int i = 0; i < NR; ++i) dot_piece(wv[i], a, c[i]);
+            }
+          }
+          pcol += 4u * (uint32_t)(rows * n);
+          const float t = reduce_rows<NR>(c, lane);
+          if (mine) rowacc[S == 1 ? k : k * S + s] = t * sc;
+          s += kConsumerWarps;
+          while (s >= S) {
+            s -= S;
+            ++b;
+          }
+          continue;
+        }
+      }
+      const uint32_t bar = full_s + 8 * (chunk & (kRingBars - 1));
+      const uint32_t par = (chunk / kRingBars) & 1u;
+      if (!dev::mbar_test_wait(bar, par) && !wait_slow(bar, par)) bad = true;
+      const uint32_t off = offs[chunk & (kRingBars - 1)];
+      if (u == nu - 1 && lane == 0) kie_ring_end = off + (uint32_t)(rows * n * PB);
       if (!bad) {
         // rows past the end of a short last block read the block's last
         // row again (their sums are not written), so that every load is
@@ -1217,7 +1336,7 @@ struct Consumer {
       const int u = r.x + tid;
       if (u < r.y && u < np_all) cs0 = cs[(u < nqp ? u : u - nqp) % half];
     }
-    if (!load_vec(p.x_attn, tag, emb, p.d, w.attn_norm, ss, 10)) return false;
+    if (!load_vec(p.x_attn, tag, emb, p.d, w.attn_norm, ss, 10, ST_QKV)) return false;
     if (!gemv_stage(ST_QKV, layer)) return false;
     const StagePlan pl = sm_plan(p)[ST_QKV];
     const float rs = 1.0f / sqrtf(ss / (float)p.d + p.eps);
@@ -1581,7 +1700,7 @@ struct Consumer {
     const int2 r = p.ranges[ST_O * p.grid + blockIdx.x];
     if (r.y <= r.x) return true;
     float ss;
-    if (!load_vec(p.obuf, tag, nullptr, p.H * p.hd, nullptr, ss, 30)) return false;
+    if (!load_vec(p.obuf, tag, nullptr, p.H * p.hd, nullptr, ss, 30, ST_O)) return false;
     if (!gemv_stage(ST_O, layer)) return false;
     const StagePlan pl = sm_plan(p)[ST_O];
     for (int u = r.x + tid; u < r.y; u += kConsumerThreads) {
@@ -1602,7 +1721,7 @@ struct Consumer {
     const int2 r = p.ranges[ST_GU * p.grid + blockIdx.x];
     if (r.y <= r.x) return true;
     float ss;
-    if (!load_vec(p.x_ffn, tag, nullptr, p.d, w.ffn_norm, ss, 40)) return false;
+    if (!load_vec(p.x_ffn, tag, nullptr, p.d, w.ffn_norm, ss, 40, ST_GU)) return false;
     if (!gemv_stage(ST_GU, layer)) return false;
     const StagePlan pl = sm_plan(p)[ST_GU];
     const float rs = 1.0f / sqrtf(ss / (float)p.d + p.eps);
@@ -1623,7 +1742,7 @@ struct Consumer {
     const int2 r = p.ranges[ST_DOWN * p.grid + blockIdx.x];
     if (r.y <= r.x) return true;
     float ss;
-    if (!load_vec(p.hbuf, tag, nullptr, p.F, nullptr, ss, 50)) return false;
+    if (!load_vec(p.hbuf, tag, nullptr, p.F, nullptr, ss, 50, ST_DOWN)) return false;
     if (!gemv_stage(ST_DOWN, layer)) return false;
     const StagePlan pl = sm_plan(p)[ST_DOWN];
     for (int u = r.x + tid; u < r.y; u += kConsumerThreads) {
@@ -1851,7 +1970,7 @@ struct Consumer {
     const int2 r = p.ranges[ST_LM * p.grid + blockIdx.x];
     if (pick && r.y > r.x) {
       float ss;
-      if (!load_vec(p.x_attn, tag, nullptr, p.d, p.final_norm, ss, 60)) return -1;
+      if (!load_vec(p.x_attn, tag, nullptr, p.d, p.final_norm, ss, 60, ST_LM)) return -1;
       if (!gemv_stage(ST_LM, 0)) return -1;
       const StagePlan pl = sm_plan(p)[ST_LM];
       trace(2);
@@ -1994,7 +2113,11 @@ struct Consumer {
   __device__ void run() {
     const MonoParams& p = kie_p;
     const int tid = (int)threadIdx.x;
+    const bool tmem = parking(p);
+    if (tmem && (tid >> 5) == 0) dev::tmem_alloc(dev::smem_u32(&kie_tmem), 2 * kParkCols);
+    dev::tmem_fence_before_sync();
     dev::consumer_sync();
+    dev::tmem_fence_after_sync();
     const long long c_begin = clock64();
     int tok = p.forced ? p.forced[0] : p.first_tok;
     int done = 0;
@@ -2043,6 +2166,13 @@ struct Consumer {
       else tok = next;
     }
     if (tid == 0) sm_flags(p)[F_STOP] = 1;
+    if (tmem) {
+      // every warp's tensor-memory accesses are done before warp 0 frees it
+      dev::tmem_fence_before_sync();
+      dev::consumer_sync();
+      dev::tmem_fence_after_sync();
+      if ((tid >> 5) == 0) dev::tmem_dealloc(kie_tmem, 2 * kParkCols);
+    }
     if (blockIdx.x == 0 && tid == 0) p.status->n_done = done;
     if (tid == 0) {
       u64* st = p.cta_stats + kStatsPerCta * blockIdx.x;
@@ -2072,6 +2202,7 @@ __device__ __forceinline__ void kernel_setup(const MonoParams& p) {
     kie_ctr[0] = kie_ctr[1] = kie_ctr[2] = 0;
     kie_cur[0] = kie_cur[1] = kie_cur[2] = 0u;
     kie_at[0] = kie_at[1] = kie_at[2] = 0;
+    for (int w = 0; w < kConsumerWarps; ++w) kie_park_n[w] = 0;
     dev::mbar_fence_init();
   }
   setup_plans(p);

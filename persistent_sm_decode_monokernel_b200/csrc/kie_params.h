@@ -35,6 +35,10 @@ constexpr int kPieceBytes = kPieceElems * 2;   // an fp16 piece (16 bytes a lane
 // a lane).
 __host__ __device__ constexpr int piece_bytes(int w8) { return w8 ? kPieceElems : kPieceBytes; }
 constexpr int kRingBars = 32;                // mbarrier pairs of the byte ring (power of 2)
+// Tensor-memory columns (32-bit, of its own 32 lanes) each consumer warp
+// parks weight chunks in: 8 warps x 32 lanes x 256 columns = all 256 KB.
+constexpr int kParkCols = 256;
+static_assert(kConsumerWarps == 8 && kParkCols * 2 == 512, "tensor-memory split");
 constexpr int kMaxGroup = 8;                 // heads per KV head handled by one CTA
 constexpr int kAttnBlock = 256;              // positions per attention block
 constexpr int kMaxSplitCombine = 96;         // most attention splits of one KV head
@@ -141,6 +145,7 @@ struct MonoParams {
   long long timeout_ns;
   unsigned poll_ns;        // sleep between re-polls of tagged words
   long long l2_prefetch;   // weight-stream bytes kept requested into L2 ahead of the copies
+  int tmem_park;           // 1: waiting consumer warps park landed GEMV chunks in tensor memory
   unsigned long long* trace;  // stage timestamps of CTA trace_cta, or null
   int trace_cta, trace_steps;
   int trace_clock;         // 1: stamps are SM cycles (clock64), 0: %globaltimer ns

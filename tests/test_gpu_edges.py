@@ -194,6 +194,16 @@ def test_l2_prefetch_option_keeps_parity(torch_cuda):
     assert rep.compared == 13
 
 
+@pytest.mark.parametrize("park", [0, 1])
+def test_tmem_park_option_keeps_parity(torch_cuda, park):
+    # on (the default): the chunks a warp parked while it waited are read
+    # back from tensor memory; off: every chunk is read from the ring
+    from persistent_sm_decode_monokernel_b200 import _kie
+    rep = _forced_parity(synth.WORKLOADS["l16-d1024"].shape, 300, 12,
+                         options=[(_kie.KIE_OPT_TMEM_PARK, park)])
+    assert rep.compared == 13
+
+
 def test_trace_of_every_cta(tiny):
     from persistent_sm_decode_monokernel_b200 import TRACE_PER_LAYER
     w, m, dev, prompt = tiny
