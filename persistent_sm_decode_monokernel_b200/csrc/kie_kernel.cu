@@ -964,15 +964,15 @@ struct Consumer {
   // embedding row.  The polls of one thread are issued in batches of 8
   // 16-byte loads (one batch for K <= 4096) so that their L2 round trips
   // overlap.  With parking on, each warp first parks the landed chunks of
-  // stage park_st (the GEMV that reads this vector).  Returns false
-  // (uniformly) on abort.
+  // stage park_st (the GEMV that reads this vector; -1: none).  Returns
+  // false (uniformly) on abort.
   __device__ __noinline__ bool load_vec(const u64* src, unsigned tag, const __half* emb, int K,
                            const __half* gain, float& ss, int where, int park_st) {
     const MonoParams& p = kie_p;
     const int tid = (int)threadIdx.x, warp = (int)(threadIdx.x >> 5), lane = (int)(threadIdx.x & 31);
     constexpr int NB = 8;
     const long long c0 = clock64();
-    if (parking(p)) {
+    if (parking(p) && park_st >= 0) {
       // the previous stage's ring cursors are visible after this barrier
       dev::consumer_sync();
       park(park_st);
@@ -1700,7 +1700,9 @@ struct Consumer {
     const int2 r = p.ranges[ST_O * p.grid + blockIdx.x];
     if (r.y <= r.x) return true;
     float ss;
-    if (!load_vec(p.obuf, tag, nullptr, p.H * p.hd, nullptr, ss, 30, ST_O)) return false;
+    // O's chunks are not parked (measured 0.5% faster on the 2.2B model:
+    // the whole O stage fits the ring and is read right after the wait)
+    if (!load_vec(p.obuf, tag, nullptr, p.H * p.hd, nullptr, ss, 30, -1)) return false;
     if (!gemv_stage(ST_O, layer)) return false;
     const StagePlan pl = sm_plan(p)[ST_O];
     for (int u = r.x + tid; u < r.y; u += kConsumerThreads) {
