@@ -374,8 +374,8 @@ KIE_API kie_status kie_quantize_e4m3(const void *W, int32_t N, int32_t K, void *
  * no device memory.
  *
  * The first call on a device looks up the array's address on that device
- * (cudaGetSymbolAddress, which may load the library's device code there);
- * make that first call before any stream capture.  The address belongs to
+ * (cudaGetSymbolAddress, which may load the library's device code there,
+ * so the first call takes longer than the ones after it).  The address belongs to
  * the device's current driver context: after cudaDeviceReset, or with
  * another context made current, the next call looks it up again (so that
  * call is again a first call).  Another host thread's kie_gemv_f16 does not
