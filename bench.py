@@ -54,7 +54,7 @@ def _peaks():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-KERNEL_SOURCES = ["kie_kernel.cu", "kie_device.cuh", "kie_params.h"]
+KERNEL_SOURCES = ["kie_kernel.cu", "kie_device.cuh", "kie_params.h", "kie_units.h"]
 
 
 def kernel_sha() -> str:

@@ -132,10 +132,11 @@ typedef struct {
   int32_t last_steps;       /* forward passes run by the last launch */
   float last_device_ms;     /* device time of the last launch (CUDA events) */
   uint64_t launches;        /* kernel launches made by this context */
-  /* Per-CTA cycle counters of the last launch, averaged over CTAs:
-   * consumer-side cycles in the persistent loop, cycles spent polling for
-   * other CTAs' outputs (the intra-kernel sync), and cycles spent waiting
-   * for the weight stream to land in shared memory. */
+  /* Per-CTA cycle counters of the last launch, averaged over CTAs, as seen
+   * by consumer thread 0: cycles in the persistent loop, cycles spent
+   * polling for other CTAs' outputs (the intra-kernel sync), and cycles
+   * spent waiting for the weight stream to land in shared memory (for the
+   * GEMV units warp 0 computes itself: each unit belongs to one warp). */
   double loop_cycles;
   double sync_wait_cycles;
   double stream_wait_cycles;
@@ -147,7 +148,8 @@ typedef struct {
 
 typedef enum {
   KIE_OPT_TIMEOUT_NS = 1,     /* bound of every device-side wait (default 2e9) */
-  KIE_OPT_CHUNK_BYTES = 2,    /* largest weight chunk in bytes (>= 8192, multiple of 512;
+  KIE_OPT_CHUNK_BYTES = 2,    /* largest weight chunk -- one GEMV work unit, one bulk
+                                 copy -- in bytes (>= 8192, multiple of 512;
                                  default 32768, or 16384 where two 32 KB chunks do not
                                  fit the ring); re-plans the ring and rebuilds the packed
                                  weight copy, so the caller's matrices must still be valid */
@@ -395,6 +397,19 @@ KIE_API kie_status kie_gemv_f16_noalloc(const void *W, const float *x, float *y,
  * rows and gate/up row pairs, which count as one unit of two rows. */
 KIE_API kie_status kie_plan_units(const kie_model_desc *desc, int32_t grid, int32_t stage,
                           int32_t cta, int32_t *begin, int32_t *end);
+
+/* Host-only planning query (no CUDA call): how CTA `cta` of a `grid`-CTA
+ * decode launch splits its GEMV work in stage `stage` for KIE_OPT_CHUNK_BYTES
+ * = chunk_bytes (>= 8192, multiple of 512) and fp16 (fp8 = 0) or FP8 (1)
+ * weights -- the same computation the decode kernel and its weight repack
+ * make.  The CTA's rows are cut into blocks of nr <= 4 rows and each row's
+ * 256-weight pieces into S parts; a block's part is one work unit (one bulk
+ * copy, computed by one consumer warp).  out[6] (caller-owned) receives
+ * {rows, pieces per row, nr, S, blocks, result slots reserved per CTA}.
+ * Errors: KIE_ERR_INVALID_ARG, or the descriptor checks of kie_check_desc. */
+KIE_API kie_status kie_plan_gemv_work(const kie_model_desc *desc, int32_t grid, int32_t stage,
+                                      int32_t cta, int32_t chunk_bytes, int32_t fp8,
+                                      int32_t *out);
 
 #ifdef __cplusplus
 }

@@ -104,6 +104,7 @@ SIGNATURES = {
     "kie_last_error": (ctypes.c_char_p, [_P]),
     "kie_destroy": (ctypes.c_int, [_P]),
     "kie_plan_units": (ctypes.c_int, [_PDESC, _I32, _I32, _I32, _PI32, _PI32]),
+    "kie_plan_gemv_work": (ctypes.c_int, [_PDESC, _I32, _I32, _I32, _I32, _I32, _PI32]),
     "kie_gemv_f16": (ctypes.c_int, [_P, _P, _P, _I32, _I32, _I32, _I32, _I32, _P,
                                     ctypes.POINTER(ctypes.c_float),
                                     ctypes.POINTER(ctypes.c_double)]),
@@ -170,6 +171,16 @@ def kie_plan_units(desc: KieModelDesc, grid: int, stage: int, cta: int):
     _check(load_library().kie_plan_units(ctypes.byref(desc), grid, stage, cta,
                                          ctypes.byref(b), ctypes.byref(e)), "kie_plan_units")
     return b.value, e.value
+
+
+def kie_plan_gemv_work(desc: KieModelDesc, grid: int, stage: int, cta: int,
+                       chunk_bytes: int = 32768, fp8: int = 0):
+    """(rows, pieces per row, rows per block, parts per row, blocks, result
+    slots) of CTA `cta`'s GEMV work in `stage` (see kie.h)."""
+    out = (ctypes.c_int32 * 6)()
+    _check(load_library().kie_plan_gemv_work(ctypes.byref(desc), grid, stage, cta, chunk_bytes,
+                                             fp8, out), "kie_plan_gemv_work")
+    return tuple(int(v) for v in out)
 
 
 LAYER_NAMES = ("attn_norm", "wq", "wk", "wv", "wo", "ffn_norm", "w_gate", "w_up", "w_down")

@@ -19,7 +19,8 @@ INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(HERE, "libkie.so")
 
 SOURCES = ["kie_host.cu", "kie_kernel.cu", "kie_plan.cpp", "kie_noalloc.cu", "kie_prefill.cu"]
-HEADERS = ["kie_params.h", "kie_plan.h", "kie_kernel.h", "kie_device.cuh", "kie_prefill.h"]
+HEADERS = ["kie_params.h", "kie_plan.h", "kie_kernel.h", "kie_device.cuh", "kie_prefill.h",
+           "kie_units.h"]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",

@@ -17,6 +17,7 @@
 #include "kie_params.h"
 #include "kie_plan.h"
 #include "kie_prefill.h"
+#include "kie_units.h"
 
 using kie::DevStatus;
 using kie::LayerW;
@@ -483,6 +484,33 @@ kie_status kie_plan_units(const kie_model_desc* d, int32_t grid, int32_t stage, 
     const auto r = kie::partition(shape_of(*d), grid, stage);
     *begin = r[cta].x;
     *end = r[cta].y;
+    return KIE_OK;
+  });
+}
+
+kie_status kie_plan_gemv_work(const kie_model_desc* d, int32_t grid, int32_t stage, int32_t cta,
+                              int32_t chunk_bytes, int32_t fp8, int32_t* out) {
+  return kie::no_throw([&]() -> kie_status {
+    if (!d || !out) return KIE_ERR_INVALID_ARG;
+    kie_status s = kie_check_desc(d);
+    if (s != KIE_OK) return s;
+    if (grid < 1 || stage < 0 || stage >= kie::N_STAGES || cta < 0 || cta >= grid ||
+        chunk_bytes < 8192 || chunk_bytes % 512 || chunk_bytes > (1 << 20) || (fp8 != 0 && fp8 != 1))
+      return KIE_ERR_INVALID_ARG;
+    const kie::Shape sh = shape_of(*d);
+    std::vector<std::vector<int2>> ranges(kie::N_STAGES);
+    for (int st = 0; st < kie::N_STAGES; ++st) ranges[st] = kie::partition(sh, grid, st);
+    kie::StagePlan pl{};
+    pl.rows = kie::rows_in_range(sh, stage, ranges[stage][cta].x, ranges[stage][cta].y);
+    pl.kp = kie::stage_k(sh, stage) / kie::kPieceElems;
+    const int slots = kie::gemv_slots(sh, ranges, grid, chunk_bytes);
+    kie::plan_units(pl, chunk_bytes, kie::piece_bytes(fp8), slots);
+    out[0] = pl.rows;
+    out[1] = pl.kp;
+    out[2] = pl.nr;
+    out[3] = pl.S;
+    out[4] = pl.nb;
+    out[5] = slots;
     return KIE_OK;
   });
 }

@@ -100,18 +100,26 @@ int result_slots(int rows, int kp, int chunk_bytes) {
   return std::max(256, rows * parts);
 }
 
+int gemv_slots(const Shape& s, const std::vector<std::vector<int2>>& ranges, int grid,
+               int chunk_bytes) {
+  int slots = 0;
+  for (int st = 0; st < N_STAGES; ++st)
+    for (int c = 0; c < grid; ++c)
+      slots = std::max(slots, result_slots(rows_in_range(s, st, ranges[st][c].x, ranges[st][c].y),
+                                           stage_k(s, st) / kPieceElems, chunk_bytes));
+  return slots;
+}
+
 bool plan_smem(const Shape& s, int grid, int chunk_bytes, int smem_limit,
                const std::vector<std::vector<int2>>& ranges, SmemLayout* out, int* ring_bytes) {
   const int G = s.H / s.KV;
   const int kmax = std::max(std::max(s.d, s.H * s.hd), s.F);
   SmemLayout L{};
-  int maxrows = 0, slots = 0;
+  int maxrows = 0;
   for (int st = 0; st < N_STAGES; ++st)
-    for (int c = 0; c < grid; ++c) {
-      const int rows = rows_in_range(s, st, ranges[st][c].x, ranges[st][c].y);
-      maxrows = std::max(maxrows, rows);
-      slots = std::max(slots, result_slots(rows, stage_k(s, st) / kPieceElems, chunk_bytes));
-    }
+    for (int c = 0; c < grid; ++c)
+      maxrows = std::max(maxrows, rows_in_range(s, st, ranges[st][c].x, ranges[st][c].y));
+  const int slots = gemv_slots(s, ranges, grid, chunk_bytes);
   // fp16 input vector; the area also holds the attention scratch and the
   // top-k / top-p selection of the LM-head pick
   L.xs_bytes = align_up(std::max(std::max(kmax * 2, attn_smem_bytes(G, s.hd)),

@@ -37,6 +37,10 @@ int attn_smem_bytes(int G, int hd);
 // a row (a row then spans several work units); at least 256, so that the
 // kernel's unit planner may split the rows of small shares into parts.
 int result_slots(int rows, int kp, int chunk_bytes);
+// The result words every CTA of the plan reserves: result_slots of the
+// largest need over all stages and CTAs.
+int gemv_slots(const Shape& s, const std::vector<std::vector<int2>>& ranges, int grid,
+               int chunk_bytes);
 
 // Shared memory carve-up: fixed regions first, the rest (rounded down to
 // 512 B) is the weight ring.  Returns false if the ring would be smaller
