@@ -99,9 +99,8 @@ __device__ __forceinline__ float* sm_rowacc(const MonoParams& p) {
 __device__ __forceinline__ float* sm_misc(const MonoParams& p) {
   return reinterpret_cast<float*>(kie_smem + p.sm.misc_off);
 }
-// per-warp scratch words, kConsumerWarps each (<= 16): partial sums, two
-// reductions with their indices; then flags
-__device__ __forceinline__ float* sm_part(const MonoParams& p) { return sm_misc(p); }
+// per-warp scratch words, kConsumerWarps each (<= 16; words 0-15 unused):
+// two reductions with their indices; then flags
 __device__ __forceinline__ float* sm_red(const MonoParams& p) { return sm_misc(p) + 16; }
 __device__ __forceinline__ float* sm_red2(const MonoParams& p) { return sm_misc(p) + 32; }
 __device__ __forceinline__ int* sm_redi(const MonoParams& p) {

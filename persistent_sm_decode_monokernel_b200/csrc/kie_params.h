@@ -26,9 +26,6 @@ static_assert(kConsumerWarps * kRegsConsumer + 4 * kRegsProducer <=
                   (kConsumerWarps + 4) * kRegsLaunch,
               "register split exceeds the launch's registers");
 static_assert((kConsumerWarps + 4) * 32 * kRegsLaunch <= 65536, "launch registers");
-constexpr int kGroupRows = 16;              // rows streamed together
-constexpr int kRowsPerWarp = kGroupRows / kConsumerWarps;  // rows of a full group per warp
-static_assert(kRowsPerWarp == 1 || kRowsPerWarp == 2, "group mapping");
 constexpr int kPieceElems = 256;             // one warp pass: 32 lanes x 8 weights
 constexpr int kPieceBytes = kPieceElems * 2;   // an fp16 piece (16 bytes a lane)
 // Bytes of a piece in the packed stream: fp16 weights, or fp8 E4M3 (8 bytes
